@@ -1,0 +1,483 @@
+#!/usr/bin/env python
+"""Paged decode attention benchmark on B200: KV GB/s and sequences/s.
+
+One step = one decode step of the hot path over one batch: the step's cache
+write (pa_reshape_and_cache of every sequence's new token), the partition
+kernel (pa_decode_partitions) and the log-sum-exp merge (pa_decode_reduce),
+all through the C ABI.  The default workload is the Llama-3-70B-shaped batch:
+256 sequences, 64 query / 8 kv heads, head_dim 128, bf16, 16-token pages from
+a shuffled pool, context lengths log-uniform in [512, 8192] (2.9 GB of KV per
+step, far above the 126 MB L2, so no flush is needed between steps).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torchrun) every rank decodes its own batch of the same
+shape (weak scaling, no data-path collective); the step time is the max over
+ranks.  ``--impl reference`` times the CPU oracle on a bounded sample of the
+same workload instead (rank 0 only).  Prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention KV GB/s"
+UNIT = "GB/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama70b", choices=["llama8b", "llama70b", "prefix", "beam32k"])
+    ap.add_argument("--kernel", default="auto", choices=["auto", "tc", "cc"])
+    ap.add_argument("--tiling", default="4x3", help="tensor-core kernel warps x stages")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle time budget for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------------------------
+# workload accounting
+# ---------------------------------------------------------------------------------------------
+
+def kv_bytes(w, tables, ctx):
+    """(unique, logical) KV bytes one decode step reads: shared pages counted once for unique."""
+    per_token = 2 * w.num_kv_heads * w.head_dim * w.elem_bytes
+    used = {}
+    for b in range(w.num_seqs):
+        c = int(ctx[b])
+        for i in range(-(-c // w.block_size)):
+            page = int(tables[b, i])
+            used[page] = max(used.get(page, 0), min(w.block_size, c - i * w.block_size))
+    return sum(used.values()) * per_token, int(np.sum(ctx)) * per_token
+
+
+def partition_kernel_bytes(w, ctx, unique_kv):
+    """Algorithmic bytes of one partition-kernel launch: KV + q + tables + lengths + partials / rows out."""
+    eb = w.elem_bytes
+    nparts = [-(-int(c) // 512) for c in ctx]
+    q = w.num_seqs * w.num_q_heads * w.head_dim * eb
+    tables = 4 * sum(-(-int(c) // w.block_size) for c in ctx)
+    lens = 4 * w.num_seqs
+    partials = sum(n for n in nparts if n > 1) * w.num_q_heads * (w.head_dim + 2) * 4
+    rows = sum(1 for n in nparts if n <= 1) * w.num_q_heads * w.head_dim * eb
+    return unique_kv + q + tables + lens + partials + rows
+
+
+def describe(w):
+    ctx = np.array(w.context_lens)
+    return {"workload": f"{w.name}: {w.num_seqs} seqs, {w.num_q_heads} q / {w.num_kv_heads} kv heads, head_dim "
+                        f"{w.head_dim}, {w.dtype}, block_size {w.block_size}, context {int(ctx.min())}..{int(ctx.max())} "
+                        f"(mean {ctx.mean():.0f})",
+            "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
+            "head_dim": w.head_dim, "block_size": w.block_size, "num_blocks": w.num_blocks,
+            "context_tokens": int(ctx.sum()), "partition_tokens": 512}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic(kernel_hash):
+    """DRAM bytes per launch of the partition kernel from the committed ncu summary, if still current."""
+    path = os.path.join(ROOT, "profiles", "decode_partitions_llama70b.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None, None
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip().split()[0].replace(",", "")
+    if vals.get("kernel_source_sha256") != kernel_hash or "dram_bytes_per_launch_full_size" not in vals:
+        return None, vals.get("kernel_source_sha256")
+    return int(float(vals["dram_bytes_per_launch_full_size"])), kernel_hash
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("decode.cu", "device.cuh"):
+        with open(os.path.join(ROOT, "paged_kv_cache_356_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons of one GPU while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, flag in zip(names, parts[4:8]):
+                if flag.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_smi_id(torch, device):
+    props = torch.cuda.get_device_properties(device)
+    uuid = getattr(props, "uuid", None)
+    if uuid is not None:
+        s = str(uuid)
+        return s if s.startswith("GPU-") else "GPU-" + s
+    return device
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU oracle (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------------------------
+
+class OracleSample:
+    """The oracle's decode step on a bounded sample (a prefix of the batch) of a workload.
+
+    The sample is sized so one oracle step takes about ``seconds_per_step`` on
+    this host; setup (allocator, cache writes of the prefill) is not timed.
+    """
+
+    def __init__(self, name, seconds_per_step, max_seqs=256):
+        from oracle import attention, scenario
+        from paged_kv_cache_356_b200 import workloads
+
+        try:
+            from threadpoolctl import threadpool_info
+            self.cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        except Exception:
+            self.cores = 1
+        full = workloads.by_name(name)
+        key = "num_beams" if name == "beam32k" else "num_seqs"
+        probe = workloads.by_name(name, **{key: 1})
+        res = scenario.run(probe)
+        t0 = time.perf_counter()
+        attention.decode_attention(probe.query(), res["key_cache"], res["value_cache"], res["block_tables"],
+                                   res["context_lens"], probe.scale, probe.dtype)
+        per_seq = max(time.perf_counter() - t0, 1e-3) * (np.mean(full.context_lens) / probe.context_lens[0])
+        n = int(max(1, min(max_seqs, full.num_seqs, seconds_per_step / per_seq)))
+        self.w = w = workloads.by_name(name, **{key: n})
+        self.res = res = scenario.run(w)
+        self.q = w.query()
+        step_writes = [op for op in w.trace if op[0] == "write"][-w.num_seqs:]
+        self.k_new, self.v_new = w.batched_token_kv(step_writes)
+        self.slots = res["write_slots"][-sum(op[3] for op in step_writes):]
+        self.unique, _ = kv_bytes(w, res["block_tables"], res["context_lens"])
+        self.desc = (f"first {w.num_seqs} of {full.num_seqs} sequences of the {name} batch "
+                     f"({int(np.sum(w.context_lens))} context tokens, {self.unique / 1e6:.1f} MB of KV)")
+
+    def step(self):
+        from oracle import attention, cache_ops
+        r, w = self.res, self.w
+        t0 = time.perf_counter()
+        cache_ops.reshape_and_cache(self.k_new, self.v_new, self.slots, r["key_cache"], r["value_cache"])
+        attention.decode_attention(self.q, r["key_cache"], r["value_cache"], r["block_tables"], r["context_lens"],
+                                   w.scale, w.dtype)
+        return time.perf_counter() - t0
+
+
+def cpu_baseline(name, seconds):
+    sample = OracleSample(name, seconds / 4)
+    times = []
+    while not times or sum(times) < seconds * 0.75:
+        times.append(sample.step())
+    rate = sample.unique * len(times) / sum(times) / 1e9
+    return {"value": rate, "unit": UNIT, "cores": sample.cores, "kind": "oracle",
+            "sample": f"{sample.desc}; {len(times)} oracle step(s), {sum(times):.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from paged_kv_cache_356_b200 import workloads
+    w = workloads.by_name(args.workload)
+    sample = OracleSample(args.workload, max(0.05, 90.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        sample.step()
+    times = [sample.step() for _ in range(args.steps)]
+    per_step = statistics.median(times)
+    value = sample.unique / per_step / 1e9
+    desc = f"{sample.desc}; median of {args.steps} oracle steps"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": describe(w),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": sample.cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "note": "fp64 NumPy CPU oracle, as it stands, on the host cores; each step is a bounded sample"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from paged_kv_cache_356_b200 import binding as pa
+    from paged_kv_cache_356_b200 import build as pa_build
+    from paged_kv_cache_356_b200 import workloads
+    from paged_kv_cache_356_b200.runner import TraceRunner
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    pa_build.build()
+    pa.pa_set_decode_kernel({"auto": pa.PA_DECODE_AUTO, "tc": pa.PA_DECODE_TENSOR_CORES,
+                             "cc": pa.PA_DECODE_CUDA_CORES}[args.kernel])
+    warps, stages = (int(x) for x in args.tiling.split("x"))
+    pa.pa_set_decode_tiling(warps, stages)
+
+    seed_shift = 1000 * rank
+    w = workloads.by_name(args.workload, seed=workloads.by_name(args.workload).seed + seed_shift)
+    run = TraceRunner(w)
+    run.run(decode=False)
+    torch.cuda.synchronize()
+    if run.status() != 0:
+        raise RuntimeError(f"device status {run.status()} after setup")
+    tables_np = run.block_tables.cpu().numpy()
+    ctx_np = run.context_lens.cpu().numpy()
+    unique, logical = kv_bytes(w, tables_np, ctx_np)
+    part_bytes = partition_kernel_bytes(w, ctx_np, unique)
+    max_ctx = w.max_blocks_per_seq * w.block_size
+    stream = torch.cuda.current_stream()
+    kd, vd, sd = run.step_write
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        pa.pa_reshape_and_cache(kd, vd, sd, run.key_cache, run.value_cache, stream=stream)
+        if evs is not None:
+            evs[1].record(stream)
+        pa.pa_decode_partitions(run.q, run.key_cache, run.value_cache, run.block_tables, run.context_lens, w.scale,
+                                run.out, run.workspace, stream=stream)
+        if evs is not None:
+            evs[2].record(stream)
+        pa.pa_decode_reduce(run.context_lens, max_ctx, run.out, run.workspace, stream=stream)
+        if evs is not None:
+            evs[3].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(gpu_smi_id(torch, local))
+    sampler.start()
+    time.sleep(0.3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = evs[0][0].elapsed_time(evs[-1][3])
+    # keep identical steps running until the clock record spans at least ~1.5 s under load
+    soak_until = time.perf_counter() + max(0.0, 1.5 - total_ms / 1000)
+    while time.perf_counter() < soak_until:
+        for _ in range(20):
+            step()
+        torch.cuda.synchronize()
+    clocks = sampler.stop()
+
+    write_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    part_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    reduce_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+
+    t = torch.tensor([total_ms, float(unique), float(w.num_seqs)], dtype=torch.float64, device="cuda")
+    if world > 1:
+        tmax = t[:1].clone()
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+        tsum = t[1:].clone()
+        dist.all_reduce(tsum, op=dist.ReduceOp.SUM)
+        total_ms_max, all_unique, all_seqs = float(tmax[0]), float(tsum[0]), float(tsum[1])
+    else:
+        total_ms_max, all_unique, all_seqs = total_ms, float(unique), float(w.num_seqs)
+    seconds = total_ms_max / 1000.0
+    value = all_unique * args.steps / seconds / 1e9
+    seqs_per_s = all_seqs * args.steps / seconds
+
+    # end to end through the API, host buffers: export tables, copy inputs in, decode, read the output back
+    e2e = None
+    if not args.no_e2e:
+        e2e = end_to_end(args, torch, pa, run, w, unique, max_ctx, world, dist)
+
+    peak, peak_kind = measured_peak()
+    achieved = part_bytes / (part_ms / 1000.0) / 1e9
+    khash = kernel_source_hash()
+    traffic, _ = profiled_traffic(khash)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload, args.cpu_seconds)
+
+    if rank == 0:
+        cfg = describe(w)
+        cfg.update({"parallelism": f"dp{world} (independent batches per GPU, no collective)",
+                    "l2": "no flush: each step reads the whole KV cache, far larger than the 126 MB L2",
+                    "kernel": args.kernel, "tiling": args.tiling, "global_batch": w.num_seqs * world})
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else w.dtype,
+            "data": "synthetic", "config": cfg,
+            "seqs_per_s": seqs_per_s,
+            "kv_bytes_per_step": {"unique": unique, "logical": logical},
+            "frac_of_hbm": {"measured": value / world / peak, "nominal_8000": value / world / NOMINAL_HBM_GBS},
+            "kernel_ms": {"reshape_and_cache": write_ms, "decode_partitions": part_ms, "decode_reduce": reduce_ms},
+            "roofline": {"bound": "hbm", "kernel": "decode_tc_kernel (pa_decode_partitions)",
+                         "achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} (copy bandwidth)",
+                         "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                         "algorithmic_bytes_per_launch": part_bytes, "kernel_source_sha256": khash},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 3 * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def end_to_end(args, torch, pa, run, w, unique, max_ctx, world, dist):
+    """Same steps through the public API from pinned host buffers; wall clock, result read back each step."""
+    kd, vd, sd = run.step_write
+    pin = dict(pin_memory=True)
+    h_q = torch.empty(run.q.shape, dtype=run.q.dtype, **pin)
+    h_q.copy_(run.q)
+    h_k = torch.empty(kd.shape, dtype=kd.dtype, **pin)
+    h_k.copy_(kd)
+    h_v = torch.empty(vd.shape, dtype=vd.dtype, **pin)
+    h_v.copy_(vd)
+    h_s = torch.empty(sd.shape, dtype=sd.dtype, **pin)
+    h_s.copy_(sd)
+    h_tab = torch.empty(run.block_tables.shape, dtype=torch.int32, **pin)
+    h_ctx = torch.empty(run.context_lens.shape, dtype=torch.int32, **pin)
+    h_out = torch.empty(run.out.shape, dtype=run.out.dtype, **pin)
+    d_q, d_k, d_v, d_s = (torch.empty_like(x, device="cuda") for x in (h_q, h_k, h_v, h_s))
+    d_tab = torch.empty_like(run.block_tables)
+    d_ctx = torch.empty_like(run.context_lens)
+    d_out = torch.empty_like(run.out)
+    seqs = list(range(w.num_seqs))
+    tab_np, ctx_np = h_tab.numpy(), h_ctx.numpy()
+
+    def e2e_step():
+        run.alloc.block_tables(seqs, w.max_blocks_per_seq, pad=-1, out=tab_np, lens_out=ctx_np)
+        for dst, src in ((d_q, h_q), (d_k, h_k), (d_v, h_v), (d_s, h_s), (d_tab, h_tab), (d_ctx, h_ctx)):
+            dst.copy_(src, non_blocking=True)
+        pa.pa_reshape_and_cache(d_k, d_v, d_s, run.key_cache, run.value_cache)
+        pa.pa_decode(d_q, run.key_cache, run.value_cache, d_tab, d_ctx, w.scale, out=d_out, workspace=run.workspace)
+        h_out.copy_(d_out, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    for _ in range(3):
+        e2e_step()
+    if not torch.equal(h_out.view(torch.int16), run.out.cpu().view(torch.int16)):
+        raise RuntimeError("end-to-end output differs from the device-resident step")
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        e2e_step()
+    elapsed = time.perf_counter() - t0
+    el = torch.tensor([elapsed, float(unique)], dtype=torch.float64, device="cuda")
+    if world > 1:
+        mx = el[:1].clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        sm = el[1:].clone()
+        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+        elapsed, unique = float(mx[0]), float(sm[0])
+    h2d = sum(x.numel() * x.element_size() for x in (h_q, h_k, h_v, h_s, h_tab, h_ctx))
+    d2h = h_out.numel() * h_out.element_size()
+    return {"value": unique * args.steps / elapsed / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": 1000 * elapsed / args.steps,
+            "includes": "host table export (C ABI), pinned H2D of q/new K,V/slots/tables/lengths, "
+                        "reshape_and_cache + decode, D2H of out, stream sync"}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,275 @@
+/*
+ * pa.h -- C ABI of the B200 paged KV-cache decode path (libpa_b200.so).
+ *
+ * Sources of the operations (web pages on PagedAttention):
+ *   [Glossary]    "What is PagedAttention? Definition & Virtual Memory Architecture
+ *                 in Enterprise AI" (esaholic.com AI glossary)
+ *   [Internals]   "PagedAttention Internals: How Memory Fragmentation in LLM
+ *                 Serving Was Solved" (dailyaiworld.com)
+ *   [Terminology] "Paged Attention" (invest-in.ai AI terminology)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * KV cache layout.  key_cache and value_cache are two separate device arrays of
+ *   shape [num_blocks][num_kv_heads][block_size][head_dim], row-major, element
+ *   type `dtype`.  One physical page ("block") holds block_size consecutive
+ *   token positions of one sequence for every kv head; the slab of one
+ *   (page, kv head) pair is block_size * head_dim contiguous elements.
+ * Slots.  Physical slot s names page s / block_size, position s % block_size.
+ * Ownership.  The caller allocates and owns every device buffer (PyTorch or
+ *   cudaMalloc); no entry point allocates or frees device memory.  The
+ *   allocator handle (pa_block_alloc) is host memory owned by the library
+ *   between create and destroy.
+ * Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream).  Device entry points only enqueue work on it; none synchronises.
+ * Errors.  Every entry point returns a pa_status.  Argument errors are detected
+ *   on the host before anything is enqueued, and nothing is enqueued then.
+ *   pa_last_error() returns a thread-local message for the last failure.
+ * Device status.  Kernels check every index they dereference (page ids,
+ *   slots, copy pairs, context lengths) and skip what is out of range instead
+ *   of touching memory outside the arrays.  If `dev_status` is non-NULL (a
+ *   device int32) they OR the PA_DEV_* bits of what they skipped into it; the
+ *   caller reads it after the stream has run the work.  The word is never
+ *   cleared by the library.
+ * Alignment.  Device pointers must be 16-byte aligned and
+ *   head_dim * sizeof(element) a multiple of 16 bytes.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_status {
+  PA_OK = 0,
+  PA_ERR_INVALID = -1,     /* bad argument: null pointer, bad size, misalignment */
+  PA_ERR_OOM = -2,         /* the free-page pool cannot satisfy the request; state unchanged */
+  PA_ERR_CUDA = -3,        /* a CUDA runtime call failed; see pa_last_error() */
+  PA_ERR_NOT_FOUND = -4,   /* unknown sequence id */
+  PA_ERR_UNSUPPORTED = -5  /* a shape / dtype combination this build has no kernel for */
+} pa_status;
+
+typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1, PA_F16 = 2 } pa_dtype;
+
+/* Bits a kernel ORs into *dev_status when it skips an out-of-range index. */
+#define PA_DEV_BAD_SLOT 1 /* reshape_and_cache: slot >= num_blocks * block_size           */
+#define PA_DEV_BAD_PAGE 2 /* decode: a block-table entry the context needs is outside the pool */
+#define PA_DEV_BAD_CTX 4  /* decode: context_len < 0 or > max_blocks_per_seq * block_size  */
+#define PA_DEV_BAD_PAIR 8 /* copy_blocks: a source or destination page is outside the pool  */
+
+/* Tokens per split-context partition of pa_decode. */
+#define PA_PARTITION_TOKENS 512
+
+PA_API const char* pa_last_error(void);
+PA_API const char* pa_version(void);
+
+/* ------------------------------------------------------------------------
+ * pa_reshape_and_cache -- store new tokens' K and V in their physical slots.
+ *
+ * [Internals] "2. The Dynamic Block Table": as the model generates tokens,
+ * their K/V go to pages taken on demand from the free pool; [Glossary]
+ * "Technical Architecture": a page table maps logical positions to pages.
+ *
+ * key, value      device, [num_tokens][num_kv_heads][head_dim]; consecutive
+ *                 tokens key_token_stride / value_token_stride elements apart
+ *                 (heads and dims contiguous; stride >= num_kv_heads*head_dim).
+ * slot_mapping    device int64 [num_tokens]: token t goes to slot_mapping[t];
+ *                 a negative slot skips the token (padding).
+ * key_cache, value_cache  device, layout above; written, bit-exact copies.
+ * Slots must be distinct (two tokens to one slot race).  A slot
+ * >= num_blocks*block_size is skipped and flagged PA_DEV_BAD_SLOT.
+ * ---------------------------------------------------------------------- */
+PA_API pa_status pa_reshape_and_cache(const void* key, const void* value, int64_t key_token_stride,
+                               int64_t value_token_stride, const int64_t* slot_mapping,
+                               int64_t num_tokens, void* key_cache, void* value_cache,
+                               int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+                               int32_t head_dim, pa_dtype dtype, int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------
+ * pa_copy_blocks -- copy whole pages, K and V: the device half of a
+ * copy-on-write fork.
+ *
+ * [Glossary] "Copy-on-Write Memory Forking": pages are duplicated only when
+ * parallel outputs diverge; [Internals] "Copy-on-Write and Prefix Sharing".
+ *
+ * block_mapping   device int64 [num_pairs][2] = (src page, dst page).  Every
+ *                 slot of every kv head of page src is copied onto page dst,
+ *                 in key_cache and in value_cache.  Destinations must be
+ *                 distinct and must not appear as sources (the pairs run in
+ *                 parallel).  Pages outside [0, num_blocks) are skipped and
+ *                 flagged PA_DEV_BAD_PAIR.
+ * ---------------------------------------------------------------------- */
+PA_API pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* block_mapping,
+                         int32_t num_pairs, int32_t num_blocks, int32_t block_size,
+                         int32_t num_kv_heads, int32_t head_dim, pa_dtype dtype,
+                         int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------
+ * pa_decode -- one decode step of scaled dot-product attention over the
+ * paged cache: for each sequence b and query head h,
+ *     s_j   = scale * <q[b][h], K_b[j][h / G]>,   j < context_lens[b]
+ *     out[b][h] = sum_j softmax(s)_j * V_b[j][h / G],   G = num_q_heads / num_kv_heads
+ * where K_b[j], V_b[j] sit in page block_tables[b][j / block_size], position
+ * j % block_size.
+ *
+ * [Internals] "3. Fused PagedAttention CUDA Kernel": the inner attention loop
+ * fetches non-contiguous K/V through the block table and runs scaled
+ * dot-product attention; [Glossary] "On-the-Fly CUDA Block Fetching".
+ *
+ * q               device [num_seqs][num_q_heads][head_dim], dtype.
+ * block_tables    device int32 [num_seqs][max_blocks_per_seq]; entries past a
+ *                 sequence's last block are never read.
+ * context_lens    device int32 [num_seqs]; 0 gives a zero output row.
+ * scale           softmax scale (1/sqrt(head_dim) for standard attention).
+ * out             device [num_seqs][num_q_heads][head_dim], dtype (rounded to
+ *                 nearest even from fp32 accumulators for bf16/f16).
+ * workspace       device scratch of at least
+ *                 pa_decode_workspace_size(num_seqs, num_q_heads, head_dim,
+ *                 max_blocks_per_seq * block_size) bytes, 256-byte aligned.
+ *                 Sequences longer than PA_PARTITION_TOKENS are split into
+ *                 partitions whose partial results go here and are then
+ *                 merged by a log-sum-exp reduction.  Layout, with
+ *                 P = ceil(max_blocks_per_seq*block_size / PA_PARTITION_TOKENS):
+ *                   float o_part[num_seqs][num_q_heads][P][head_dim]  (o_p / l_p)
+ *                   float m_part[num_seqs][num_q_heads][P]  (max score, natural log units)
+ *                   float l_part[num_seqs][num_q_heads][P]  (sum of exp(s - m_p))
+ *                 Only partitions of sequences with more than one partition
+ *                 are written.
+ * GQA: query head h reads kv head h / G.  Supported: head_dim in
+ * {64, 128, 256}; num_q_heads a multiple of num_kv_heads; block_size in
+ * [1, 256].  An out-of-range page id needed by the context is skipped
+ * (its tokens are dropped) and flagged PA_DEV_BAD_PAGE; a context length
+ * outside [0, max_blocks_per_seq*block_size] is clamped and flagged
+ * PA_DEV_BAD_CTX.
+ * ---------------------------------------------------------------------- */
+PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                int64_t max_context_len);
+
+PA_API pa_status pa_decode(const void* q, const void* key_cache, const void* value_cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                    const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                    int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                    float scale, void* out, pa_dtype dtype, void* workspace,
+                    size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* The two steps of pa_decode, callable on their own (same arguments and
+ * workspace contract; pa_decode = pa_decode_partitions, then, when
+ * max_blocks_per_seq * block_size > PA_PARTITION_TOKENS, pa_decode_reduce).
+ * pa_decode_partitions writes the output rows of one-partition sequences and
+ * the workspace partials of the others; pa_decode_reduce merges those
+ * partials into their output rows (max_context_len = max_blocks_per_seq *
+ * block_size of the partition call) and leaves the other rows untouched. */
+PA_API pa_status pa_decode_partitions(const void* q, const void* key_cache, const void* value_cache,
+                                      const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                      const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                                      int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                      int32_t num_blocks, float scale, void* out, pa_dtype dtype,
+                                      void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                      void* stream);
+PA_API pa_status pa_decode_reduce(const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                                  int32_t head_dim, int64_t max_context_len, void* out, pa_dtype dtype,
+                                  const void* workspace, size_t workspace_bytes, void* stream);
+
+/* Which partition kernel pa_decode runs (process-wide; default AUTO).
+ * AUTO picks the tensor-core kernel whenever it supports the call (bf16/f16,
+ * head_dim 64/128/256, G <= 8, block_size a multiple of 16 up to 256) and the
+ * CUDA-core kernel otherwise.  Forcing TENSOR_CORES on a call it does not
+ * support makes pa_decode return PA_ERR_UNSUPPORTED.  Both kernels compute
+ * the same result; the switch exists for testing and measurement. */
+typedef enum pa_decode_kernel {
+  PA_DECODE_AUTO = 0,
+  PA_DECODE_CUDA_CORES = 1,
+  PA_DECODE_TENSOR_CORES = 2
+} pa_decode_kernel;
+PA_API pa_status pa_set_decode_kernel(pa_decode_kernel kernel);
+
+/* Tiling of the tensor-core kernel (process-wide): warps per CTA and
+ * shared-memory pipeline stages per warp.  Built: (4,2) (4,3) (4,4) (2,4)
+ * (8,2); default (4,3).  Others return PA_ERR_UNSUPPORTED.  For tuning. */
+PA_API pa_status pa_set_decode_tiling(int32_t warps, int32_t stages);
+
+/* ------------------------------------------------------------------------
+ * pa_block_alloc -- host-side ref-counted free-page pool and block tables
+ * (control plane; never touches device memory).
+ *
+ * [Internals] "2. The Dynamic Block Table" and "Implementation: Custom Block
+ * Manager Simulation in Python" (allocate_sequence / append_token /
+ * free_sequence); [Internals] "Copy-on-Write and Prefix Sharing" and
+ * [Glossary] "Copy-on-Write Memory Forking" (shared pages, reference counts).
+ *
+ * Policy: a sequence of n tokens holds ceil(n / block_size) pages; pages leave
+ * the free pool at its front and return to its back when their reference
+ * count drops to zero (a freed table is visited in order); a new page starts
+ * at count 1.  Every operation is all-or-nothing: on error nothing changes.
+ * A handle is not thread-safe; sequence ids are arbitrary int64 keys.
+ * ---------------------------------------------------------------------- */
+typedef struct pa_block_alloc pa_block_alloc;
+
+/* initial_free_order: NULL for 0..num_blocks-1, else a host permutation of it
+ * giving the pool's starting order.  *out receives the handle. */
+PA_API pa_status pa_block_alloc_create(int32_t num_blocks, int32_t block_size,
+                                const int32_t* initial_free_order, pa_block_alloc** out);
+PA_API void pa_block_alloc_destroy(pa_block_alloc* a);
+
+/* Admit a new sequence holding num_tokens positions.  PA_ERR_OOM if fewer than
+ * ceil(num_tokens / block_size) pages are free; PA_ERR_INVALID if seq exists. */
+PA_API pa_status pa_block_alloc_allocate_sequence(pa_block_alloc* a, int64_t seq, int64_t num_tokens);
+
+/* Grow seq by one position.  *slot_out receives its physical slot.  If the
+ * position starts a new block a page is taken.  If it falls in a page shared
+ * with another sequence (count > 1) the sequence first takes a fresh page,
+ * the shared page loses a reference, and (*cow_src, *cow_dst) receive the
+ * page pair the caller must copy with pa_copy_blocks before writing either;
+ * otherwise both receive -1.  cow_src / cow_dst may be NULL only if the
+ * caller knows no page is shared. */
+PA_API pa_status pa_block_alloc_append_token(pa_block_alloc* a, int64_t seq, int64_t* slot_out,
+                                      int32_t* cow_src, int32_t* cow_dst);
+
+/* New sequence `child` sharing every page of `parent` (each gains one
+ * reference); it starts with the parent's token count. */
+PA_API pa_status pa_block_alloc_fork(pa_block_alloc* a, int64_t parent, int64_t child);
+
+/* Drop seq: every page loses a reference; pages reaching zero return to the
+ * back of the pool in table order.  An unknown seq is a no-op (PA_OK). */
+PA_API pa_status pa_block_alloc_free_sequence(pa_block_alloc* a, int64_t seq);
+
+/* Physical slots of positions [start, start + count) of seq, into out[count]. */
+PA_API pa_status pa_block_alloc_slot_mapping(const pa_block_alloc* a, int64_t seq, int64_t start,
+                                      int64_t count, int64_t* out);
+
+/* seq's table into out[cap]; *n_out receives its length (even if > cap, in
+ * which case nothing is written and PA_ERR_INVALID is returned). */
+PA_API pa_status pa_block_alloc_block_table(const pa_block_alloc* a, int64_t seq, int32_t* out,
+                                     int32_t cap, int32_t* n_out);
+
+/* Padded tables of n sequences into out[n][max_blocks_per_seq] (row-major),
+ * entries past each table set to pad; context_lens_out[n] (may be NULL)
+ * receives each token count.  PA_ERR_INVALID if a table is longer. */
+PA_API pa_status pa_block_alloc_block_tables(const pa_block_alloc* a, const int64_t* seqs, int32_t n,
+                                      int32_t* out, int32_t max_blocks_per_seq, int32_t pad,
+                                      int32_t* context_lens_out);
+
+PA_API int64_t pa_block_alloc_num_tokens(const pa_block_alloc* a, int64_t seq); /* -1 if unknown */
+PA_API int32_t pa_block_alloc_num_free(const pa_block_alloc* a);
+PA_API int32_t pa_block_alloc_num_sequences(const pa_block_alloc* a);
+PA_API int32_t pa_block_alloc_ref_count(const pa_block_alloc* a, int32_t page); /* -1 if out of range */
+
+/* The free pool front to back into out[cap]; *n_out receives its length. */
+PA_API pa_status pa_block_alloc_free_pool(const pa_block_alloc* a, int32_t* out, int32_t cap,
+                                   int32_t* n_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

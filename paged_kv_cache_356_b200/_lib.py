@@ -1,0 +1,79 @@
+"""Loads libpa_b200.so and declares the C signatures of include/pa.h.
+
+There is no fallback: if the library is missing the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpa_b200.so")
+
+PA_OK, PA_ERR_INVALID, PA_ERR_OOM, PA_ERR_CUDA, PA_ERR_NOT_FOUND, PA_ERR_UNSUPPORTED = 0, -1, -2, -3, -4, -5
+PA_F32, PA_BF16, PA_F16 = 0, 1, 2
+PA_DEV_BAD_SLOT, PA_DEV_BAD_PAGE, PA_DEV_BAD_CTX, PA_DEV_BAD_PAIR = 1, 2, 4, 8
+PA_DECODE_AUTO, PA_DECODE_CUDA_CORES, PA_DECODE_TENSOR_CORES = 0, 1, 2
+PA_PARTITION_TOKENS = 512
+
+_c = ctypes
+_vp, _i32, _i64, _f32, _sz = _c.c_void_p, _c.c_int32, _c.c_int64, _c.c_float, _c.c_size_t
+_pi32, _pi64 = _c.POINTER(_c.c_int32), _c.POINTER(_c.c_int64)
+
+# name -> (restype, argtypes); mirrors include/pa.h
+SIGNATURES = {
+    "pa_last_error": (_c.c_char_p, []),
+    "pa_version": (_c.c_char_p, []),
+    "pa_reshape_and_cache": (_i32, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
+                                    _vp, _vp]),
+    "pa_copy_blocks": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
+    "pa_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i64]),
+    "pa_decode": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _i32,
+                         _vp, _sz, _vp, _vp]),
+    "pa_decode_partitions": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp,
+                                    _i32, _vp, _sz, _vp, _vp]),
+    "pa_decode_reduce": (_i32, [_vp, _i32, _i32, _i32, _i64, _vp, _i32, _vp, _sz, _vp]),
+    "pa_set_decode_kernel": (_i32, [_i32]),
+    "pa_set_decode_tiling": (_i32, [_i32, _i32]),
+    "pa_block_alloc_create": (_i32, [_i32, _i32, _pi32, _c.POINTER(_vp)]),
+    "pa_block_alloc_destroy": (None, [_vp]),
+    "pa_block_alloc_allocate_sequence": (_i32, [_vp, _i64, _i64]),
+    "pa_block_alloc_append_token": (_i32, [_vp, _i64, _pi64, _pi32, _pi32]),
+    "pa_block_alloc_fork": (_i32, [_vp, _i64, _i64]),
+    "pa_block_alloc_free_sequence": (_i32, [_vp, _i64]),
+    "pa_block_alloc_slot_mapping": (_i32, [_vp, _i64, _i64, _i64, _pi64]),
+    "pa_block_alloc_block_table": (_i32, [_vp, _i64, _pi32, _i32, _pi32]),
+    "pa_block_alloc_block_tables": (_i32, [_vp, _pi64, _i32, _pi32, _i32, _i32, _pi32]),
+    "pa_block_alloc_num_tokens": (_i64, [_vp, _i64]),
+    "pa_block_alloc_num_free": (_i32, [_vp]),
+    "pa_block_alloc_num_sequences": (_i32, [_vp]),
+    "pa_block_alloc_ref_count": (_i32, [_vp, _i32]),
+    "pa_block_alloc_free_pool": (_i32, [_vp, _pi32, _i32, _pi32]),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """The loaded library with every signature declared (raises if absent)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(f"{LIB_PATH} is missing: build it with "
+                                  "`python -m paged_kv_cache_356_b200.build` (needs nvcc)")
+            lib = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def last_error() -> str:
+    msg = load().pa_last_error()
+    return msg.decode() if msg else ""

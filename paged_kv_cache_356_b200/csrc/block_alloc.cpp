@@ -1,0 +1,227 @@
+// pa_block_alloc: host-side ref-counted free-page pool and per-sequence block
+// tables -- the control plane of the paged KV cache.
+//
+// PagedAttention Internals, "2. The Dynamic Block Table": one table per
+// sequence maps logical blocks to physical pages taken on demand from a global
+// free-page pool.  "Implementation: Custom Block Manager Simulation in Python":
+// ceil(n / bs) pages per sequence, an out-of-memory failure checked before any
+// page is taken, pages taken from the front of the pool and returned to its
+// back in table order when their count reaches zero, a fresh page at count 1,
+// freeing an unknown sequence is a no-op.  "Copy-on-Write and Prefix Sharing"
+// (and the glossary's "Copy-on-Write Memory Forking"): shared pages carry a
+// reference count, and a page is duplicated only when a sequence writes into
+// it while others still hold it.
+//
+// The pool is a fixed ring of num_blocks ids (it can never hold more), so
+// taking from the front and returning to the back are O(1).
+#include <unordered_map>
+#include <vector>
+
+#include "pa_internal.h"
+
+struct pa_block_alloc {
+  int32_t num_blocks = 0;
+  int32_t block_size = 0;
+  std::vector<int32_t> ring;  // free pool, front at `head`, `count` ids
+  int64_t head = 0;
+  int64_t count = 0;
+  std::vector<int32_t> refs;
+  struct Seq {
+    std::vector<int32_t> pages;
+    int64_t tokens = 0;
+  };
+  std::unordered_map<int64_t, Seq> seqs;
+
+  int32_t take_front() {
+    int32_t page = ring[head];
+    head = (head + 1) % num_blocks;
+    --count;
+    refs[page] = 1;
+    return page;
+  }
+  void release(int32_t page) {
+    if (--refs[page] == 0) {
+      ring[(head + count) % num_blocks] = page;
+      ++count;
+    }
+  }
+};
+
+using pa::fail;
+
+extern "C" {
+
+pa_status pa_block_alloc_create(int32_t num_blocks, int32_t block_size,
+                                const int32_t* initial_free_order, pa_block_alloc** out) {
+  if (!out) return fail(PA_ERR_INVALID, "pa_block_alloc_create: out is NULL");
+  *out = nullptr;
+  if (num_blocks < 0 || block_size <= 0)
+    return fail(PA_ERR_INVALID, "pa_block_alloc_create: num_blocks=%d block_size=%d", num_blocks,
+                block_size);
+  auto* a = new pa_block_alloc();
+  a->num_blocks = num_blocks;
+  a->block_size = block_size;
+  a->ring.resize(num_blocks > 0 ? num_blocks : 1);
+  a->refs.assign(num_blocks, 0);
+  if (initial_free_order) {
+    std::vector<char> seen(num_blocks, 0);
+    for (int32_t i = 0; i < num_blocks; ++i) {
+      int32_t p = initial_free_order[i];
+      if (p < 0 || p >= num_blocks || seen[p]) {
+        delete a;
+        return fail(PA_ERR_INVALID, "pa_block_alloc_create: initial_free_order is not a permutation");
+      }
+      seen[p] = 1;
+      a->ring[i] = p;
+    }
+  } else {
+    for (int32_t i = 0; i < num_blocks; ++i) a->ring[i] = i;
+  }
+  a->count = num_blocks;
+  *out = a;
+  return PA_OK;
+}
+
+void pa_block_alloc_destroy(pa_block_alloc* a) { delete a; }
+
+pa_status pa_block_alloc_allocate_sequence(pa_block_alloc* a, int64_t seq, int64_t num_tokens) {
+  if (!a) return fail(PA_ERR_INVALID, "allocate_sequence: NULL handle");
+  if (num_tokens < 0) return fail(PA_ERR_INVALID, "allocate_sequence: num_tokens=%lld", (long long)num_tokens);
+  if (a->seqs.count(seq)) return fail(PA_ERR_INVALID, "allocate_sequence: sequence %lld exists", (long long)seq);
+  int64_t need = (num_tokens + a->block_size - 1) / a->block_size;
+  if (need > a->count)
+    return fail(PA_ERR_OOM, "allocate_sequence: %lld pages needed, %lld free", (long long)need,
+                (long long)a->count);
+  auto& s = a->seqs[seq];
+  s.pages.reserve(need);
+  for (int64_t i = 0; i < need; ++i) s.pages.push_back(a->take_front());
+  s.tokens = num_tokens;
+  return PA_OK;
+}
+
+pa_status pa_block_alloc_append_token(pa_block_alloc* a, int64_t seq, int64_t* slot_out,
+                                      int32_t* cow_src, int32_t* cow_dst) {
+  if (!a) return fail(PA_ERR_INVALID, "append_token: NULL handle");
+  auto it = a->seqs.find(seq);
+  if (it == a->seqs.end()) return fail(PA_ERR_NOT_FOUND, "append_token: unknown sequence %lld", (long long)seq);
+  auto& s = it->second;
+  const int64_t pos = s.tokens;
+  const int64_t logical = pos / a->block_size;
+  const int64_t offset = pos % a->block_size;
+  int32_t src = -1, dst = -1;
+  if (offset == 0) {
+    if (a->count == 0) return fail(PA_ERR_OOM, "append_token: no free page for the next block");
+    s.pages.push_back(a->take_front());
+  } else if (a->refs[s.pages[logical]] > 1) {
+    if (!cow_src || !cow_dst)
+      return fail(PA_ERR_INVALID, "append_token: page %d is shared but cow_src/cow_dst are NULL",
+                  s.pages[logical]);
+    if (a->count == 0) return fail(PA_ERR_OOM, "append_token: no free page for the copy-on-write fork");
+    src = s.pages[logical];
+    dst = a->take_front();
+    a->release(src);
+    s.pages[logical] = dst;
+  }
+  s.tokens = pos + 1;
+  if (slot_out) *slot_out = (int64_t)s.pages[logical] * a->block_size + offset;
+  if (cow_src) *cow_src = src;
+  if (cow_dst) *cow_dst = dst;
+  return PA_OK;
+}
+
+pa_status pa_block_alloc_fork(pa_block_alloc* a, int64_t parent, int64_t child) {
+  if (!a) return fail(PA_ERR_INVALID, "fork: NULL handle");
+  auto it = a->seqs.find(parent);
+  if (it == a->seqs.end()) return fail(PA_ERR_NOT_FOUND, "fork: unknown parent %lld", (long long)parent);
+  if (a->seqs.count(child)) return fail(PA_ERR_INVALID, "fork: sequence %lld exists", (long long)child);
+  pa_block_alloc::Seq copy = it->second;  // copy before inserting (rehash may move `it`)
+  for (int32_t p : copy.pages) ++a->refs[p];
+  a->seqs.emplace(child, std::move(copy));
+  return PA_OK;
+}
+
+pa_status pa_block_alloc_free_sequence(pa_block_alloc* a, int64_t seq) {
+  if (!a) return fail(PA_ERR_INVALID, "free_sequence: NULL handle");
+  auto it = a->seqs.find(seq);
+  if (it == a->seqs.end()) return PA_OK;
+  for (int32_t p : it->second.pages) a->release(p);
+  a->seqs.erase(it);
+  return PA_OK;
+}
+
+pa_status pa_block_alloc_slot_mapping(const pa_block_alloc* a, int64_t seq, int64_t start,
+                                      int64_t count, int64_t* out) {
+  if (!a || (!out && count > 0)) return fail(PA_ERR_INVALID, "slot_mapping: NULL argument");
+  auto it = a->seqs.find(seq);
+  if (it == a->seqs.end()) return fail(PA_ERR_NOT_FOUND, "slot_mapping: unknown sequence %lld", (long long)seq);
+  const auto& s = it->second;
+  if (start < 0 || count < 0 || start + count > s.tokens)
+    return fail(PA_ERR_INVALID, "slot_mapping: positions [%lld, %lld) outside [0, %lld)", (long long)start,
+                (long long)(start + count), (long long)s.tokens);
+  const int64_t bs = a->block_size;
+  for (int64_t i = 0; i < count; ++i) {
+    const int64_t pos = start + i;
+    out[i] = (int64_t)s.pages[pos / bs] * bs + pos % bs;
+  }
+  return PA_OK;
+}
+
+pa_status pa_block_alloc_block_table(const pa_block_alloc* a, int64_t seq, int32_t* out, int32_t cap,
+                                     int32_t* n_out) {
+  if (!a) return fail(PA_ERR_INVALID, "block_table: NULL handle");
+  auto it = a->seqs.find(seq);
+  if (it == a->seqs.end()) return fail(PA_ERR_NOT_FOUND, "block_table: unknown sequence %lld", (long long)seq);
+  const auto& pages = it->second.pages;
+  if (n_out) *n_out = (int32_t)pages.size();
+  if ((int64_t)pages.size() > cap || (!out && !pages.empty()))
+    return fail(PA_ERR_INVALID, "block_table: %zu entries, capacity %d", pages.size(), cap);
+  for (size_t i = 0; i < pages.size(); ++i) out[i] = pages[i];
+  return PA_OK;
+}
+
+pa_status pa_block_alloc_block_tables(const pa_block_alloc* a, const int64_t* seqs, int32_t n, int32_t* out,
+                                      int32_t max_blocks_per_seq, int32_t pad, int32_t* context_lens_out) {
+  if (!a || n < 0 || max_blocks_per_seq < 0 || (n > 0 && (!seqs || !out)))
+    return fail(PA_ERR_INVALID, "block_tables: bad argument");
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = a->seqs.find(seqs[i]);
+    if (it == a->seqs.end())
+      return fail(PA_ERR_NOT_FOUND, "block_tables: unknown sequence %lld", (long long)seqs[i]);
+    const auto& pages = it->second.pages;
+    if ((int64_t)pages.size() > max_blocks_per_seq)
+      return fail(PA_ERR_INVALID, "block_tables: sequence %lld holds %zu pages > %d", (long long)seqs[i],
+                  pages.size(), max_blocks_per_seq);
+    int32_t* row = out + (int64_t)i * max_blocks_per_seq;
+    size_t j = 0;
+    for (; j < pages.size(); ++j) row[j] = pages[j];
+    for (; j < (size_t)max_blocks_per_seq; ++j) row[j] = pad;
+    if (context_lens_out) context_lens_out[i] = (int32_t)it->second.tokens;
+  }
+  return PA_OK;
+}
+
+int64_t pa_block_alloc_num_tokens(const pa_block_alloc* a, int64_t seq) {
+  if (!a) return -1;
+  auto it = a->seqs.find(seq);
+  return it == a->seqs.end() ? -1 : it->second.tokens;
+}
+
+int32_t pa_block_alloc_num_free(const pa_block_alloc* a) { return a ? (int32_t)a->count : -1; }
+
+int32_t pa_block_alloc_num_sequences(const pa_block_alloc* a) { return a ? (int32_t)a->seqs.size() : -1; }
+
+int32_t pa_block_alloc_ref_count(const pa_block_alloc* a, int32_t page) {
+  if (!a || page < 0 || page >= a->num_blocks) return -1;
+  return a->refs[page];
+}
+
+pa_status pa_block_alloc_free_pool(const pa_block_alloc* a, int32_t* out, int32_t cap, int32_t* n_out) {
+  if (!a) return fail(PA_ERR_INVALID, "free_pool: NULL handle");
+  if (n_out) *n_out = (int32_t)a->count;
+  if (a->count > cap || (!out && a->count > 0))
+    return fail(PA_ERR_INVALID, "free_pool: %lld entries, capacity %d", (long long)a->count, cap);
+  for (int64_t i = 0; i < a->count; ++i) out[i] = a->ring[(a->head + i) % a->num_blocks];
+  return PA_OK;
+}
+
+}  // extern "C"

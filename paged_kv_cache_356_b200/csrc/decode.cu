@@ -1,0 +1,831 @@
+// pa_decode: one decode step of scaled dot-product attention over the paged
+// KV cache, with the block-table translation inside the inner loop, a
+// split-context partition of PA_PARTITION_TOKENS tokens, and a log-sum-exp
+// merge of the partitions.
+//
+// PagedAttention Internals, "3. Fused PagedAttention CUDA Kernel": the kernel
+// walks the block table in its inner attention loop, fetches the scattered
+// K/V pages into shared memory and runs scaled dot-product attention.
+// What is PagedAttention?, "On-the-Fly CUDA Block Fetching".
+//
+// Work decomposition: one CTA per (sequence b, kv head, partition p).  Every
+// K/V byte of a sequence is read exactly once; the CTA serves all G query
+// heads that share the kv head (GQA), so a page is never fetched twice.
+//
+// Two partition kernels produce identical partials:
+//   decode_tc_kernel   (bf16/f16, head_dim 64/128/256, G <= 8, block_size a
+//                      multiple of 16): each warp streams 16-token tiles of K
+//                      and V through a cp.async multi-stage pipeline into
+//                      XOR-swizzled shared memory and runs both contractions
+//                      on the tensor cores with mma.sync m16n8k16:
+//                        S^T[16 tok x 8 heads] = K_tile[16 x D] . Q^T[D x 8]
+//                        O^T[D x 8 heads]     += V_tile^T[D x 16] . P^T[16 x 8]
+//                      (tokens on M, the GQA group on N -- no padded rows);
+//                      P^T is re-laid out between the two with movmatrix.
+//   decode_cc_kernel   (any dtype incl. fp32, any block size): CUDA cores, one
+//                      token per warp step, lanes split head_dim.
+// Both keep an online softmax (running max m, running sum l, fp32) per head,
+// merge their warps through shared memory, and write either the final output
+// (one partition) or the partition's (o_p / l_p, m_p, l_p).  decode_reduce
+// then merges partitions: M = max m_p, w_p = l_p e^(m_p - M),
+// out = sum w_p o_p / sum w_p.
+#include <math.h>
+
+#include <atomic>
+
+#include "device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+constexpr int kPartition = PA_PARTITION_TOKENS;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr unsigned kFull = 0xffffffffu;
+
+struct DecodeArgs {
+  const void* q;
+  const void* key_cache;
+  const void* value_cache;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  void* out;
+  float* o_part;
+  float* m_part;
+  float* l_part;
+  int32_t* status;
+  int max_blocks_per_seq;
+  int num_q_heads;
+  int num_kv_heads;
+  int group;
+  int block_size;
+  int num_blocks;
+  int max_partitions;
+  float qk_scale_log2;  // softmax scale * log2(e): scores are kept in base 2
+};
+
+// Context length of sequence b, clamped to what its table can address.
+__device__ __forceinline__ int context_of(const DecodeArgs& a, int b, bool report) {
+  int ctx = __ldg(a.context_lens + b);
+  const int cap = a.max_blocks_per_seq * a.block_size;
+  if (ctx < 0 || ctx > cap) {
+    if (report) flag_status(a.status, PA_DEV_BAD_CTX);
+    ctx = ctx < 0 ? 0 : cap;
+  }
+  return ctx;
+}
+
+// Merge per-warp (m, l, o) held in shared memory and store the CTA's result
+// for heads [h0, h0 + nh): the final row if the sequence has one partition,
+// else the partition's partials.  o_w is [warps][heads_stride][D].
+template <typename T, int D>
+__device__ __forceinline__ void merge_and_store(const DecodeArgs& a, int b, int h0, int nh, int p, int np,
+                                                int warps, int heads_stride, const float* o_w, const float* m_w,
+                                                const float* l_w) {
+  for (int i = threadIdx.x; i < nh * D; i += blockDim.x) {
+    const int j = i / D;
+    const int d = i - j * D;
+    float mx = -INFINITY;
+    for (int w = 0; w < warps; ++w) mx = fmaxf(mx, m_w[w * heads_stride + j]);
+    float l = 0.f, o = 0.f;
+    if (mx != -INFINITY) {
+      for (int w = 0; w < warps; ++w) {
+        const float c = exp2f(m_w[w * heads_stride + j] - mx);
+        l += l_w[w * heads_stride + j] * c;
+        o += o_w[((size_t)w * heads_stride + j) * D + d] * c;
+      }
+    }
+    const float res = l > 0.f ? o / l : 0.f;
+    const int64_t row = (int64_t)b * a.num_q_heads + h0 + j;
+    if (np <= 1) {
+      reinterpret_cast<T*>(a.out)[row * D + d] = from_float<T>(res);
+    } else {
+      const int64_t part = row * a.max_partitions + p;
+      a.o_part[part * D + d] = res;
+      if (d == 0) {
+        a.m_part[part] = mx == -INFINITY ? -INFINITY : mx * kLn2;
+        a.l_part[part] = l;
+      }
+    }
+  }
+}
+
+template <typename T, int D>
+__device__ __forceinline__ void store_zero_rows(const DecodeArgs& a, int b, int h0, int nh) {
+  T* out = reinterpret_cast<T*>(a.out);
+  for (int i = threadIdx.x; i < nh * D; i += blockDim.x)
+    out[((int64_t)b * a.num_q_heads + h0) * D + i] = from_float<T>(0.f);
+}
+
+// ---------------------------------------------------------------------------
+// CUDA-core partition kernel.  Grid (num_seqs, num_kv_heads * head_chunks, P);
+// a CTA serves up to GC query heads of one kv head.
+// ---------------------------------------------------------------------------
+template <typename T, int D, int GC, int NW>
+__global__ void __launch_bounds__(NW * 32) decode_cc_kernel(const DecodeArgs a) {
+  constexpr int VPL = D / 32;
+  __shared__ float o_w[NW * GC * D];
+  __shared__ float m_w[NW * GC];
+  __shared__ float l_w[NW * GC];
+
+  const int b = blockIdx.x;
+  const int chunks = (a.group + GC - 1) / GC;
+  const int kvh = blockIdx.y / chunks;
+  const int chunk = blockIdx.y - kvh * chunks;
+  const int h0 = kvh * a.group + chunk * GC;
+  const int nh = min(GC, a.group - chunk * GC);
+  const int p = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int ctx = context_of(a, b, threadIdx.x == 0 && blockIdx.y == 0 && p == 0);
+  const int np = (ctx + kPartition - 1) / kPartition;
+  if (p >= max(np, 1)) return;
+  if (ctx == 0) {
+    store_zero_rows<T, D>(a, b, h0, nh);
+    return;
+  }
+  const int tok_begin = p * kPartition;
+  const int tok_end = min(ctx, tok_begin + kPartition);
+
+  float qv[GC][VPL];
+#pragma unroll
+  for (int g = 0; g < GC; ++g) {
+    if (g < nh) {
+      load_floats<T, VPL>(reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.num_q_heads + h0 + g) * D + lane * VPL,
+                          qv[g]);
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) qv[g][i] *= a.qk_scale_log2;
+    } else {
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) qv[g][i] = 0.f;
+    }
+  }
+  float m[GC], l[GC], o[GC][VPL];
+#pragma unroll
+  for (int g = 0; g < GC; ++g) {
+    m[g] = -INFINITY;
+    l[g] = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) o[g][i] = 0.f;
+  }
+
+  const T* kc = reinterpret_cast<const T*>(a.key_cache);
+  const T* vc = reinterpret_cast<const T*>(a.value_cache);
+  const int32_t* table = a.block_tables + (int64_t)b * a.max_blocks_per_seq;
+  for (int tok = tok_begin + warp; tok < tok_end; tok += NW) {
+    const int page = __ldg(table + tok / a.block_size);
+    if ((unsigned)page >= (unsigned)a.num_blocks) {
+      if (lane == 0) flag_status(a.status, PA_DEV_BAD_PAGE);
+      continue;
+    }
+    const int64_t row =
+        (((int64_t)page * a.num_kv_heads + kvh) * a.block_size + tok % a.block_size) * D + lane * VPL;
+    float kf[VPL], vf[VPL];
+    load_floats<T, VPL>(kc + row, kf);
+    load_floats<T, VPL>(vc + row, vf);
+    float s[GC];
+#pragma unroll
+    for (int g = 0; g < GC; ++g) {
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) acc = fmaf(qv[g][i], kf[i], acc);
+      s[g] = acc;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+      for (int g = 0; g < GC; ++g) s[g] += __shfl_xor_sync(kFull, s[g], off);
+    }
+#pragma unroll
+    for (int g = 0; g < GC; ++g) {
+      const float mn = fmaxf(m[g], s[g]);
+      const float alpha = exp2f(m[g] - mn);
+      const float pr = exp2f(s[g] - mn);
+      l[g] = l[g] * alpha + pr;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) o[g][i] = fmaf(pr, vf[i], o[g][i] * alpha);
+      m[g] = mn;
+    }
+  }
+
+#pragma unroll
+  for (int g = 0; g < GC; ++g) {
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) o_w[(warp * GC + g) * D + lane * VPL + i] = o[g][i];
+    if (lane == 0) {
+      m_w[warp * GC + g] = m[g];
+      l_w[warp * GC + g] = l[g];
+    }
+  }
+  __syncthreads();
+  merge_and_store<T, D>(a, b, h0, nh, p, np, NW, GC, o_w, m_w, l_w);
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core partition kernel.  Grid (num_seqs, num_kv_heads, P); NW warps,
+// each streaming its own contiguous run of 16-token tiles of the partition
+// through STAGES shared-memory buffers.
+//
+// Shared memory per warp and stage: K tile then V tile, [16 rows][D] 16-bit,
+// rows of 2*D bytes; 16-byte chunk c of row r is stored at chunk c ^ (r & 7),
+// so the 8 row addresses of every ldmatrix phase hit 8 distinct bank groups.
+// ---------------------------------------------------------------------------
+template <int D, int NW, int STAGES>
+struct TcShape {
+  static constexpr int kRowBytes = 2 * D;
+  static constexpr int kChunksPerRow = kRowBytes / 16;
+  static constexpr int kTile = 16;
+  static constexpr int kTileBytes = kTile * kRowBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kWarpBytes = STAGES * kStageBytes;
+  static constexpr int kSmemBytes = NW * kWarpBytes;
+  static constexpr int kChunksPerLane = kTile * kChunksPerRow / 32;
+  static_assert(8 * D * 4 + 16 * 4 <= kWarpBytes, "warp region must hold its merge scratch");
+};
+
+template <typename T, int D, int NW, int STAGES>
+__global__ void __launch_bounds__(NW * 32) decode_tc_kernel(const DecodeArgs a) {
+  using S = TcShape<D, NW, STAGES>;
+  constexpr int KSTEPS = D / 16;
+  constexpr int MTILES = D / 16;
+  extern __shared__ __align__(128) uint8_t smem[];
+
+  const int b = blockIdx.x;
+  const int kvh = blockIdx.y;
+  const int p = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2;  // fragment row group
+  const int t = lane & 3;   // fragment column pair
+  const int G = a.group;
+  const int h0 = kvh * G;
+
+  const int ctx = context_of(a, b, threadIdx.x == 0 && kvh == 0 && p == 0);
+  const int np = (ctx + kPartition - 1) / kPartition;
+  if (p >= max(np, 1)) return;
+  if (ctx == 0) {
+    store_zero_rows<T, D>(a, b, h0, G);
+    return;
+  }
+  const int bs = a.block_size;
+  const int tok_begin = p * kPartition;
+  const int tok_end = min(ctx, tok_begin + kPartition);
+  const int ntiles = (tok_end - tok_begin + S::kTile - 1) / S::kTile;
+  const int per_warp = (ntiles + NW - 1) / NW;
+  const int first_tile = warp * per_warp;
+  const int my_tiles = max(0, min(per_warp, ntiles - first_tile));
+
+  // This partition's block-table entries, one per lane (at most 32 since
+  // block_size >= 16); every tile's page is then a register shuffle away.
+  const int first_block = tok_begin / bs;
+  const int nblk = (tok_end - 1) / bs - first_block + 1;
+  int lane_page = 0;
+  if (lane < nblk) lane_page = __ldg(a.block_tables + (int64_t)b * a.max_blocks_per_seq + first_block + lane);
+
+  // Q^T fragments (B operand, k = head_dim, n = query head of the group).
+  uint32_t qf[KSTEPS][2];
+  {
+    const bool real = g < G;
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(reinterpret_cast<const T*>(a.q) +
+                                                             ((int64_t)b * a.num_q_heads + h0 + (real ? g : 0)) * D);
+#pragma unroll
+    for (int ks = 0; ks < KSTEPS; ++ks) {
+      qf[ks][0] = real ? __ldg(qrow + 8 * ks + t) : 0u;
+      qf[ks][1] = real ? __ldg(qrow + 8 * ks + 4 + t) : 0u;
+    }
+  }
+
+  uint8_t* wsm = smem + warp * S::kWarpBytes;
+  const uint32_t wsm_u32 = smem_u32(wsm);
+  const T* kc = reinterpret_cast<const T*>(a.key_cache);
+  const T* vc = reinterpret_cast<const T*>(a.value_cache);
+
+  // Issue the cp.async copies of local tile i into stage `stage`.
+  auto load_tile = [&](int i, int stage) {
+    const int tok0 = tok_begin + (first_tile + i) * S::kTile;
+    int valid = min(S::kTile, tok_end - tok0);
+    int page = __shfl_sync(kFull, lane_page, tok0 / bs - first_block);
+    if ((unsigned)page >= (unsigned)a.num_blocks) {
+      if (lane == 0) flag_status(a.status, PA_DEV_BAD_PAGE);
+      valid = 0;
+      page = 0;
+    }
+    const int64_t row0 = ((int64_t)page * a.num_kv_heads + kvh) * bs + (tok0 % bs);
+    const T* ksrc = kc + row0 * D;
+    const T* vsrc = vc + row0 * D;
+    const uint32_t kdst = wsm_u32 + stage * S::kStageBytes;
+    const uint32_t vdst = kdst + S::kTileBytes;
+#pragma unroll
+    for (int j = 0; j < S::kChunksPerLane; ++j) {
+      const int idx = lane + 32 * j;
+      const int r = idx / S::kChunksPerRow;
+      const int c = idx - r * S::kChunksPerRow;
+      const bool ok = r < valid;
+      const int64_t src = (int64_t)(ok ? r : 0) * D + c * 8;
+      const uint32_t dst = r * S::kRowBytes + ((c ^ (r & 7)) << 4);
+      cp_async_16(kdst + dst, ksrc + src, ok ? 16u : 0u);
+      cp_async_16(vdst + dst, vsrc + src, ok ? 16u : 0u);
+    }
+    return valid;
+  };
+
+  float o[MTILES][4];
+#pragma unroll
+  for (int mt = 0; mt < MTILES; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  float m[2] = {-INFINITY, -INFINITY};  // heads 2t, 2t+1 (base-2 scores)
+  float l[2] = {0.f, 0.f};              // this lane's tokens only; reduced at the end
+
+#pragma unroll
+  for (int i = 0; i < STAGES - 1; ++i) {
+    if (i < my_tiles) load_tile(i, i);
+    cp_async_commit();
+  }
+
+  for (int i = 0; i < my_tiles; ++i) {
+    {
+      const int nxt = i + STAGES - 1;
+      if (nxt < my_tiles) load_tile(nxt, nxt % STAGES);
+      cp_async_commit();
+    }
+    cp_async_wait<STAGES - 1>();
+    __syncwarp();
+
+    const int stage = i % STAGES;
+    const uint32_t kbase = wsm_u32 + stage * S::kStageBytes;
+    const uint32_t vbase = kbase + S::kTileBytes;
+    const int tok0 = tok_begin + (first_tile + i) * S::kTile;
+    int valid = min(S::kTile, tok_end - tok0);
+    {
+      const int page = __shfl_sync(kFull, lane_page, tok0 / bs - first_block);
+      if ((unsigned)page >= (unsigned)a.num_blocks) valid = 0;
+    }
+
+    // S^T = K_tile . Q^T : two accumulator chains over the head_dim k-steps.
+    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+      const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
+      const uint32_t rbase = kbase + r * S::kRowBytes;
+#pragma unroll
+      for (int ks = 0; ks < KSTEPS; ++ks) {
+        const int c = 2 * ks + (lane >> 4);
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(rbase + ((c ^ (r & 7)) << 4), a0, a1, a2, a3);
+        if (ks & 1)
+          mma_16816<T>(s1, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+        else
+          mma_16816<T>(s0, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+      }
+    }
+    // s[0], s[1]: token g, heads 2t, 2t+1; s[2], s[3]: token g + 8.
+    float s[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[e] = (s0[e] + s1[e]) * a.qk_scale_log2;
+    if (g >= valid) s[0] = s[1] = -INFINITY;
+    if (g + 8 >= valid) s[2] = s[3] = -INFINITY;
+
+    float pr[4], alpha[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float mx = fmaxf(s[j], s[2 + j]);
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+      const float mn = fmaxf(m[j], mx);
+      const float base = mn == -INFINITY ? 0.f : mn;
+      alpha[j] = exp2f(m[j] - base);
+      pr[j] = exp2f(s[j] - base);
+      pr[2 + j] = exp2f(s[2 + j] - base);
+      l[j] = l[j] * alpha[j] + pr[j] + pr[2 + j];
+      m[j] = mn;
+    }
+#pragma unroll
+    for (int mt = 0; mt < MTILES; ++mt) {
+      o[mt][0] *= alpha[0];
+      o[mt][1] *= alpha[1];
+      o[mt][2] *= alpha[0];
+      o[mt][3] *= alpha[1];
+    }
+    // P^T as the B operand (k = token, n = head): transpose the two 8x8 halves.
+    const uint32_t pb0 = movmatrix_trans(pack2<T>(pr[0], pr[1]));
+    const uint32_t pb1 = movmatrix_trans(pack2<T>(pr[2], pr[3]));
+
+    // O^T += V_tile^T . P^T, one m16 tile of head_dim at a time.
+    {
+      const int mat = lane >> 3;
+      const int r = (lane & 7) + ((mat >> 1) << 3);
+      const uint32_t rbase = vbase + r * S::kRowBytes;
+#pragma unroll
+      for (int mt = 0; mt < MTILES; ++mt) {
+        const int c = 2 * mt + (mat & 1);
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4_trans(rbase + ((c ^ (r & 7)) << 4), a0, a1, a2, a3);
+        mma_16816<T>(o[mt], a0, a1, a2, a3, pb0, pb1);
+      }
+    }
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+  __syncwarp();
+
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    l[j] += __shfl_xor_sync(kFull, l[j], 4);
+    l[j] += __shfl_xor_sync(kFull, l[j], 8);
+    l[j] += __shfl_xor_sync(kFull, l[j], 16);
+  }
+  // Warp partials into this warp's own region: o[8][D], then m[8], l[8].
+  float* o_w = reinterpret_cast<float*>(wsm);
+  float* ml_w = o_w + 8 * D;
+#pragma unroll
+  for (int mt = 0; mt < MTILES; ++mt) {
+    const int d = 16 * mt + g;
+    o_w[(2 * t) * D + d] = o[mt][0];
+    o_w[(2 * t + 1) * D + d] = o[mt][1];
+    o_w[(2 * t) * D + d + 8] = o[mt][2];
+    o_w[(2 * t + 1) * D + d + 8] = o[mt][3];
+  }
+  if (g == 0) {
+    ml_w[2 * t] = m[0];
+    ml_w[2 * t + 1] = m[1];
+    ml_w[8 + 2 * t] = l[0];
+    ml_w[8 + 2 * t + 1] = l[1];
+  }
+  __syncthreads();
+
+  // Merge the warps: each region is kWarpBytes apart.
+  constexpr int kStrideF = S::kWarpBytes / 4;
+  const float* base_f = reinterpret_cast<const float*>(smem);
+  for (int i = threadIdx.x; i < G * D; i += NW * 32) {
+    const int j = i / D;
+    const int d = i - j * D;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) mx = fmaxf(mx, base_f[w * kStrideF + 8 * D + j]);
+    float lsum = 0.f, osum = 0.f;
+    if (mx != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float c = exp2f(base_f[w * kStrideF + 8 * D + j] - mx);
+        lsum += base_f[w * kStrideF + 8 * D + 8 + j] * c;
+        osum += base_f[w * kStrideF + j * D + d] * c;
+      }
+    }
+    const float res = lsum > 0.f ? osum / lsum : 0.f;
+    const int64_t row = (int64_t)b * a.num_q_heads + h0 + j;
+    if (np <= 1) {
+      reinterpret_cast<T*>(a.out)[row * D + d] = from_float<T>(res);
+    } else {
+      const int64_t part = row * a.max_partitions + p;
+      a.o_part[part * D + d] = res;
+      if (d == 0) {
+        a.m_part[part] = mx == -INFINITY ? -INFINITY : mx * kLn2;
+        a.l_part[part] = lsum;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Log-sum-exp merge of the partitions: one warp per (sequence, query head).
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeArgs a, int num_seqs) {
+  constexpr int VPL = D / 32;
+  const int64_t item = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (item >= (int64_t)num_seqs * a.num_q_heads) return;
+  const int b = (int)(item / a.num_q_heads);
+  const int ctx = context_of(a, b, false);
+  const int np = (ctx + kPartition - 1) / kPartition;
+  if (np <= 1) return;
+  const int64_t base = item * a.max_partitions;
+
+  float mx = -INFINITY;
+  for (int pp = lane; pp < np; pp += 32) mx = fmaxf(mx, a.m_part[base + pp]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
+
+  float acc[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
+  float lsum = 0.f;
+  if (mx != -INFINITY) {
+    for (int p0 = 0; p0 < np; p0 += 32) {
+      float w = 0.f;
+      if (p0 + lane < np) w = a.l_part[base + p0 + lane] * expf(a.m_part[base + p0 + lane] - mx);
+      lsum += w;
+      const int cnt = min(32, np - p0);
+      for (int k = 0; k < cnt; ++k) {
+        const float wk = __shfl_sync(kFull, w, k);
+        const float* src = a.o_part + (base + p0 + k) * D + lane * VPL;
+        if constexpr (VPL % 4 == 0) {
+#pragma unroll
+          for (int v = 0; v < VPL / 4; ++v) {
+            const float4 x = reinterpret_cast<const float4*>(src)[v];
+            acc[4 * v] = fmaf(wk, x.x, acc[4 * v]);
+            acc[4 * v + 1] = fmaf(wk, x.y, acc[4 * v + 1]);
+            acc[4 * v + 2] = fmaf(wk, x.z, acc[4 * v + 2]);
+            acc[4 * v + 3] = fmaf(wk, x.w, acc[4 * v + 3]);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < VPL; ++i) acc[i] = fmaf(wk, src[i], acc[i]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(kFull, lsum, off);
+  T* out = reinterpret_cast<T*>(a.out) + item * D + lane * VPL;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) out[i] = from_float<T>(lsum > 0.f ? acc[i] / lsum : 0.f);
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+std::atomic<int> g_kernel_choice{PA_DECODE_AUTO};
+std::atomic<int> g_tc_warps{4};
+std::atomic<int> g_tc_stages{3};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WorkspaceLayout {
+  size_t o_off, m_off, l_off, total;
+};
+
+WorkspaceLayout workspace_layout(int64_t num_seqs, int64_t num_q_heads, int64_t head_dim, int64_t partitions) {
+  const size_t rows = (size_t)num_seqs * num_q_heads * partitions;
+  WorkspaceLayout w;
+  w.o_off = 0;
+  w.m_off = align256(rows * head_dim * sizeof(float));
+  w.l_off = w.m_off + align256(rows * sizeof(float));
+  w.total = w.l_off + align256(rows * sizeof(float));
+  return w;
+}
+
+// Sets the kernel's dynamic shared-memory limit once per device.
+template <typename Kernel>
+cudaError_t ensure_smem(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+  if (bit && (done.load() & bit)) return cudaSuccess;
+  err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err == cudaSuccess && bit) done.fetch_or(bit);
+  return err;
+}
+
+template <typename T, int D, int NW, int STAGES>
+cudaError_t launch_tc(const DecodeArgs& a, dim3 grid, cudaStream_t stream) {
+  using S = TcShape<D, NW, STAGES>;
+  static std::atomic<uint64_t> done{0};
+  auto kernel = decode_tc_kernel<T, D, NW, STAGES>;
+  cudaError_t err = ensure_smem(kernel, S::kSmemBytes, done);
+  if (err != cudaSuccess) return err;
+  kernel<<<grid, NW * 32, S::kSmemBytes, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_tc_config(const DecodeArgs& a, dim3 grid, cudaStream_t stream, int warps, int stages) {
+  if (warps == 4 && stages == 3) return launch_tc<T, D, 4, 3>(a, grid, stream);
+  if (warps == 4 && stages == 2) return launch_tc<T, D, 4, 2>(a, grid, stream);
+  if (warps == 4 && stages == 4) return launch_tc<T, D, 4, 4>(a, grid, stream);
+  if (warps == 2 && stages == 4) return launch_tc<T, D, 2, 4>(a, grid, stream);
+  if (warps == 8 && stages == 2) return launch_tc<T, D, 8, 2>(a, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+template <typename T>
+cudaError_t launch_tc_dim(const DecodeArgs& a, int head_dim, dim3 grid, cudaStream_t stream, int warps,
+                          int stages) {
+  switch (head_dim) {
+    case 64: return launch_tc_config<T, 64>(a, grid, stream, warps, stages);
+    case 128: return launch_tc_config<T, 128>(a, grid, stream, warps, stages);
+    case 256:
+      // 256-wide rows: keep to configurations within the shared-memory limit.
+      if (warps * stages * 16384 > 200 * 1024) return cudaErrorInvalidValue;
+      return launch_tc_config<T, 256>(a, grid, stream, warps, stages);
+  }
+  return cudaErrorInvalidValue;
+}
+
+constexpr int kCcHeads = 4;
+constexpr int kCcWarps = 4;
+
+template <typename T>
+cudaError_t launch_cc(const DecodeArgs& a, int head_dim, int num_seqs, int partitions, cudaStream_t stream) {
+  const int chunks = (a.group + kCcHeads - 1) / kCcHeads;
+  dim3 grid(num_seqs, a.num_kv_heads * chunks, partitions);
+  switch (head_dim) {
+    case 64: decode_cc_kernel<T, 64, kCcHeads, kCcWarps><<<grid, kCcWarps * 32, 0, stream>>>(a); break;
+    case 128: decode_cc_kernel<T, 128, kCcHeads, kCcWarps><<<grid, kCcWarps * 32, 0, stream>>>(a); break;
+    case 256: decode_cc_kernel<T, 256, kCcHeads, kCcWarps><<<grid, kCcWarps * 32, 0, stream>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_reduce(const DecodeArgs& a, int head_dim, int num_seqs, cudaStream_t stream) {
+  const int64_t items = (int64_t)num_seqs * a.num_q_heads;
+  const unsigned grid = (unsigned)((items + 3) / 4);
+  switch (head_dim) {
+    case 64: decode_reduce_kernel<T, 64><<<grid, 128, 0, stream>>>(a, num_seqs); break;
+    case 128: decode_reduce_kernel<T, 128><<<grid, 128, 0, stream>>>(a, num_seqs); break;
+    case 256: decode_reduce_kernel<T, 256><<<grid, 128, 0, stream>>>(a, num_seqs); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+bool tc_supported(pa_dtype dt, int head_dim, int group, int block_size) {
+  return (dt == PA_BF16 || dt == PA_F16) && (head_dim == 64 || head_dim == 128 || head_dim == 256) &&
+         group >= 1 && group <= 8 && block_size % 16 == 0 && block_size <= 256;
+}
+
+}  // namespace
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" pa_status pa_set_decode_kernel(pa_decode_kernel k) {
+  if (k != PA_DECODE_AUTO && k != PA_DECODE_CUDA_CORES && k != PA_DECODE_TENSOR_CORES)
+    return fail(PA_ERR_INVALID, "pa_set_decode_kernel: unknown kernel %d", (int)k);
+  g_kernel_choice.store((int)k);
+  return PA_OK;
+}
+
+extern "C" pa_status pa_set_decode_tiling(int32_t warps, int32_t stages) {
+  const bool ok = (warps == 4 && (stages == 2 || stages == 3 || stages == 4)) || (warps == 2 && stages == 4) ||
+                  (warps == 8 && stages == 2);
+  if (!ok) return fail(PA_ERR_UNSUPPORTED, "pa_set_decode_tiling: (%d warps, %d stages) not built", warps, stages);
+  g_tc_warps.store(warps);
+  g_tc_stages.store(stages);
+  return PA_OK;
+}
+
+extern "C" size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                           int64_t max_context_len) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0) return 0;
+  const int64_t partitions = (max_context_len + kPartition - 1) / kPartition;
+  if (partitions <= 1) return 0;
+  return workspace_layout(num_seqs, num_q_heads, head_dim, partitions).total;
+}
+
+namespace {
+
+// Validates a decode call and fills `a`; *partitions receives P.
+pa_status prepare_decode(const void* q, const void* key_cache, const void* value_cache, const int32_t* block_tables,
+                         int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t num_seqs,
+                         int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                         int32_t num_blocks, float scale, void* out, pa_dtype dtype, void* workspace,
+                         size_t workspace_bytes, int32_t* dev_status, DecodeArgs& a, int& partitions) {
+  if (dtype_bytes(dtype) == 0) return fail(PA_ERR_INVALID, "decode: bad dtype %d", (int)dtype);
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0)
+    return fail(PA_ERR_INVALID, "decode: num_q_heads must be a positive multiple of num_kv_heads");
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256)
+    return fail(PA_ERR_UNSUPPORTED, "decode: head_dim %d (supported: 64, 128, 256)", head_dim);
+  if (block_size < 1 || block_size > 256) return fail(PA_ERR_UNSUPPORTED, "decode: block_size %d", block_size);
+  if (max_blocks_per_seq < 1 || num_blocks < 1) return fail(PA_ERR_INVALID, "decode: empty table or pool");
+  if ((int64_t)max_blocks_per_seq * block_size > (1 << 30))
+    return fail(PA_ERR_UNSUPPORTED, "decode: max_blocks_per_seq * block_size above 2^30");
+  if (num_kv_heads > 65535) return fail(PA_ERR_UNSUPPORTED, "decode: too many kv heads");
+  if (!(scale == scale)) return fail(PA_ERR_INVALID, "decode: scale is NaN");
+  const int64_t max_ctx = (int64_t)max_blocks_per_seq * block_size;
+  partitions = (int)((max_ctx + kPartition - 1) / kPartition);
+  if (partitions > 65535) return fail(PA_ERR_UNSUPPORTED, "decode: more than 65535 partitions");
+  if (num_seqs == 0) return PA_OK;
+  if (!q || !key_cache || !value_cache || !block_tables || !context_lens || !out)
+    return fail(PA_ERR_INVALID, "decode: NULL pointer");
+  if (!aligned16(q) || !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(out))
+    return fail(PA_ERR_INVALID, "decode: q, caches and out must be 16-byte aligned");
+  a = DecodeArgs{};
+  a.q = q;
+  a.key_cache = key_cache;
+  a.value_cache = value_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.out = out;
+  a.status = dev_status;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.group = num_q_heads / num_kv_heads;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.max_partitions = partitions;
+  a.qk_scale_log2 = scale * kLog2e;
+  if (partitions > 1) {
+    const WorkspaceLayout w = workspace_layout(num_seqs, num_q_heads, head_dim, partitions);
+    if (!workspace || workspace_bytes < w.total)
+      return fail(PA_ERR_INVALID, "decode: workspace of %zu bytes needed, %zu given", w.total, workspace_bytes);
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+      return fail(PA_ERR_INVALID, "decode: workspace must be 256-byte aligned");
+    char* ws = static_cast<char*>(workspace);
+    a.o_part = reinterpret_cast<float*>(ws + w.o_off);
+    a.m_part = reinterpret_cast<float*>(ws + w.m_off);
+    a.l_part = reinterpret_cast<float*>(ws + w.l_off);
+  }
+  return PA_OK;
+}
+
+pa_status launch_partitions(const DecodeArgs& a, pa_dtype dtype, int head_dim, int num_seqs, int partitions,
+                            cudaStream_t s) {
+  const int choice = g_kernel_choice.load();
+  const bool tc_ok = tc_supported(dtype, head_dim, a.group, a.block_size);
+  if (choice == PA_DECODE_TENSOR_CORES && !tc_ok)
+    return fail(PA_ERR_UNSUPPORTED, "decode: tensor-core kernel needs bf16/f16, G <= 8, block_size %% 16 == 0");
+  cudaError_t err;
+  if (tc_ok && choice != PA_DECODE_CUDA_CORES) {
+    dim3 grid(num_seqs, a.num_kv_heads, partitions);
+    const int warps = g_tc_warps.load(), stages = g_tc_stages.load();
+    err = dtype == PA_BF16 ? launch_tc_dim<__nv_bfloat16>(a, head_dim, grid, s, warps, stages)
+                           : launch_tc_dim<__half>(a, head_dim, grid, s, warps, stages);
+  } else {
+    err = dtype == PA_F32    ? launch_cc<float>(a, head_dim, num_seqs, partitions, s)
+          : dtype == PA_BF16 ? launch_cc<__nv_bfloat16>(a, head_dim, num_seqs, partitions, s)
+                             : launch_cc<__half>(a, head_dim, num_seqs, partitions, s);
+  }
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode partition kernel: %s", cudaGetErrorString(err));
+  return PA_OK;
+}
+
+pa_status launch_reduce_any(const DecodeArgs& a, pa_dtype dtype, int head_dim, int num_seqs, cudaStream_t s) {
+  const cudaError_t err = dtype == PA_F32    ? launch_reduce<float>(a, head_dim, num_seqs, s)
+                          : dtype == PA_BF16 ? launch_reduce<__nv_bfloat16>(a, head_dim, num_seqs, s)
+                                             : launch_reduce<__half>(a, head_dim, num_seqs, s);
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode reduce kernel: %s", cudaGetErrorString(err));
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode(const void* q, const void* key_cache, const void* value_cache,
+                               const int32_t* block_tables, int32_t max_blocks_per_seq,
+                               const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                               int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                               float scale, void* out, pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                               int32_t* dev_status, void* stream) {
+  DecodeArgs a;
+  int partitions = 0;
+  pa_status st = prepare_decode(q, key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                                num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, out, dtype,
+                                workspace, workspace_bytes, dev_status, a, partitions);
+  if (st != PA_OK || num_seqs == 0) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_partitions(a, dtype, head_dim, num_seqs, partitions, s);
+  if (st != PA_OK || partitions <= 1) return st;
+  return launch_reduce_any(a, dtype, head_dim, num_seqs, s);
+}
+
+extern "C" pa_status pa_decode_partitions(const void* q, const void* key_cache, const void* value_cache,
+                                          const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                          const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                                          int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                          int32_t num_blocks, float scale, void* out, pa_dtype dtype,
+                                          void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                          void* stream) {
+  DecodeArgs a;
+  int partitions = 0;
+  pa_status st = prepare_decode(q, key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                                num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, out, dtype,
+                                workspace, workspace_bytes, dev_status, a, partitions);
+  if (st != PA_OK || num_seqs == 0) return st;
+  return launch_partitions(a, dtype, head_dim, num_seqs, partitions, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" pa_status pa_decode_reduce(const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                                      int32_t head_dim, int64_t max_context_len, void* out, pa_dtype dtype,
+                                      const void* workspace, size_t workspace_bytes, void* stream) {
+  if (dtype_bytes(dtype) == 0) return fail(PA_ERR_INVALID, "decode_reduce: bad dtype %d", (int)dtype);
+  if (num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0 || max_context_len > (1 << 30))
+    return fail(PA_ERR_INVALID, "decode_reduce: bad sizes");
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256)
+    return fail(PA_ERR_UNSUPPORTED, "decode_reduce: head_dim %d", head_dim);
+  const int partitions = (int)((max_context_len + kPartition - 1) / kPartition);
+  if (num_seqs == 0 || partitions <= 1) return PA_OK;
+  if (!context_lens || !out) return fail(PA_ERR_INVALID, "decode_reduce: NULL pointer");
+  if (!aligned16(out)) return fail(PA_ERR_INVALID, "decode_reduce: out must be 16-byte aligned");
+  const WorkspaceLayout w = workspace_layout(num_seqs, num_q_heads, head_dim, partitions);
+  if (!workspace || workspace_bytes < w.total)
+    return fail(PA_ERR_INVALID, "decode_reduce: workspace of %zu bytes needed, %zu given", w.total, workspace_bytes);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+    return fail(PA_ERR_INVALID, "decode_reduce: workspace must be 256-byte aligned");
+  DecodeArgs a{};
+  a.context_lens = context_lens;
+  a.out = out;
+  a.num_q_heads = num_q_heads;
+  a.max_blocks_per_seq = (int)max_context_len;
+  a.block_size = 1;
+  a.max_partitions = partitions;
+  char* ws = static_cast<char*>(const_cast<void*>(workspace));
+  a.o_part = reinterpret_cast<float*>(ws + w.o_off);
+  a.m_part = reinterpret_cast<float*>(ws + w.m_off);
+  a.l_part = reinterpret_cast<float*>(ws + w.l_off);
+  return launch_reduce_any(a, dtype, head_dim, num_seqs, static_cast<cudaStream_t>(stream));
+}

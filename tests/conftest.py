@@ -8,6 +8,12 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def pytest_sessionstart(session):
+    # Build libpa_b200.so in-tree if its sources changed (no-op otherwise).
+    from paged_kv_cache_356_b200 import build
+    build.build()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a); run with -m gpu")
     config.addinivalue_line("markers", "slow: full-size workload on the GPU")
