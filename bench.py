@@ -51,6 +51,7 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle time budget for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true", help="skip the nvidia-smi clock record (profiler runs)")
     return ap.parse_args(argv)
 
 
@@ -334,9 +335,11 @@ def run_ours(args):
         step()
     torch.cuda.synchronize()
 
-    sampler = ClockSampler(gpu_smi_id(torch, local))
-    sampler.start()
-    time.sleep(0.3)
+    sampler = None
+    if not args.no_clocks:
+        sampler = ClockSampler(gpu_smi_id(torch, local))
+        sampler.start()
+        time.sleep(0.3)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
@@ -347,13 +350,16 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     total_ms = evs[0][0].elapsed_time(evs[-1][3])
-    # keep identical steps running until the clock record spans at least ~1.5 s under load
-    soak_until = time.perf_counter() + max(0.0, 1.5 - total_ms / 1000)
-    while time.perf_counter() < soak_until:
-        for _ in range(20):
-            step()
-        torch.cuda.synchronize()
-    clocks = sampler.stop()
+    clocks = None
+    if sampler is not None:
+        # keep identical steps running until the clock record spans at least ~1.5 s under load
+        soak_until = time.perf_counter() + max(0.0, 1.5 - total_ms / 1000)
+        while time.perf_counter() < soak_until:
+            for _ in range(20):
+                step()
+            torch.cuda.synchronize()
+        clocks = sampler.stop()
+        clocks["window"] = "timed region, extended by identical steps to >= 1.5 s of samples"
 
     write_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     part_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps

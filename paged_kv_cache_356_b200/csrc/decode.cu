@@ -21,7 +21,8 @@
 //                        S^T[16 tok x 8 heads] = K_tile[16 x D] . Q^T[D x 8]
 //                        O^T[D x 8 heads]     += V_tile^T[D x 16] . P^T[16 x 8]
 //                      (tokens on M, the GQA group on N -- no padded rows);
-//                      P^T is re-laid out between the two with movmatrix.
+//                      P^T is re-laid out between the two with movmatrix and
+//                      fed as a 16-bit high part plus its rounding residual.
 //   decode_cc_kernel   (any dtype incl. fp32, any block size): CUDA cores, one
 //                      token per warp step, lanes split head_dim.
 // Both keep an online softmax (running max m, running sum l, fp32) per head,
@@ -407,11 +408,19 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(const DecodeArgs a) 
       o[mt][2] *= alpha[0];
       o[mt][3] *= alpha[1];
     }
-    // P^T as the B operand (k = token, n = head): transpose the two 8x8 halves.
-    const uint32_t pb0 = movmatrix_trans(pack2<T>(pr[0], pr[1]));
-    const uint32_t pb1 = movmatrix_trans(pack2<T>(pr[2], pr[3]));
+    // P^T as the B operand (k = token, n = head), split into a 16-bit high
+    // part and the 16-bit rounding residual (P = P_hi + P_lo to ~2^-17), so
+    // the weights lose nothing to the 16-bit operand format; each 8x8 half is
+    // transposed into the B layout with movmatrix.
+    const uint32_t hi0 = pack2<T>(pr[0], pr[1]);
+    const uint32_t hi1 = pack2<T>(pr[2], pr[3]);
+    const float2 r0 = unpack2<T>(hi0), r1 = unpack2<T>(hi1);
+    const uint32_t lo0 = pack2<T>(pr[0] - r0.x, pr[1] - r0.y);
+    const uint32_t lo1 = pack2<T>(pr[2] - r1.x, pr[3] - r1.y);
+    const uint32_t pb0 = movmatrix_trans(hi0), pb1 = movmatrix_trans(hi1);
+    const uint32_t pl0 = movmatrix_trans(lo0), pl1 = movmatrix_trans(lo1);
 
-    // O^T += V_tile^T . P^T, one m16 tile of head_dim at a time.
+    // O^T += V_tile^T . (P_hi^T + P_lo^T), one m16 tile of head_dim at a time.
     {
       const int mat = lane >> 3;
       const int r = (lane & 7) + ((mat >> 1) << 3);
@@ -422,6 +431,7 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(const DecodeArgs a) 
         uint32_t a0, a1, a2, a3;
         ldmatrix_x4_trans(rbase + ((c ^ (r & 7)) << 4), a0, a1, a2, a3);
         mma_16816<T>(o[mt], a0, a1, a2, a3, pb0, pb1);
+        mma_16816<T>(o[mt], a0, a1, a2, a3, pl0, pl1);
       }
     }
     __syncwarp();

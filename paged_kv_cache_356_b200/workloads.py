@@ -198,13 +198,14 @@ class Workload:
 
 
 def _independent_trace(context_lens) -> Tuple[tuple, ...]:
-    """Prefill ctx-1 tokens per sequence, then append and write the new token.
+    """Admit every sequence with ctx-1 tokens, prefill them, then append and write the new token.
 
     A sequence of context 0 is admitted empty and never written.
     """
     ops = []
     for b, ctx in enumerate(context_lens):
         ops.append(("allocate", b, max(ctx - 1, 0)))
+    for b, ctx in enumerate(context_lens):
         if ctx - 1 > 0:
             ops.append(("write", b, 0, ctx - 1))
     for b, ctx in enumerate(context_lens):
