@@ -47,7 +47,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama70b", choices=["llama8b", "llama70b", "prefix", "beam32k"])
     ap.add_argument("--kernel", default="auto", choices=["auto", "tc", "cc"])
-    ap.add_argument("--tiling", default="4x3", help="tensor-core kernel warps x stages")
+    ap.add_argument("--tiling", default="4x2", help="tensor-core kernel warps x stages")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle time budget for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

@@ -195,7 +195,8 @@ PA_API pa_status pa_set_decode_kernel(pa_decode_kernel kernel);
 
 /* Tiling of the tensor-core kernel (process-wide): warps per CTA and
  * shared-memory pipeline stages per warp.  Built: (4,2) (4,3) (4,4) (2,4)
- * (8,2); default (4,3).  Others return PA_ERR_UNSUPPORTED.  For tuning. */
+ * (8,2); default (4,2): three 64 KB CTAs per SM keep more bytes in flight
+ * than deeper per-warp pipelines.  Others return PA_ERR_UNSUPPORTED. */
 PA_API pa_status pa_set_decode_tiling(int32_t warps, int32_t stages);
 
 /* ------------------------------------------------------------------------

@@ -558,7 +558,7 @@ __global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeArgs a, 
 // ---------------------------------------------------------------------------
 std::atomic<int> g_kernel_choice{PA_DECODE_AUTO};
 std::atomic<int> g_tc_warps{4};
-std::atomic<int> g_tc_stages{3};
+std::atomic<int> g_tc_stages{2};
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 

@@ -27,7 +27,7 @@ KERNELS = {"tc": pa.PA_DECODE_TENSOR_CORES, "cc": pa.PA_DECODE_CUDA_CORES, "auto
 def _reset_kernel():
     yield
     pa.pa_set_decode_kernel(pa.PA_DECODE_AUTO)
-    pa.pa_set_decode_tiling(4, 3)
+    pa.pa_set_decode_tiling(4, 2)
 
 
 def _values(rng, n, dtype):

@@ -38,7 +38,7 @@ def _sampled_reference(w, seqs, heads=None):
 def full_run(request):
     import torch
     pa.pa_set_decode_kernel(pa.PA_DECODE_AUTO)
-    pa.pa_set_decode_tiling(4, 3)
+    pa.pa_set_decode_tiling(4, 2)
     w = workloads.by_name(request.param)
     run = TraceRunner(w)
     out = run.run()
