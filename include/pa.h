@@ -180,6 +180,40 @@ PA_API pa_status pa_decode_reduce(const int32_t* context_lens, int32_t num_seqs,
                                   int32_t head_dim, int64_t max_context_len, void* out, pa_dtype dtype,
                                   const void* workspace, size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * pa_decode_fixed_scratch -- pa_decode for callers that cannot allocate
+ * device memory.  (The pages have no counterpart: this is a deployment
+ * convenience of this library.)
+ *
+ * Some callers may not call cudaMalloc or any allocating routine on their
+ * own: a plugin running inside an engine whose memory planner owns every
+ * device allocation, or a serving loop that fixes its memory footprint at
+ * start-up and forbids allocation on the decode path.  They still pass their
+ * inputs and outputs, but no workspace: the split-context partials go to a
+ * library-owned device array of PA_FIXED_SCRATCH_BYTES (32 MiB), which every
+ * GPU that loads the library holds until the process exits.
+ *
+ * Arguments, results and errors are those of pa_decode, minus workspace.
+ * A call whose partials would exceed PA_FIXED_SCRATCH_BYTES (that is, when
+ * pa_decode_workspace_size(num_seqs, num_q_heads, head_dim,
+ * max_blocks_per_seq * block_size) > PA_FIXED_SCRATCH_BYTES) returns
+ * PA_ERR_INVALID without launching anything; use pa_decode for it.
+ * The first call on each device does a one-time set-up (it looks up the
+ * array's device address with that device current); make that first call
+ * before any stream capture.  The call allocates nothing and frees nothing.
+ * Every call shares the one array and leaves its contents behind; nothing in
+ * it needs to start at zero (each call writes every partial it later reads),
+ * but calls that overlap on the GPU (on different streams, or from several
+ * threads) race on it and must be serialised by the caller.
+ * ---------------------------------------------------------------------- */
+#define PA_FIXED_SCRATCH_BYTES (32 * 1024 * 1024)
+PA_API pa_status pa_decode_fixed_scratch(const void* q, const void* key_cache, const void* value_cache,
+                                         const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                         const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                                         int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                         int32_t num_blocks, float scale, void* out, pa_dtype dtype,
+                                         int32_t* dev_status, void* stream);
+
 /* Which partition kernel pa_decode runs (process-wide; default AUTO).
  * AUTO picks the tensor-core kernel whenever it supports the call (bf16/f16,
  * head_dim 64/128/256, G <= 8, block_size a multiple of 16 up to 256) and the

@@ -15,6 +15,7 @@ PA_F32, PA_BF16, PA_F16 = 0, 1, 2
 PA_DEV_BAD_SLOT, PA_DEV_BAD_PAGE, PA_DEV_BAD_CTX, PA_DEV_BAD_PAIR = 1, 2, 4, 8
 PA_DECODE_AUTO, PA_DECODE_CUDA_CORES, PA_DECODE_TENSOR_CORES = 0, 1, 2
 PA_PARTITION_TOKENS = 512
+PA_FIXED_SCRATCH_BYTES = 32 * 1024 * 1024
 
 _c = ctypes
 _vp, _i32, _i64, _f32, _sz = _c.c_void_p, _c.c_int32, _c.c_int64, _c.c_float, _c.c_size_t
@@ -33,6 +34,8 @@ SIGNATURES = {
     "pa_decode_partitions": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp,
                                     _i32, _vp, _sz, _vp, _vp]),
     "pa_decode_reduce": (_i32, [_vp, _i32, _i32, _i32, _i64, _vp, _i32, _vp, _sz, _vp]),
+    "pa_decode_fixed_scratch": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
+                                       _vp, _i32, _vp, _vp]),
     "pa_set_decode_kernel": (_i32, [_i32]),
     "pa_set_decode_tiling": (_i32, [_i32, _i32]),
     "pa_block_alloc_create": (_i32, [_i32, _i32, _pi32, _c.POINTER(_vp)]),

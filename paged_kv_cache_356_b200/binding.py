@@ -183,6 +183,33 @@ def pa_decode_reduce(context_lens, max_context_len: int, out, workspace, stream=
     return out
 
 
+def pa_decode_fixed_scratch(q, key_cache, value_cache, block_tables, context_lens, scale: float, out,
+                            dev_status=None, stream=None):
+    """pa_decode without a workspace argument, for callers that may not allocate device memory.
+
+    Nothing is allocated here or in the library: ``out`` is the caller's, and
+    the split-context partials use the library's fixed 32 MiB device array
+    (calls needing more are rejected).  Calls that overlap on the GPU race on
+    that array.  The first call on a device does a one-time set-up: make it
+    before any stream capture.
+    """
+    torch = _torch()
+    nb, hkv, bs, d = _cache_shape(key_cache, value_cache)
+    if q.dim() != 3 or q.shape[2] != d or q.dtype != key_cache.dtype:
+        raise ValueError("q must be [num_seqs, num_q_heads, head_dim] of the cache dtype")
+    if out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("out must match q")
+    num_seqs, hq = int(q.shape[0]), int(q.shape[1])
+    if block_tables.dim() != 2 or block_tables.shape[0] != num_seqs or context_lens.shape != (num_seqs,):
+        raise ValueError("block_tables must be [num_seqs, max_blocks_per_seq], context_lens [num_seqs]")
+    _check(_lib.load().pa_decode_fixed_scratch(
+        _cuda(q, "q"), _cuda(key_cache, "key_cache"), _cuda(value_cache, "value_cache"),
+        _cuda(block_tables, "block_tables", torch.int32), int(block_tables.shape[1]),
+        _cuda(context_lens, "context_lens", torch.int32), num_seqs, hq, hkv, d, bs, nb, float(scale),
+        _cuda(out, "out"), dtype_code(q.dtype), _opt_status(dev_status), _stream_handle(stream, q.device)))
+    return out
+
+
 def pa_set_decode_kernel(kernel: int) -> None:
     _check(_lib.load().pa_set_decode_kernel(int(kernel)))
 

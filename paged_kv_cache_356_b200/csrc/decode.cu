@@ -33,6 +33,7 @@
 #include <math.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "device.cuh"
 #include "pa_internal.h"
@@ -838,4 +839,65 @@ extern "C" pa_status pa_decode_reduce(const int32_t* context_lens, int32_t num_s
   a.m_part = reinterpret_cast<float*>(ws + w.m_off);
   a.l_part = reinterpret_cast<float*>(ws + w.l_off);
   return launch_reduce_any(a, dtype, head_dim, num_seqs, static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------------------
+// pa_decode_fixed_scratch: pa_decode for callers that cannot allocate device
+// memory themselves.  The split-context partials go to a file-scope device
+// array owned by the library instead of a caller-provided workspace.
+// ---------------------------------------------------------------------------
+namespace {
+
+// Part of the loaded module: every GPU that loads this library holds these
+// PA_FIXED_SCRATCH_BYTES until the process exits.  Host code must not use the
+// symbol's name as an address (it is a host-side stand-in); it takes the
+// device address from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_fixed_scratch[PA_FIXED_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_fixed_scratch_mutex;
+void* g_fixed_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_fixed_scratch on the current device, looked up once per
+// device (with that device current) and cached.
+pa_status fixed_scratch_address(void** addr) {
+  int dev = -1;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode_fixed_scratch: cudaGetDevice: %s", cudaGetErrorString(err));
+  if (dev < 0 || dev >= kMaxDevices) return fail(PA_ERR_UNSUPPORTED, "decode_fixed_scratch: device %d", dev);
+  std::lock_guard<std::mutex> lock(g_fixed_scratch_mutex);
+  if (!g_fixed_scratch_addr[dev]) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_fixed_scratch);
+    if (err != cudaSuccess || !p)
+      return fail(PA_ERR_CUDA, "decode_fixed_scratch: cudaGetSymbolAddress: %s", cudaGetErrorString(err));
+    g_fixed_scratch_addr[dev] = p;
+  }
+  *addr = g_fixed_scratch_addr[dev];
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_fixed_scratch(const void* q, const void* key_cache, const void* value_cache,
+                                             const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                             const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                                             int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                             int32_t num_blocks, float scale, void* out, pa_dtype dtype,
+                                             int32_t* dev_status, void* stream) {
+  void* scratch = nullptr;
+  pa_status st = fixed_scratch_address(&scratch);  // first call on a device: the one-time set-up
+  if (st != PA_OK) return st;
+  if (max_blocks_per_seq > 0 && block_size > 0 && num_seqs > 0 && num_q_heads > 0 && head_dim > 0) {
+    const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim,
+                                                 (int64_t)max_blocks_per_seq * block_size);
+    if (need > (size_t)PA_FIXED_SCRATCH_BYTES)
+      return fail(PA_ERR_INVALID,
+                  "decode_fixed_scratch: this call needs %zu bytes of scratch, more than the fixed %zu-byte array; "
+                  "use pa_decode with a caller-provided workspace",
+                  need, (size_t)PA_FIXED_SCRATCH_BYTES);
+  }
+  return pa_decode(q, key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs, num_q_heads,
+                   num_kv_heads, head_dim, block_size, num_blocks, scale, out, dtype, scratch,
+                   (size_t)PA_FIXED_SCRATCH_BYTES, dev_status, stream);
 }
