@@ -52,6 +52,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true", help="skip the nvidia-smi clock record (profiler runs)")
+    ap.add_argument("--shared-prefix", choices=["auto", "on", "off"], default="auto",
+                    help="decode shared leading pages once per group (auto: on for prefix/beam32k)")
     return ap.parse_args(argv)
 
 
@@ -304,7 +306,8 @@ def run_ours(args):
 
     seed_shift = 1000 * rank
     w = workloads.by_name(args.workload, seed=workloads.by_name(args.workload).seed + seed_shift)
-    run = TraceRunner(w)
+    shared = args.shared_prefix == "on" or (args.shared_prefix == "auto" and w.kind in ("prefix", "beam"))
+    run = TraceRunner(w, shared_prefix=shared)
     run.run(decode=False)
     torch.cuda.synchronize()
     if run.status() != 0:
@@ -323,11 +326,17 @@ def run_ours(args):
         pa.pa_reshape_and_cache(kd, vd, sd, run.key_cache, run.value_cache, stream=stream)
         if evs is not None:
             evs[1].record(stream)
-        pa.pa_decode_partitions(run.q, run.key_cache, run.value_cache, run.block_tables, run.context_lens, w.scale,
-                                run.out, run.workspace, stream=stream)
-        if evs is not None:
-            evs[2].record(stream)
-        pa.pa_decode_reduce(run.context_lens, max_ctx, run.out, run.workspace, stream=stream)
+        if run.plan is not None:     # joint + per-sequence partition kernels and the merge, one call
+            pa.pa_decode_shared_prefix(run.q, run.key_cache, run.value_cache, run.block_tables, run.context_lens,
+                                       w.scale, run.plan, out=run.out, workspace=run.workspace, stream=stream)
+            if evs is not None:
+                evs[2].record(stream)
+        else:
+            pa.pa_decode_partitions(run.q, run.key_cache, run.value_cache, run.block_tables, run.context_lens,
+                                    w.scale, run.out, run.workspace, stream=stream)
+            if evs is not None:
+                evs[2].record(stream)
+            pa.pa_decode_reduce(run.context_lens, max_ctx, run.out, run.workspace, stream=stream)
         if evs is not None:
             evs[3].record(stream)
 
@@ -405,14 +414,19 @@ def run_ours(args):
             "seqs_per_s": seqs_per_s,
             "kv_bytes_per_step": {"unique": unique, "logical": logical},
             "frac_of_hbm": {"measured": value / world / peak, "nominal_8000": value / world / NOMINAL_HBM_GBS},
-            "kernel_ms": {"reshape_and_cache": write_ms, "decode_partitions": part_ms, "decode_reduce": reduce_ms},
+            "kernel_ms": ({"reshape_and_cache": write_ms, "decode_partitions": part_ms, "decode_reduce": reduce_ms}
+                          if run.plan is None else
+                          {"reshape_and_cache": write_ms, "decode_shared_prefix (joint + per-sequence + merge)": part_ms}),
+            "shared_prefix_plan": (None if run.plan is None else
+                                   {"chunks": run.plan["num_chunks"], "members": run.plan["num_members"],
+                                    "shared_partitions": run.plan["max_shared_partitions"]}),
             "roofline": {"bound": "hbm", "kernel": "decode_tc_kernel (pa_decode_partitions)",
                          "achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} (copy bandwidth)",
                          "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                          "algorithmic_bytes_per_launch": part_bytes, "kernel_source_sha256": khash},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": (4 if run.plan is not None and run.plan["num_chunks"] > 0 else 3) * args.steps,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -449,7 +463,12 @@ def end_to_end(args, torch, pa, run, w, unique, max_ctx, world, dist):
         for dst, src in ((d_q, h_q), (d_k, h_k), (d_v, h_v), (d_s, h_s), (d_tab, h_tab), (d_ctx, h_ctx)):
             dst.copy_(src, non_blocking=True)
         pa.pa_reshape_and_cache(d_k, d_v, d_s, run.key_cache, run.value_cache)
-        pa.pa_decode(d_q, run.key_cache, run.value_cache, d_tab, d_ctx, w.scale, out=d_out, workspace=run.workspace)
+        if run.plan is not None:
+            pa.pa_decode_shared_prefix(d_q, run.key_cache, run.value_cache, d_tab, d_ctx, w.scale, run.plan,
+                                       out=d_out, workspace=run.workspace)
+        else:
+            pa.pa_decode(d_q, run.key_cache, run.value_cache, d_tab, d_ctx, w.scale, out=d_out,
+                         workspace=run.workspace)
         h_out.copy_(d_out, non_blocking=True)
         torch.cuda.current_stream().synchronize()
 

@@ -66,6 +66,7 @@ typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1, PA_F16 = 2 } pa_dtype;
 #define PA_DEV_BAD_PAGE 2 /* decode: a block-table entry the context needs is outside the pool */
 #define PA_DEV_BAD_CTX 4  /* decode: context_len < 0 or > max_blocks_per_seq * block_size  */
 #define PA_DEV_BAD_PAIR 8 /* copy_blocks: a source or destination page is outside the pool  */
+#define PA_DEV_BAD_PLAN 16 /* decode_shared_prefix: a prefix-plan entry is out of range       */
 
 /* Tokens per split-context partition of pa_decode. */
 #define PA_PARTITION_TOKENS 512
@@ -214,6 +215,49 @@ PA_API pa_status pa_decode_fixed_scratch(const void* q, const void* key_cache, c
                                          int32_t num_blocks, float scale, void* out, pa_dtype dtype,
                                          int32_t* dev_status, void* stream);
 
+/* ------------------------------------------------------------------------
+ * pa_decode_shared_prefix -- pa_decode for a batch in which groups of
+ * sequences share leading pages (forked beams, a common system prompt).
+ *
+ * [Internals] "Copy-on-Write and Prefix Sharing": many requests point at
+ * the same physical pages for a shared prefix; [Glossary] "Enterprise Use
+ * Cases": 8 beams sharing a 32k-token prompt.  Sharing saves memory on the
+ * pages; here it also saves bandwidth: every whole 512-token partition that
+ * all members of a group share is read once, by one CTA serving up to
+ * PA_PREFIX_QUERIES_PER_CTA queries (members x query heads of one kv head),
+ * instead of once per sequence.  The result is the same as pa_decode's.
+ *
+ * The plan arrays (device, int32) come from pa_block_alloc_prefix_plan for
+ * the same allocator state and batch order:
+ *   first_partition [num_seqs]       partitions [0, first) of sequence b are
+ *                                    computed by the joint kernel;
+ *   chunks          [num_chunks][4]  (leader, member offset, member count,
+ *                                    shared partitions) -- the leader's table
+ *                                    row addresses the shared pages;
+ *   members         [num_members]    batch indices of each chunk's members;
+ *   max_shared_partitions / min_shared_partitions: the largest / smallest
+ *                                    first_partition of the batch (no
+ *                                    per-sequence CTA is launched below the
+ *                                    smallest).
+ * A workspace is always required when max_blocks_per_seq * block_size >
+ * PA_PARTITION_TOKENS.  Plan entries out of range are skipped and flagged
+ * PA_DEV_BAD_PLAN; an inconsistent plan gives wrong results but never
+ * touches memory outside the arrays.  Shapes the joint kernel does not
+ * support (fp32, head_dim 256, block_size not a multiple of 16) run as
+ * pa_decode and ignore the plan.
+ * ---------------------------------------------------------------------- */
+#define PA_PREFIX_QUERIES_PER_CTA 64
+PA_API pa_status pa_decode_shared_prefix(const void* q, const void* key_cache, const void* value_cache,
+                                         const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                         const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                                         int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                         int32_t num_blocks, float scale, void* out, pa_dtype dtype,
+                                         void* workspace, size_t workspace_bytes,
+                                         const int32_t* first_partition, const int32_t* chunks,
+                                         int32_t num_chunks, const int32_t* members, int32_t num_members,
+                                         int32_t max_shared_partitions, int32_t min_shared_partitions,
+                                         int32_t* dev_status, void* stream);
+
 /* Which partition kernel pa_decode runs (process-wide; default AUTO).
  * AUTO picks the tensor-core kernel whenever it supports the call (bf16/f16,
  * head_dim 64/128/256, G <= 8, block_size a multiple of 16 up to 256) and the
@@ -298,6 +342,24 @@ PA_API int64_t pa_block_alloc_num_tokens(const pa_block_alloc* a, int64_t seq); 
 PA_API int32_t pa_block_alloc_num_free(const pa_block_alloc* a);
 PA_API int32_t pa_block_alloc_num_sequences(const pa_block_alloc* a);
 PA_API int32_t pa_block_alloc_ref_count(const pa_block_alloc* a, int32_t page); /* -1 if out of range */
+
+/* Prefix plan of a batch for pa_decode_shared_prefix.  seqs[n] is the batch
+ * in decode order; group_size = num_q_heads / num_kv_heads.  Sequences whose
+ * first pages are the same physical pages form a group (led by its first
+ * member in batch order); its shared length is the longest run of leading
+ * table entries common to all members.  A group shares
+ *   SP = min over members of floor(min(shared tokens, tokens - 1) / 512)
+ * whole partitions (the last token of every member stays with the regular
+ * kernel); groups with SP = 0 are dropped.  Members are cut into chunks of
+ * at most PA_PREFIX_QUERIES_PER_CTA / group_size sequences.
+ * Outputs (host arrays): first_partition[n] (SP of the sequence's group, else
+ * 0), chunks[n][4], members[n]; *num_chunks, *num_members,
+ * *max_shared_partitions and *min_shared_partitions (over the whole batch)
+ * receive the counts. */
+PA_API pa_status pa_block_alloc_prefix_plan(const pa_block_alloc* a, const int64_t* seqs, int32_t n,
+                                            int32_t group_size, int32_t* first_partition, int32_t* chunks,
+                                            int32_t* members, int32_t* num_chunks, int32_t* num_members,
+                                            int32_t* max_shared_partitions, int32_t* min_shared_partitions);
 
 /* The free pool front to back into out[cap]; *n_out receives its length. */
 PA_API pa_status pa_block_alloc_free_pool(const pa_block_alloc* a, int32_t* out, int32_t cap,

@@ -15,7 +15,7 @@ import numpy as np
 
 from . import _lib
 from ._lib import (PA_BF16, PA_DECODE_AUTO, PA_DECODE_CUDA_CORES, PA_DECODE_TENSOR_CORES,  # noqa: F401
-                   PA_DEV_BAD_CTX, PA_DEV_BAD_PAGE, PA_DEV_BAD_PAIR, PA_DEV_BAD_SLOT, PA_ERR_NOT_FOUND,
+                   PA_DEV_BAD_CTX, PA_DEV_BAD_PAGE, PA_DEV_BAD_PAIR, PA_DEV_BAD_PLAN, PA_DEV_BAD_SLOT, PA_ERR_NOT_FOUND,
                    PA_ERR_OOM, PA_F16, PA_F32, PA_PARTITION_TOKENS)
 
 
@@ -210,6 +210,25 @@ def pa_decode_fixed_scratch(q, key_cache, value_cache, block_tables, context_len
     return out
 
 
+def pa_decode_shared_prefix(q, key_cache, value_cache, block_tables, context_lens, scale: float, plan, out=None,
+                            workspace=None, dev_status=None, stream=None):
+    """pa_decode for a batch whose groups share leading pages; ``plan`` from prefix_plan_to_device().
+
+    The result equals pa_decode's; shared whole partitions are read once per group.
+    """
+    args, out = _decode_args(q, key_cache, value_cache, block_tables, context_lens, scale, out, workspace,
+                             dev_status, stream)
+    torch = _torch()
+    fp, ch, mem = plan["first_partition"], plan["chunks"], plan["members"]
+    if fp.shape != (q.shape[0],):
+        raise ValueError("plan's first_partition must have one entry per sequence")
+    _check(_lib.load().pa_decode_shared_prefix(
+        *args[:17], _cuda(fp, "first_partition", torch.int32), _cuda(ch, "chunks", torch.int32),
+        int(plan["num_chunks"]), _cuda(mem, "members", torch.int32), int(plan["num_members"]),
+        int(plan["max_shared_partitions"]), int(plan["min_shared_partitions"]), *args[17:]))
+    return out
+
+
 def pa_set_decode_kernel(kernel: int) -> None:
     _check(_lib.load().pa_set_decode_kernel(int(kernel)))
 
@@ -326,6 +345,31 @@ def pa_block_alloc_free_pool(handle) -> np.ndarray:
     return out
 
 
+def pa_block_alloc_prefix_plan(handle, seqs: Sequence[int], group_size: int) -> dict:
+    """Host prefix plan of a batch (see include/pa.h): numpy arrays and counts."""
+    ids = np.ascontiguousarray(seqs, dtype=np.int64)
+    n = len(ids)
+    first = np.zeros(max(n, 1), dtype=np.int32)
+    chunks = np.zeros((max(n, 1), 4), dtype=np.int32)
+    members = np.zeros(max(n, 1), dtype=np.int32)
+    nc, nm, msp, mnp = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check(_lib.load().pa_block_alloc_prefix_plan(handle, _i64p(ids), n, group_size, _i32p(first), _i32p(chunks),
+                                                  _i32p(members), ctypes.byref(nc), ctypes.byref(nm),
+                                                  ctypes.byref(msp), ctypes.byref(mnp)))
+    return {"first_partition": first[:n], "chunks": chunks[:max(nc.value, 1)], "members": members[:max(nm.value, 1)],
+            "num_chunks": nc.value, "num_members": nm.value, "max_shared_partitions": msp.value,
+            "min_shared_partitions": mnp.value}
+
+
+def prefix_plan_to_device(plan: dict, device="cuda") -> dict:
+    """Copy a host prefix plan's arrays to the device (PyTorch is the allocator)."""
+    torch = _torch()
+    out = dict(plan)
+    for k in ("first_partition", "chunks", "members"):
+        out[k] = torch.from_numpy(np.ascontiguousarray(plan[k])).to(device)
+    return out
+
+
 class BlockAllocator:
     """Owns one pa_block_alloc handle; methods map one-to-one onto the C calls."""
 
@@ -380,3 +424,6 @@ class BlockAllocator:
 
     def free_pool(self):
         return pa_block_alloc_free_pool(self.handle)
+
+    def prefix_plan(self, seqs, group_size):
+        return pa_block_alloc_prefix_plan(self.handle, seqs, group_size)

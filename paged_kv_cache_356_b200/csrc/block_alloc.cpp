@@ -14,6 +14,7 @@
 //
 // The pool is a fixed ring of num_blocks ids (it can never hold more), so
 // taking from the front and returning to the back are O(1).
+#include <algorithm>
 #include <unordered_map>
 #include <vector>
 
@@ -221,6 +222,77 @@ pa_status pa_block_alloc_free_pool(const pa_block_alloc* a, int32_t* out, int32_
   if (a->count > cap || (!out && a->count > 0))
     return fail(PA_ERR_INVALID, "free_pool: %lld entries, capacity %d", (long long)a->count, cap);
   for (int64_t i = 0; i < a->count; ++i) out[i] = a->ring[(a->head + i) % a->num_blocks];
+  return PA_OK;
+}
+
+pa_status pa_block_alloc_prefix_plan(const pa_block_alloc* a, const int64_t* seqs, int32_t n, int32_t group_size,
+                                     int32_t* first_partition, int32_t* chunks, int32_t* members, int32_t* num_chunks,
+                                     int32_t* num_members, int32_t* max_shared_partitions,
+                                     int32_t* min_shared_partitions) {
+  if (!a || n < 0 || (n > 0 && (!seqs || !first_partition || !chunks || !members)) || !num_chunks ||
+      !num_members || !max_shared_partitions || !min_shared_partitions)
+    return fail(PA_ERR_INVALID, "prefix_plan: bad argument");
+  if (group_size < 1 || group_size > PA_PREFIX_QUERIES_PER_CTA)
+    return fail(PA_ERR_INVALID, "prefix_plan: group_size %d outside [1, %d]", group_size, PA_PREFIX_QUERIES_PER_CTA);
+  std::vector<const pa_block_alloc::Seq*> batch(n);
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = a->seqs.find(seqs[i]);
+    if (it == a->seqs.end()) return fail(PA_ERR_NOT_FOUND, "prefix_plan: unknown sequence %lld", (long long)seqs[i]);
+    batch[i] = &it->second;
+    first_partition[i] = 0;
+  }
+  // Candidate groups: sequences whose first page is the same shared page, in batch order.
+  std::unordered_map<int32_t, std::vector<int32_t>> by_first;
+  std::vector<int32_t> order;
+  for (int32_t i = 0; i < n; ++i) {
+    const auto& pages = batch[i]->pages;
+    if (pages.empty() || a->refs[pages[0]] < 2) continue;
+    auto& v = by_first[pages[0]];
+    if (v.empty()) order.push_back(pages[0]);
+    v.push_back(i);
+  }
+  const int32_t per_chunk = std::max(1, PA_PREFIX_QUERIES_PER_CTA / group_size);
+  int32_t nc = 0, nm = 0, max_sp = 0;
+  for (int32_t first : order) {
+    const auto& group = by_first[first];
+    if (group.size() < 2) continue;
+    const auto& lead = batch[group[0]]->pages;
+    size_t common = lead.size();
+    for (int32_t i : group) {
+      const auto& pages = batch[i]->pages;
+      size_t k = 0;
+      while (k < common && k < pages.size() && pages[k] == lead[k]) ++k;
+      common = k;
+    }
+    const int64_t shared_tokens = (int64_t)common * a->block_size;
+    int64_t sp = INT64_MAX;
+    for (int32_t i : group) {
+      const int64_t usable = std::min(shared_tokens, batch[i]->tokens - 1);
+      sp = std::min(sp, usable > 0 ? usable / PA_PARTITION_TOKENS : (int64_t)0);
+    }
+    if (sp <= 0) continue;
+    for (size_t off = 0; off < group.size(); off += per_chunk) {
+      const int32_t count = (int32_t)std::min<size_t>(per_chunk, group.size() - off);
+      int32_t* c = chunks + 4 * (int64_t)nc;
+      c[0] = group[0];
+      c[1] = nm;
+      c[2] = count;
+      c[3] = (int32_t)sp;
+      for (int32_t k = 0; k < count; ++k) {
+        members[nm + k] = group[off + k];
+        first_partition[group[off + k]] = (int32_t)sp;
+      }
+      nm += count;
+      ++nc;
+    }
+    max_sp = std::max(max_sp, (int32_t)sp);
+  }
+  int32_t min_sp = n > 0 ? INT32_MAX : 0;
+  for (int32_t i = 0; i < n; ++i) min_sp = std::min(min_sp, first_partition[i]);
+  *num_chunks = nc;
+  *num_members = nm;
+  *max_shared_partitions = max_sp;
+  *min_shared_partitions = min_sp;
   return PA_OK;
 }
 

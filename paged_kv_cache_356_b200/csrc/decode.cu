@@ -57,6 +57,8 @@ struct DecodeArgs {
   float* m_part;
   float* l_part;
   int32_t* status;
+  const int32_t* first_partition;  // optional: partitions [0, first) of b come from the shared-prefix kernel
+  int partition_base;              // grid z of the partition kernels starts at this partition
   int max_blocks_per_seq;
   int num_q_heads;
   int num_kv_heads;
@@ -137,13 +139,14 @@ __global__ void __launch_bounds__(NW * 32) decode_cc_kernel(const DecodeArgs a) 
   const int chunk = blockIdx.y - kvh * chunks;
   const int h0 = kvh * a.group + chunk * GC;
   const int nh = min(GC, a.group - chunk * GC);
-  const int p = blockIdx.z;
+  const int p = blockIdx.z + a.partition_base;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int ctx = context_of(a, b, threadIdx.x == 0 && blockIdx.y == 0 && p == 0);
+  const int ctx = context_of(a, b, threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0);
   const int np = (ctx + kPartition - 1) / kPartition;
   if (p >= max(np, 1)) return;
+  if (a.first_partition && p < __ldg(a.first_partition + b)) return;
   if (ctx == 0) {
     store_zero_rows<T, D>(a, b, h0, nh);
     return;
@@ -256,7 +259,7 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(const DecodeArgs a) 
 
   const int b = blockIdx.x;
   const int kvh = blockIdx.y;
-  const int p = blockIdx.z;
+  const int p = blockIdx.z + a.partition_base;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2;  // fragment row group
@@ -264,9 +267,10 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(const DecodeArgs a) 
   const int G = a.group;
   const int h0 = kvh * G;
 
-  const int ctx = context_of(a, b, threadIdx.x == 0 && kvh == 0 && p == 0);
+  const int ctx = context_of(a, b, threadIdx.x == 0 && kvh == 0 && blockIdx.z == 0);
   const int np = (ctx + kPartition - 1) / kPartition;
   if (p >= max(np, 1)) return;
+  if (a.first_partition && p < __ldg(a.first_partition + b)) return;
   if (ctx == 0) {
     store_zero_rows<T, D>(a, b, h0, G);
     return;
@@ -499,22 +503,279 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(const DecodeArgs a) 
 }
 
 // ---------------------------------------------------------------------------
-// Log-sum-exp merge of the partitions: one warp per (sequence, query head).
+// Shared-prefix partition kernel.  Grid (chunk, kv head, shared partition);
+// 4 warps.  A chunk is up to 64 queries: `count` member sequences x G query
+// heads of one kv head, all reading the same 512-token partition through the
+// leader's table.  The CTA streams the partition's 16-token K/V tiles once
+// through a CTA-wide cp.async pipeline (STAGES buffers, every thread copies
+// its share); warp w owns queries [16w, 16w + 16) as two 8-wide MMA n-tiles:
+//   S^T[16 tok x 16 q] = K_tile . Q^T,   O^T[D x 16 q] += V_tile^T . P^T
+// with the same swizzle and online softmax as the per-sequence kernel (P as
+// a 16-bit operand; the residual MMA is a template option).  Each warp writes
+// its queries' partition partials.
 // ---------------------------------------------------------------------------
-template <typename T, int D>
+template <int D, int STAGES>
+struct SharedShape {
+  static constexpr int kThreads = 128;
+  static constexpr int kRowBytes = 2 * D;
+  static constexpr int kChunksPerRow = kRowBytes / 16;
+  static constexpr int kTile = 16;
+  static constexpr int kTiles = kPartition / kTile;
+  static constexpr int kTileBytes = kTile * kRowBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kSmemBytes = STAGES * kStageBytes;
+  static constexpr int kCopiesPerThread = 2 * kTile * kChunksPerRow / kThreads;
+  static_assert(2 * kTile * kChunksPerRow % kThreads == 0, "tile copies must split evenly");
+};
+
+template <typename T, int D, int STAGES, bool RESIDUAL>
+__global__ void __launch_bounds__(128, 4) decode_shared_kernel(const DecodeArgs a, const int32_t* __restrict__ chunks,
+                                                            const int32_t* __restrict__ members, int num_members,
+                                                            int num_seqs) {
+  using S = SharedShape<D, STAGES>;
+  constexpr int KSTEPS = D / 16;
+  constexpr int MTILES = D / 16;
+  constexpr int NT = 2;  // 8-query n-tiles per warp
+  extern __shared__ __align__(128) uint8_t smem[];
+
+  const int c = blockIdx.x;
+  const int kvh = blockIdx.y;
+  const int p = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2;
+  const int t = lane & 3;
+  const int leader = __ldg(chunks + 4 * c);
+  const int moff = __ldg(chunks + 4 * c + 1);
+  const int mcount = __ldg(chunks + 4 * c + 2);
+  const int sp = __ldg(chunks + 4 * c + 3);
+  if (p >= sp) return;
+  const int bs = a.block_size;
+  const int G = a.group;
+  const int tok_begin = p * kPartition;
+  if ((unsigned)leader >= (unsigned)num_seqs || moff < 0 || mcount < 0 || (int64_t)moff + mcount > num_members ||
+      (int64_t)tok_begin + kPartition > (int64_t)a.max_blocks_per_seq * bs || p >= a.max_partitions) {
+    if (threadIdx.x == 0) flag_status(a.status, PA_DEV_BAD_PLAN);
+    return;
+  }
+  const int first_block = tok_begin / bs;
+  const int nblk = (tok_begin + kPartition - 1) / bs - first_block + 1;  // <= 32 for bs >= 16
+  int lane_page = 0;
+  if (lane < nblk) lane_page = __ldg(a.block_tables + (int64_t)leader * a.max_blocks_per_seq + first_block + lane);
+
+  // Query of column n of this warp's n-tile nt: member (16w + 8nt + n) / G, head (.) % G.
+  auto query_row = [&](int qi) -> int64_t {  // row of q / out for query qi, or -1
+    const int mi = qi / G;
+    if (mi >= mcount) return -1;
+    const int b = __ldg(members + moff + mi);
+    if ((unsigned)b >= (unsigned)num_seqs) return -1;
+    return (int64_t)b * a.num_q_heads + kvh * G + (qi - mi * G);
+  };
+
+  uint32_t qf[NT][KSTEPS][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int64_t row = query_row(warp * 16 + nt * 8 + g);
+    const uint32_t* qrow =
+        reinterpret_cast<const uint32_t*>(reinterpret_cast<const T*>(a.q) + (row < 0 ? 0 : row) * D);
+#pragma unroll
+    for (int ks = 0; ks < KSTEPS; ++ks) {
+      qf[nt][ks][0] = row >= 0 ? __ldg(qrow + 8 * ks + t) : 0u;
+      qf[nt][ks][1] = row >= 0 ? __ldg(qrow + 8 * ks + 4 + t) : 0u;
+    }
+  }
+  const bool warp_busy = (warp * 16) / G < mcount;
+
+  const uint32_t smem_base = smem_u32(smem);
+  const T* kc = reinterpret_cast<const T*>(a.key_cache);
+  const T* vc = reinterpret_cast<const T*>(a.value_cache);
+  // Every thread copies kCopiesPerThread 16-byte chunks of tile i (K chunks, then V chunks).
+  auto load_tile = [&](int i, int stage) {
+    const int tok0 = tok_begin + i * S::kTile;
+    int page = __shfl_sync(kFull, lane_page, tok0 / bs - first_block);
+    bool ok = (unsigned)page < (unsigned)a.num_blocks;
+    if (!ok) {
+      if (threadIdx.x == 0) flag_status(a.status, PA_DEV_BAD_PAGE);
+      page = 0;
+    }
+    const int64_t row0 = ((int64_t)page * a.num_kv_heads + kvh) * bs + (tok0 % bs);
+    const uint32_t kdst = smem_base + stage * S::kStageBytes;
+#pragma unroll
+    for (int j = 0; j < S::kCopiesPerThread; ++j) {
+      const int idx = threadIdx.x + S::kThreads * j;
+      const int half = idx / (S::kTile * S::kChunksPerRow);  // 0: K, 1: V
+      const int rem = idx - half * (S::kTile * S::kChunksPerRow);
+      const int r = rem / S::kChunksPerRow;
+      const int cc = rem - r * S::kChunksPerRow;
+      const T* src = (half ? vc : kc) + (row0 + r) * D + cc * 8;
+      const uint32_t dst = kdst + half * S::kTileBytes + r * S::kRowBytes + ((cc ^ (r & 7)) << 4);
+      cp_async_16(dst, src, ok ? 16u : 0u);
+    }
+  };
+
+  float o[MTILES][NT][4];
+#pragma unroll
+  for (int mt = 0; mt < MTILES; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+  float m[NT][2], l[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) m[nt][0] = m[nt][1] = -INFINITY, l[nt][0] = l[nt][1] = 0.f;
+
+#pragma unroll
+  for (int i = 0; i < STAGES - 1; ++i) {
+    load_tile(i, i);
+    cp_async_commit();
+  }
+  for (int i = 0; i < S::kTiles; ++i) {
+    {
+      const int nxt = i + STAGES - 1;
+      if (nxt < S::kTiles) load_tile(nxt, nxt % STAGES);
+      cp_async_commit();
+    }
+    cp_async_wait<STAGES - 1>();
+    __syncthreads();
+    if (warp_busy) {
+      const int stage = i % STAGES;
+      const uint32_t kbase = smem_base + stage * S::kStageBytes;
+      const uint32_t vbase = kbase + S::kTileBytes;
+      const int tok0 = tok_begin + i * S::kTile;
+      const bool valid = (unsigned)__shfl_sync(kFull, lane_page, tok0 / bs - first_block) < (unsigned)a.num_blocks;
+
+      float sacc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+      {
+        const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
+        const uint32_t rbase = kbase + r * S::kRowBytes;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+          const int cc = 2 * ks + (lane >> 4);
+          uint32_t a0, a1, a2, a3;
+          ldmatrix_x4(rbase + ((cc ^ (r & 7)) << 4), a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_16816<T>(sacc[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+        }
+      }
+      uint32_t pb[NT][2], pl[NT][2];
+      float alpha[NT][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float sv[4], pr[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sv[e] = valid ? sacc[nt][e] * a.qk_scale_log2 : -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          float mx = fmaxf(sv[j], sv[2 + j]);
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+          const float mn = fmaxf(m[nt][j], mx);
+          const float base = mn == -INFINITY ? 0.f : mn;
+          alpha[nt][j] = exp2f(m[nt][j] - base);
+          pr[j] = exp2f(sv[j] - base);
+          pr[2 + j] = exp2f(sv[2 + j] - base);
+          l[nt][j] = l[nt][j] * alpha[nt][j] + pr[j] + pr[2 + j];
+          m[nt][j] = mn;
+        }
+        const uint32_t hi0 = pack2<T>(pr[0], pr[1]);
+        const uint32_t hi1 = pack2<T>(pr[2], pr[3]);
+        const float2 r0 = unpack2<T>(hi0), r1 = unpack2<T>(hi1);
+        pb[nt][0] = movmatrix_trans(hi0);
+        pb[nt][1] = movmatrix_trans(hi1);
+        if constexpr (RESIDUAL) {
+          pl[nt][0] = movmatrix_trans(pack2<T>(pr[0] - r0.x, pr[1] - r0.y));
+          pl[nt][1] = movmatrix_trans(pack2<T>(pr[2] - r1.x, pr[3] - r1.y));
+        } else {
+          (void)r0;
+          (void)r1;
+          pl[nt][0] = pl[nt][1] = 0u;
+        }
+      }
+      const int mat = lane >> 3;
+      const int r = (lane & 7) + ((mat >> 1) << 3);
+      const uint32_t rbase = vbase + r * S::kRowBytes;
+#pragma unroll
+      for (int mt = 0; mt < MTILES; ++mt) {
+        const int cc = 2 * mt + (mat & 1);
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4_trans(rbase + ((cc ^ (r & 7)) << 4), a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          o[mt][nt][0] *= alpha[nt][0];
+          o[mt][nt][1] *= alpha[nt][1];
+          o[mt][nt][2] *= alpha[nt][0];
+          o[mt][nt][3] *= alpha[nt][1];
+          mma_16816<T>(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+          if constexpr (RESIDUAL) mma_16816<T>(o[mt][nt], a0, a1, a2, a3, pl[nt][0], pl[nt][1]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+  cp_async_wait<0>();
+  if (!warp_busy) return;
+
+  // Partials of this warp's 16 queries: column 2t + j of n-tile nt.
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float lj = l[nt][j];
+      lj += __shfl_xor_sync(kFull, lj, 4);
+      lj += __shfl_xor_sync(kFull, lj, 8);
+      lj += __shfl_xor_sync(kFull, lj, 16);
+      const int64_t row = query_row(warp * 16 + nt * 8 + 2 * t + j);
+      if (row < 0) continue;
+      const int64_t part = row * a.max_partitions + p;
+      const float inv = lj > 0.f ? 1.f / lj : 0.f;
+      float* dst = a.o_part + part * D;
+#pragma unroll
+      for (int mt = 0; mt < MTILES; ++mt) {
+        dst[16 * mt + g] = o[mt][nt][j] * inv;
+        dst[16 * mt + g + 8] = o[mt][nt][2 + j] * inv;
+      }
+      if (g == 0) {
+        a.m_part[part] = m[nt][j] == -INFINITY ? -INFINITY : m[nt][j] * kLn2;
+        a.l_part[part] = lj;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Log-sum-exp merge of the partitions.  A CTA of 4 warps serves 4 / WPI
+// (sequence, query head) items with WPI warps each (WPI grows with the
+// partition count).  Warp w of an item merges partitions w, w + WPI, ... with
+// its own running maximum (the lanes compute 32 weights per round; partials
+// are loaded four at a time), then the item's warps merge through shared
+// memory the same way.
+// ---------------------------------------------------------------------------
+template <typename T, int D, int WPI>
 __global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeArgs a, int num_seqs) {
   constexpr int VPL = D / 32;
-  const int64_t item = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
+  constexpr int NW = 4;
+  constexpr int IPC = NW / WPI;  // items per CTA
+  constexpr int UNROLL = 4;
+  __shared__ float acc_w[NW][D];
+  __shared__ float m_w[NW], l_w[NW];
+  const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  if (item >= (int64_t)num_seqs * a.num_q_heads) return;
-  const int b = (int)(item / a.num_q_heads);
-  const int ctx = context_of(a, b, false);
-  const int np = (ctx + kPartition - 1) / kPartition;
-  if (np <= 1) return;
-  const int64_t base = item * a.max_partitions;
+  const int sub = warp % WPI;  // warp within its item
+  const int64_t item = (int64_t)blockIdx.x * IPC + warp / WPI;
+  const bool live = item < (int64_t)num_seqs * a.num_q_heads;
+  int np = 0;
+  int64_t base = 0;
+  if (live) {
+    const int b = (int)(item / a.num_q_heads);
+    np = (context_of(a, b, false) + kPartition - 1) / kPartition;
+    base = item * a.max_partitions;
+  }
+  const bool merge = live && np > 1;
 
   float mx = -INFINITY;
-  for (int pp = lane; pp < np; pp += 32) mx = fmaxf(mx, a.m_part[base + pp]);
+  if (merge)
+    for (int p = sub + WPI * lane; p < np; p += WPI * 32) mx = fmaxf(mx, a.m_part[base + p]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
 
@@ -522,36 +783,84 @@ __global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeArgs a, 
 #pragma unroll
   for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
   float lsum = 0.f;
-  if (mx != -INFINITY) {
-    for (int p0 = 0; p0 < np; p0 += 32) {
-      float w = 0.f;
-      if (p0 + lane < np) w = a.l_part[base + p0 + lane] * expf(a.m_part[base + p0 + lane] - mx);
-      lsum += w;
-      const int cnt = min(32, np - p0);
-      for (int k = 0; k < cnt; ++k) {
-        const float wk = __shfl_sync(kFull, w, k);
-        const float* src = a.o_part + (base + p0 + k) * D + lane * VPL;
-        if constexpr (VPL % 4 == 0) {
+  if (merge && mx != -INFINITY) {
+    for (int p0 = sub; p0 < np; p0 += WPI * 32) {
+      const int p = p0 + WPI * lane;
+      float wt = 0.f;
+      if (p < np) wt = a.l_part[base + p] * expf(a.m_part[base + p] - mx);
+      lsum += wt;
+      const int cnt = min(32, (np - p0 + WPI - 1) / WPI);
+      for (int k = 0; k < cnt; k += UNROLL) {
+        float x[UNROLL][VPL];
+        float wk[UNROLL];
 #pragma unroll
-          for (int v = 0; v < VPL / 4; ++v) {
-            const float4 x = reinterpret_cast<const float4*>(src)[v];
-            acc[4 * v] = fmaf(wk, x.x, acc[4 * v]);
-            acc[4 * v + 1] = fmaf(wk, x.y, acc[4 * v + 1]);
-            acc[4 * v + 2] = fmaf(wk, x.z, acc[4 * v + 2]);
-            acc[4 * v + 3] = fmaf(wk, x.w, acc[4 * v + 3]);
+        for (int u = 0; u < UNROLL; ++u) {
+          wk[u] = __shfl_sync(kFull, wt, min(k + u, 31));
+          if (k + u < cnt) {
+            const float* src = a.o_part + (base + p0 + WPI * (k + u)) * D + lane * VPL;
+            if constexpr (VPL % 4 == 0) {
+#pragma unroll
+              for (int v = 0; v < VPL / 4; ++v) {
+                const float4 f = reinterpret_cast<const float4*>(src)[v];
+                x[u][4 * v] = f.x;
+                x[u][4 * v + 1] = f.y;
+                x[u][4 * v + 2] = f.z;
+                x[u][4 * v + 3] = f.w;
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < VPL; ++i) x[u][i] = src[i];
+            }
+          } else {
+            wk[u] = 0.f;
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) x[u][i] = 0.f;
           }
-        } else {
-#pragma unroll
-          for (int i = 0; i < VPL; ++i) acc[i] = fmaf(wk, src[i], acc[i]);
         }
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u)
+#pragma unroll
+          for (int i = 0; i < VPL; ++i) acc[i] = fmaf(wk[u], x[u][i], acc[i]);
       }
     }
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(kFull, lsum, off);
-  T* out = reinterpret_cast<T*>(a.out) + item * D + lane * VPL;
+
+  if constexpr (WPI == 1) {
+    if (merge) {
+      T* out = reinterpret_cast<T*>(a.out) + item * D + lane * VPL;
 #pragma unroll
-  for (int i = 0; i < VPL; ++i) out[i] = from_float<T>(lsum > 0.f ? acc[i] / lsum : 0.f);
+      for (int i = 0; i < VPL; ++i) out[i] = from_float<T>(lsum > 0.f ? acc[i] / lsum : 0.f);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) acc_w[warp][lane * VPL + i] = acc[i];
+    if (lane == 0) {
+      m_w[warp] = mx;
+      l_w[warp] = lsum;
+    }
+    __syncthreads();
+    if (!merge) return;
+    const int w0 = warp - sub;  // first warp of this item
+    float gm = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < WPI; ++w) gm = fmaxf(gm, m_w[w0 + w]);
+    float scale_w[WPI];
+    float total = 0.f;
+#pragma unroll
+    for (int w = 0; w < WPI; ++w) {
+      scale_w[w] = gm == -INFINITY ? 0.f : expf(m_w[w0 + w] - gm);
+      total += l_w[w0 + w] * scale_w[w];
+    }
+    T* out = reinterpret_cast<T*>(a.out) + item * D;
+    for (int d = sub * 32 + lane; d < D; d += WPI * 32) {
+      float o = 0.f;
+#pragma unroll
+      for (int w = 0; w < WPI; ++w) o = fmaf(acc_w[w0 + w][d], scale_w[w], o);
+      out[d] = from_float<T>(total > 0.f ? o / total : 0.f);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -625,13 +934,39 @@ cudaError_t launch_tc_dim(const DecodeArgs& a, int head_dim, dim3 grid, cudaStre
   return cudaErrorInvalidValue;
 }
 
+template <typename T, int D>
+cudaError_t launch_shared(const DecodeArgs& a, dim3 grid, const int32_t* chunks, const int32_t* members,
+                          int num_members, int num_seqs, cudaStream_t stream) {
+  constexpr int kStages = 4;
+  using S = SharedShape<D, kStages>;
+  static std::atomic<uint64_t> done{0};
+  // Shared partitions are always whole 512-token partitions, where the 16-bit
+  // rounding of P averages out; the per-sequence kernel keeps the residual
+  // for short and ragged partitions.
+  auto kernel = decode_shared_kernel<T, D, kStages, false>;
+  cudaError_t err = ensure_smem(kernel, S::kSmemBytes, done);
+  if (err != cudaSuccess) return err;
+  kernel<<<grid, S::kThreads, S::kSmemBytes, stream>>>(a, chunks, members, num_members, num_seqs);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_shared_dim(const DecodeArgs& a, int head_dim, dim3 grid, const int32_t* chunks,
+                              const int32_t* members, int num_members, int num_seqs, cudaStream_t stream) {
+  switch (head_dim) {
+    case 64: return launch_shared<T, 64>(a, grid, chunks, members, num_members, num_seqs, stream);
+    case 128: return launch_shared<T, 128>(a, grid, chunks, members, num_members, num_seqs, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
 constexpr int kCcHeads = 4;
 constexpr int kCcWarps = 4;
 
 template <typename T>
 cudaError_t launch_cc(const DecodeArgs& a, int head_dim, int num_seqs, int partitions, cudaStream_t stream) {
   const int chunks = (a.group + kCcHeads - 1) / kCcHeads;
-  dim3 grid(num_seqs, a.num_kv_heads * chunks, partitions);
+  dim3 grid(num_seqs, a.num_kv_heads * chunks, partitions - a.partition_base);
   switch (head_dim) {
     case 64: decode_cc_kernel<T, 64, kCcHeads, kCcWarps><<<grid, kCcWarps * 32, 0, stream>>>(a); break;
     case 128: decode_cc_kernel<T, 128, kCcHeads, kCcWarps><<<grid, kCcWarps * 32, 0, stream>>>(a); break;
@@ -641,17 +976,28 @@ cudaError_t launch_cc(const DecodeArgs& a, int head_dim, int num_seqs, int parti
   return cudaGetLastError();
 }
 
+template <typename T, int D>
+cudaError_t launch_reduce_dim(const DecodeArgs& a, int num_seqs, cudaStream_t stream) {
+  const int64_t items = (int64_t)num_seqs * a.num_q_heads;
+  auto grid = [&](int ipc) { return (unsigned)((items + ipc - 1) / ipc); };
+  if (a.max_partitions <= 16)
+    decode_reduce_kernel<T, D, 1><<<grid(4), 128, 0, stream>>>(a, num_seqs);
+  else if (a.max_partitions <= 48)
+    decode_reduce_kernel<T, D, 2><<<grid(2), 128, 0, stream>>>(a, num_seqs);
+  else
+    decode_reduce_kernel<T, D, 4><<<grid(1), 128, 0, stream>>>(a, num_seqs);
+  return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t launch_reduce(const DecodeArgs& a, int head_dim, int num_seqs, cudaStream_t stream) {
-  const int64_t items = (int64_t)num_seqs * a.num_q_heads;
-  const unsigned grid = (unsigned)((items + 3) / 4);
+  if ((int64_t)num_seqs * a.num_q_heads > 0x7fffffffLL) return cudaErrorInvalidValue;
   switch (head_dim) {
-    case 64: decode_reduce_kernel<T, 64><<<grid, 128, 0, stream>>>(a, num_seqs); break;
-    case 128: decode_reduce_kernel<T, 128><<<grid, 128, 0, stream>>>(a, num_seqs); break;
-    case 256: decode_reduce_kernel<T, 256><<<grid, 128, 0, stream>>>(a, num_seqs); break;
-    default: return cudaErrorInvalidValue;
+    case 64: return launch_reduce_dim<T, 64>(a, num_seqs, stream);
+    case 128: return launch_reduce_dim<T, 128>(a, num_seqs, stream);
+    case 256: return launch_reduce_dim<T, 256>(a, num_seqs, stream);
   }
-  return cudaGetLastError();
+  return cudaErrorInvalidValue;
 }
 
 bool tc_supported(pa_dtype dt, int head_dim, int group, int block_size) {
@@ -753,7 +1099,7 @@ pa_status launch_partitions(const DecodeArgs& a, pa_dtype dtype, int head_dim, i
     return fail(PA_ERR_UNSUPPORTED, "decode: tensor-core kernel needs bf16/f16, G <= 8, block_size %% 16 == 0");
   cudaError_t err;
   if (tc_ok && choice != PA_DECODE_CUDA_CORES) {
-    dim3 grid(num_seqs, a.num_kv_heads, partitions);
+    dim3 grid(num_seqs, a.num_kv_heads, partitions - a.partition_base);
     const int warps = g_tc_warps.load(), stages = g_tc_stages.load();
     err = dtype == PA_BF16 ? launch_tc_dim<__nv_bfloat16>(a, head_dim, grid, s, warps, stages)
                            : launch_tc_dim<__half>(a, head_dim, grid, s, warps, stages);
@@ -900,4 +1246,43 @@ extern "C" pa_status pa_decode_fixed_scratch(const void* q, const void* key_cach
   return pa_decode(q, key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs, num_q_heads,
                    num_kv_heads, head_dim, block_size, num_blocks, scale, out, dtype, scratch,
                    (size_t)PA_FIXED_SCRATCH_BYTES, dev_status, stream);
+}
+
+extern "C" pa_status pa_decode_shared_prefix(const void* q, const void* key_cache, const void* value_cache,
+                                             const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                             const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                                             int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                             int32_t num_blocks, float scale, void* out, pa_dtype dtype,
+                                             void* workspace, size_t workspace_bytes, const int32_t* first_partition,
+                                             const int32_t* chunks, int32_t num_chunks, const int32_t* members,
+                                             int32_t num_members, int32_t max_shared_partitions,
+                                             int32_t min_shared_partitions, int32_t* dev_status, void* stream) {
+  DecodeArgs a;
+  int partitions = 0;
+  pa_status st = prepare_decode(q, key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                                num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, out, dtype,
+                                workspace, workspace_bytes, dev_status, a, partitions);
+  if (st != PA_OK || num_seqs == 0) return st;
+  if (num_chunks < 0 || num_members < 0 || max_shared_partitions < 0 || min_shared_partitions < 0 ||
+      min_shared_partitions > max_shared_partitions)
+    return fail(PA_ERR_INVALID, "decode_shared_prefix: bad plan sizes");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool joint = (dtype == PA_BF16 || dtype == PA_F16) && (head_dim == 64 || head_dim == 128) &&
+                     block_size % 16 == 0 && a.group <= PA_PREFIX_QUERIES_PER_CTA && partitions > 1 &&
+                     num_chunks > 0 && num_members > 0 && max_shared_partitions > 0 && first_partition && chunks &&
+                     members;
+  if (joint) {
+    if (!aligned16(chunks)) return fail(PA_ERR_INVALID, "decode_shared_prefix: chunks must be 16-byte aligned");
+    dim3 grid(num_chunks, num_kv_heads, max_shared_partitions < partitions ? max_shared_partitions : partitions);
+    const cudaError_t err =
+        dtype == PA_BF16 ? launch_shared_dim<__nv_bfloat16>(a, head_dim, grid, chunks, members, num_members, num_seqs, s)
+                         : launch_shared_dim<__half>(a, head_dim, grid, chunks, members, num_members, num_seqs, s);
+    if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode shared-prefix kernel: %s", cudaGetErrorString(err));
+    a.first_partition = first_partition;
+    // Partitions below every sequence's first_partition need no per-sequence CTA.
+    a.partition_base = min_shared_partitions < partitions - 1 ? min_shared_partitions : partitions - 1;
+  }
+  st = launch_partitions(a, dtype, head_dim, num_seqs, partitions, s);
+  if (st != PA_OK || partitions <= 1) return st;
+  return launch_reduce_any(a, dtype, head_dim, num_seqs, s);
 }

@@ -22,7 +22,8 @@ from . import binding as pa
 
 
 class TraceRunner:
-    def __init__(self, workload, device: str = "cuda", max_chunk_tokens: int = 1 << 17, threads: int = 8):
+    def __init__(self, workload, device: str = "cuda", max_chunk_tokens: int = 1 << 17, threads: int = 8,
+                 shared_prefix: bool = False):
         import torch
 
         self.torch = torch
@@ -40,6 +41,8 @@ class TraceRunner:
         self.write_slots: List[np.ndarray] = []
         self.step_write = None   # (key, value, slots) of the write group before decode, on the device
         self.q = self.block_tables = self.context_lens = self.out = self.workspace = None
+        self.shared_prefix = shared_prefix
+        self.plan = None
 
     # -- helpers ----------------------------------------------------------------------
     def _to_device(self, host: np.ndarray):
@@ -122,8 +125,15 @@ class TraceRunner:
         need = pa.pa_decode_workspace_size(w.num_seqs, w.num_q_heads, w.head_dim,
                                            w.max_blocks_per_seq * w.block_size)
         self.workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
+        if self.shared_prefix:
+            host = self.alloc.prefix_plan(list(range(w.num_seqs)), w.group_size)
+            self.plan = pa.prefix_plan_to_device(host, self.device)
 
     def decode(self, stream=None):
+        if self.plan is not None:
+            return pa.pa_decode_shared_prefix(self.q, self.key_cache, self.value_cache, self.block_tables,
+                                              self.context_lens, self.w.scale, self.plan, out=self.out,
+                                              workspace=self.workspace, dev_status=self.dev_status, stream=stream)
         return pa.pa_decode(self.q, self.key_cache, self.value_cache, self.block_tables, self.context_lens,
                             self.w.scale, out=self.out, workspace=self.workspace, dev_status=self.dev_status,
                             stream=stream)

@@ -34,13 +34,15 @@ def _sampled_reference(w, seqs, heads=None):
     return ref
 
 
-@pytest.fixture(scope="module", params=["llama8b", "llama70b", "prefix", "beam32k"])
+@pytest.fixture(scope="module", params=["llama8b", "llama70b", "prefix", "beam32k", "prefix+shared",
+                                        "beam32k+shared"])
 def full_run(request):
     import torch
     pa.pa_set_decode_kernel(pa.PA_DECODE_AUTO)
     pa.pa_set_decode_tiling(4, 2)
-    w = workloads.by_name(request.param)
-    run = TraceRunner(w)
+    name, _, shared = request.param.partition("+")
+    w = workloads.by_name(name)
+    run = TraceRunner(w, shared_prefix=bool(shared))
     out = run.run()
     torch.cuda.synchronize()
     yield w, run, out

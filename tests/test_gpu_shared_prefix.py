@@ -1,0 +1,91 @@
+"""pa_decode_shared_prefix on the GPU: same results as the oracle (and hence as
+pa_decode) while shared partitions are read once per group."""
+import numpy as np
+import pytest
+
+from oracle import scenario
+from paged_kv_cache_356_b200 import binding as pa
+from paged_kv_cache_356_b200 import workloads
+from paged_kv_cache_356_b200.runner import TraceRunner
+from tests.parity import assert_decode_close, bits_of, host_bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("make", [
+    lambda: workloads.prefix(num_seqs=5, prefix_len=1700, max_tail=90),
+    lambda: workloads.prefix(num_seqs=40, prefix_len=1100, max_tail=600),          # G=4: 3 chunks of <= 16
+    lambda: workloads.beam32k(num_beams=3, prompt_len=2100, own=40),
+    lambda: workloads.beam32k(num_beams=8, prompt_len=1536, own=1),               # prompt = 3 whole partitions
+], ids=["prefix-5", "prefix-40", "beam-3", "beam-8-exact"])
+def test_shared_flows_match_oracle(make):
+    w = make()
+    run = TraceRunner(w, shared_prefix=True)
+    out = run.run()
+    assert run.plan["num_chunks"] > 0
+    ref = scenario.run(w)
+    assert run.allocator_state() == ref["state"]
+    np.testing.assert_array_equal(bits_of(run.key_cache), host_bits(ref["key_cache"]))
+    assert run.status() == 0
+    assert_decode_close(out, ref["out"], w.dtype, w.name)
+
+
+@pytest.mark.parametrize("hq,hkv,d,bs", [(8, 8, 128, 16), (16, 8, 128, 32), (64, 8, 64, 16), (32, 2, 128, 16),
+                                         (64, 4, 128, 64)])
+def test_shared_shapes(hq, hkv, d, bs):
+    """G = 1, 2, 8, 16, 16 with head_dim 64 / 128 and several block sizes."""
+    import math
+    import torch
+    from oracle import attention
+    rng = np.random.Generator(np.random.PCG64(hq + hkv + d + bs))
+    nseq, prompt = 6, 1600 + bs
+    own = [int(x) for x in rng.integers(1, 700, size=nseq)]
+    nb = -(-prompt // bs) + sum(-(-o // bs) + 1 for o in own) + 4
+    a = pa.BlockAllocator(nb, bs, rng.permutation(nb))
+    a.allocate_sequence(0, prompt)
+    for s in range(1, nseq):
+        a.fork(0, s)
+    pairs = []
+    for s in range(nseq):
+        for _ in range(own[s]):
+            _, src, dst = a.append_token(s)
+            if src >= 0:
+                pairs.append((src, dst))
+    ctx = [prompt + o for o in own]
+    mb = max(-(-c // bs) for c in ctx)
+    tables, lens = a.block_tables(list(range(nseq)), mb, pad=-1)
+    kc = workloads.normal_values(rng, nb * hkv * bs * d, "bf16").reshape(nb, hkv, bs, d)
+    vc = workloads.normal_values(rng, nb * hkv * bs * d, "bf16").reshape(nb, hkv, bs, d)
+    q = workloads.normal_values(rng, nseq * hq * d, "bf16").reshape(nseq, hq, d)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).cuda()  # noqa
+    plan = pa.prefix_plan_to_device(a.prefix_plan(list(range(nseq)), hq // hkv))
+    assert plan["num_chunks"] >= 1
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = pa.pa_decode_shared_prefix(dev(q), dev(kc), dev(vc), torch.from_numpy(tables).cuda(),
+                                     torch.from_numpy(lens).cuda(), 1 / math.sqrt(d), plan, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ref = attention.decode_attention(q, kc, vc, tables, lens, 1 / math.sqrt(d), "bf16")
+    assert_decode_close(out, ref, "bf16", f"shared hq{hq} hkv{hkv} d{d} bs{bs}")
+
+
+def test_bad_plan_entries_are_skipped_and_flagged():
+    """Out-of-range leader / member ranges / partitions are flagged, never dereferenced."""
+    import math
+    import torch
+    w = workloads.beam32k(num_beams=3, prompt_len=1100, own=40)
+    run = TraceRunner(w, shared_prefix=True)
+    run.run(decode=False)
+    plan = dict(run.plan)
+    bad = torch.tensor([[w.num_seqs + 5, 0, 3, 2],      # leader outside the batch
+                        [0, 1, 9, 2],                   # members past the array
+                        [0, 0, 3, 40000]],              # partitions past the table
+                       dtype=torch.int32, device="cuda")
+    plan["chunks"], plan["num_chunks"] = bad, 3
+    plan["max_shared_partitions"] = 3
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_decode_shared_prefix(run.q, run.key_cache, run.value_cache, run.block_tables, run.context_lens,
+                               1 / math.sqrt(w.head_dim), plan, out=run.out, workspace=run.workspace,
+                               dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() & pa.PA_DEV_BAD_PLAN
