@@ -67,6 +67,7 @@ typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1, PA_F16 = 2 } pa_dtype;
 #define PA_DEV_BAD_CTX 4  /* decode: context_len < 0 or > max_blocks_per_seq * block_size  */
 #define PA_DEV_BAD_PAIR 8 /* copy_blocks: a source or destination page is outside the pool  */
 #define PA_DEV_BAD_PLAN 16 /* decode_shared_prefix: a prefix-plan entry is out of range       */
+#define PA_DEV_TIMEOUT 32  /* a bounded wait inside a kernel gave up (the CTA's rows are not written) */
 
 /* Tokens per split-context partition of pa_decode. */
 #define PA_PARTITION_TOKENS 512
@@ -142,7 +143,10 @@ PA_API pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_
  *                 merged by a log-sum-exp reduction.  Layout, with
  *                 P = ceil(max_blocks_per_seq*block_size / PA_PARTITION_TOKENS):
  *                   float o_part[num_seqs][num_q_heads][P][head_dim]  (o_p / l_p)
- *                   float m_part[num_seqs][num_q_heads][P]  (max score, natural log units)
+ *                   float m_part[num_seqs][num_q_heads][P]  (reference score m_p, natural
+ *                                                            log units: the partition's
+ *                                                            maximum score, or up to 8 ln 2
+ *                                                            below it on the shared-prefix path)
  *                   float l_part[num_seqs][num_q_heads][P]  (sum of exp(s - m_p))
  *                 Only partitions of sequences with more than one partition
  *                 are written.
@@ -246,7 +250,7 @@ PA_API pa_status pa_decode_fixed_scratch(const void* q, const void* key_cache, c
  * support (fp32, head_dim 256, block_size not a multiple of 16) run as
  * pa_decode and ignore the plan.
  * ---------------------------------------------------------------------- */
-#define PA_PREFIX_QUERIES_PER_CTA 64
+#define PA_PREFIX_QUERIES_PER_CTA 128
 PA_API pa_status pa_decode_shared_prefix(const void* q, const void* key_cache, const void* value_cache,
                                          const int32_t* block_tables, int32_t max_blocks_per_seq,
                                          const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
@@ -257,6 +261,17 @@ PA_API pa_status pa_decode_shared_prefix(const void* q, const void* key_cache, c
                                          int32_t num_chunks, const int32_t* members, int32_t num_members,
                                          int32_t max_shared_partitions, int32_t min_shared_partitions,
                                          int32_t* dev_status, void* stream);
+
+/* Which joint kernel pa_decode_shared_prefix runs (process-wide; default
+ * AUTO = TCGEN05): the 5th-generation tensor-core kernel (tcgen05.mma with
+ * Tensor Memory accumulators) or the mma.sync kernel.  Both compute the same
+ * partials; the switch exists for testing and measurement. */
+typedef enum pa_shared_prefix_kernel {
+  PA_SHARED_PREFIX_AUTO = 0,
+  PA_SHARED_PREFIX_TCGEN05 = 1,
+  PA_SHARED_PREFIX_MMA_SYNC = 2
+} pa_shared_prefix_kernel;
+PA_API pa_status pa_set_shared_prefix_kernel(pa_shared_prefix_kernel kernel);
 
 /* Which partition kernel pa_decode runs (process-wide; default AUTO).
  * AUTO picks the tensor-core kernel whenever it supports the call (bf16/f16,

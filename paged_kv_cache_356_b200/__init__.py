@@ -16,4 +16,4 @@ from .binding import (BlockAllocator, PagedAttentionError, PagedAttentionOOM, Se
                       pa_decode_fixed_scratch, pa_decode_partitions, pa_decode_reduce,
                       pa_decode_shared_prefix, pa_block_alloc_prefix_plan, prefix_plan_to_device,
                       pa_decode_workspace_size, pa_reshape_and_cache, pa_set_decode_kernel,
-                      pa_set_decode_tiling, pa_version)
+                      pa_set_decode_tiling, pa_set_shared_prefix_kernel, pa_version)

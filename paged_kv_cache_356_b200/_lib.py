@@ -13,8 +13,10 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpa_b200.
 PA_OK, PA_ERR_INVALID, PA_ERR_OOM, PA_ERR_CUDA, PA_ERR_NOT_FOUND, PA_ERR_UNSUPPORTED = 0, -1, -2, -3, -4, -5
 PA_F32, PA_BF16, PA_F16 = 0, 1, 2
 PA_DEV_BAD_SLOT, PA_DEV_BAD_PAGE, PA_DEV_BAD_CTX, PA_DEV_BAD_PAIR, PA_DEV_BAD_PLAN = 1, 2, 4, 8, 16
-PA_PREFIX_QUERIES_PER_CTA = 64
+PA_PREFIX_QUERIES_PER_CTA = 128
+PA_DEV_TIMEOUT = 32
 PA_DECODE_AUTO, PA_DECODE_CUDA_CORES, PA_DECODE_TENSOR_CORES = 0, 1, 2
+PA_SHARED_PREFIX_AUTO, PA_SHARED_PREFIX_TCGEN05, PA_SHARED_PREFIX_MMA_SYNC = 0, 1, 2
 PA_PARTITION_TOKENS = 512
 PA_FIXED_SCRATCH_BYTES = 32 * 1024 * 1024
 
@@ -40,6 +42,7 @@ SIGNATURES = {
     "pa_decode_shared_prefix": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
                                        _vp, _i32, _vp, _sz, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _vp, _vp]),
     "pa_set_decode_kernel": (_i32, [_i32]),
+    "pa_set_shared_prefix_kernel": (_i32, [_i32]),
     "pa_set_decode_tiling": (_i32, [_i32, _i32]),
     "pa_block_alloc_create": (_i32, [_i32, _i32, _pi32, _c.POINTER(_vp)]),
     "pa_block_alloc_destroy": (None, [_vp]),

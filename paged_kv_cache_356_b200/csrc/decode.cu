@@ -33,10 +33,12 @@
 #include <math.h>
 
 #include <atomic>
+#include <type_traits>
 #include <mutex>
 
 #include "device.cuh"
 #include "pa_internal.h"
+#include "tcgen05.cuh"
 
 namespace pa {
 namespace {
@@ -503,8 +505,9 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(const DecodeArgs a) 
 }
 
 // ---------------------------------------------------------------------------
-// Shared-prefix partition kernel.  Grid (chunk, kv head, shared partition);
-// 4 warps.  A chunk is up to 64 queries: `count` member sequences x G query
+// Shared-prefix partition kernel on mma.sync (the fallback of the tcgen05
+// kernel below).  Grid (chunk, kv head, shared partition); 8 warps.  A chunk
+// is up to 128 queries: `count` member sequences x G query
 // heads of one kv head, all reading the same 512-token partition through the
 // leader's table.  The CTA streams the partition's 16-token K/V tiles once
 // through a CTA-wide cp.async pipeline (STAGES buffers, every thread copies
@@ -516,7 +519,8 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(const DecodeArgs a) 
 // ---------------------------------------------------------------------------
 template <int D, int STAGES>
 struct SharedShape {
-  static constexpr int kThreads = 128;
+  static constexpr int kWarps = PA_PREFIX_QUERIES_PER_CTA / 16;
+  static constexpr int kThreads = 32 * kWarps;
   static constexpr int kRowBytes = 2 * D;
   static constexpr int kChunksPerRow = kRowBytes / 16;
   static constexpr int kTile = 16;
@@ -529,7 +533,7 @@ struct SharedShape {
 };
 
 template <typename T, int D, int STAGES, bool RESIDUAL>
-__global__ void __launch_bounds__(128, 4) decode_shared_kernel(const DecodeArgs a, const int32_t* __restrict__ chunks,
+__global__ void __launch_bounds__(PA_PREFIX_QUERIES_PER_CTA * 2, 2) decode_shared_kernel(const DecodeArgs a, const int32_t* __restrict__ chunks,
                                                             const int32_t* __restrict__ members, int num_members,
                                                             int num_seqs) {
   using S = SharedShape<D, STAGES>;
@@ -744,6 +748,293 @@ __global__ void __launch_bounds__(128, 4) decode_shared_kernel(const DecodeArgs 
 }
 
 // ---------------------------------------------------------------------------
+// Shared-prefix partition kernel on the 5th-generation tensor cores (tcgen05,
+// accumulators in Tensor Memory).  Grid (chunk, kv head, shared partition);
+// 4 warps; one CTA serves up to 128 queries (the chunk's members x G heads of
+// one kv head, padded with zero rows to the MMA's M = 128) over one shared
+// 512-token partition, in 64-token steps:
+//   S[128 x 64]  = Q[128 x D] . K_step^T      (tcgen05.mma, A and B from smem)
+//   softmax      thread r owns query row r: reads its S row from TMEM, keeps
+//                a running max m (rescaling O only when the max grows by more
+//                than 2^8, which is exact: O and l share the reference max),
+//                writes P as 16-bit values back to TMEM
+//   O[128 x D]  += P[128 x 64] . V_step      (tcgen05.mma, A from TMEM)
+// Q and the K/V steps are staged by cp.async in the canonical 128-byte-swizzle
+// layout (8 rows x 128 B atoms; K and V share the physical layout, K is read
+// K-major, V MN-major).  Thread 0 issues the MMAs; tcgen05.commit signals
+// mbarriers.  Every wait is bounded: on timeout the CTA flags
+// PA_DEV_TIMEOUT, lets its copies land, frees its TMEM and returns.
+// ---------------------------------------------------------------------------
+template <int D>
+struct Tc05Shape {
+  static constexpr int kThreads = 128;
+  static constexpr int kRows = 128;                       // MMA M: query rows
+  static constexpr int kStep = 64;                        // tokens per step: MMA1 N, MMA2 K
+  static constexpr int kSteps = kPartition / kStep;       // 8
+  static constexpr int kBlocks = D / 64;                  // 64-element swizzle blocks along head_dim
+  static constexpr int kQBlockBytes = kRows * 128;        // one 64-wide block of Q
+  static constexpr int kQBytes = kBlocks * kQBlockBytes;
+  static constexpr int kKVBlockBytes = kStep * 128;       // one 64-wide block of a K or V step
+  static constexpr int kTileBytes = kBlocks * kKVBlockBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;      // K then V
+  static constexpr int kStages = 2;
+  static constexpr int kBarOffset = kQBytes + kStages * kStageBytes;
+  static constexpr int kSmemBytes = kBarOffset + 64 + 1024;  // + mbarriers, TMEM address, alignment slack
+  static constexpr uint32_t kSCol = 0, kPCol = kStep, kOCol = 128;
+  static constexpr uint32_t kTmemCols = 256;
+  static_assert(kOCol + D <= kTmemCols, "TMEM columns");
+  static_assert(kRows * (D / 8) % kThreads == 0 && 2 * kStep * (D / 8) % kThreads == 0, "copy split");
+};
+
+constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at 2 GHz
+
+template <typename T, int D>
+__global__ void __launch_bounds__(128, 1) decode_shared_tc05_kernel(const DecodeArgs a, const int32_t* __restrict__ chunks,
+                                                                   const int32_t* __restrict__ members,
+                                                                   int num_members, int num_seqs) {
+  using S = Tc05Shape<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const int c = blockIdx.x;
+  const int kvh = blockIdx.y;
+  const int p = blockIdx.z;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int leader = __ldg(chunks + 4 * c);
+  const int moff = __ldg(chunks + 4 * c + 1);
+  const int mcount = __ldg(chunks + 4 * c + 2);
+  const int sp = __ldg(chunks + 4 * c + 3);
+  if (p >= sp) return;
+  const int bs = a.block_size;
+  const int G = a.group;
+  const int tok_begin = p * kPartition;
+  if ((unsigned)leader >= (unsigned)num_seqs || moff < 0 || mcount < 0 || (int64_t)moff + mcount > num_members ||
+      (int64_t)mcount * G > S::kRows || (int64_t)tok_begin + kPartition > (int64_t)a.max_blocks_per_seq * bs ||
+      p >= a.max_partitions) {
+    if (tid == 0) flag_status(a.status, PA_DEV_BAD_PLAN);
+    return;
+  }
+  const int nq = mcount * G;  // real query rows
+  const int first_block = tok_begin / bs;
+  const int nblk = (tok_begin + kPartition - 1) / bs - first_block + 1;  // <= 32 for bs >= 16
+  int lane_page = 0;
+  if (lane < nblk) lane_page = __ldg(a.block_tables + (int64_t)leader * a.max_blocks_per_seq + first_block + lane);
+
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;  // swizzle atoms need 1024-byte alignment
+  const uint32_t q_smem = base;
+  const uint32_t st_smem = base + S::kQBytes;
+  const uint32_t bar_s = base + S::kBarOffset;
+  const uint32_t bar_o = bar_s + 8;
+  const uint32_t taddr_slot = bar_s + 16;
+  uint32_t* taddr_ptr = reinterpret_cast<uint32_t*>(smem_raw + (taddr_slot - raw));
+
+  // Row of q / out for query row r of this chunk, or -1 (padding / bad member).
+  auto query_row = [&](int r) -> int64_t {
+    if (r >= nq) return -1;
+    const int mi = r / G;
+    const int b = __ldg(members + moff + mi);
+    if ((unsigned)b >= (unsigned)num_seqs) return -1;
+    return (int64_t)b * a.num_q_heads + kvh * G + (r - mi * G);
+  };
+
+  // -- set-up: mbarriers, TMEM, Q ------------------------------------------------------
+  if (tid == 0) {
+    tc05::mbar_init(bar_s, 1);
+    tc05::mbar_init(bar_o, 1);
+    tc05::fence_mbar_init();
+  }
+  if (warp == 0) {
+    tc05::alloc(taddr_slot, S::kTmemCols);
+    tc05::relinquish();
+  }
+  {
+    const T* qbase = reinterpret_cast<const T*>(a.q);
+#pragma unroll 4
+    for (int j = 0; j < S::kRows * (D / 8) / S::kThreads; ++j) {
+      const int idx = tid + S::kThreads * j;
+      const int r = idx / (D / 8);
+      const int ck = idx - r * (D / 8);
+      const int64_t row = query_row(r);
+      const T* src = qbase + (row < 0 ? 0 : row) * D + ck * 8;
+      const uint32_t dst = q_smem + (ck >> 3) * S::kQBlockBytes + r * 128 + (((ck & 7) ^ (r & 7)) << 4);
+      cp_async_16(dst, src, row < 0 ? 0u : 16u);
+    }
+  }
+  const T* kc = reinterpret_cast<const T*>(a.key_cache);
+  const T* vc = reinterpret_cast<const T*>(a.value_cache);
+  // Every thread copies its share of step i's K and V rows into stage `stage`.
+  auto load_step = [&](int i, int stage) {
+    const uint32_t kdst = st_smem + stage * S::kStageBytes;
+#pragma unroll 4
+    for (int j = 0; j < 2 * S::kStep * (D / 8) / S::kThreads; ++j) {
+      const int idx = tid + S::kThreads * j;
+      const int half = idx / (S::kStep * (D / 8));  // 0: K, 1: V
+      const int rem = idx - half * (S::kStep * (D / 8));
+      const int t = rem / (D / 8);
+      const int ck = rem - t * (D / 8);
+      const int tok = tok_begin + i * S::kStep + t;
+      int page = __shfl_sync(kFull, lane_page, tok / bs - first_block);
+      const bool ok = (unsigned)page < (unsigned)a.num_blocks;
+      if (!ok) page = 0;
+      const T* src = (half ? vc : kc) + (((int64_t)page * a.num_kv_heads + kvh) * bs + tok % bs) * D + ck * 8;
+      const uint32_t dst =
+          kdst + half * S::kTileBytes + (ck >> 3) * S::kKVBlockBytes + t * 128 + (((ck & 7) ^ (t & 7)) << 4);
+      cp_async_16(dst, src, ok ? 16u : 0u);
+    }
+  };
+  load_step(0, 0);
+  cp_async_commit();  // group: Q + step 0
+
+  tc05::fence_before();
+  __syncthreads();
+  tc05::fence_after();
+  const uint32_t tmem = *taddr_ptr;
+  const uint32_t row_taddr = tmem + ((uint32_t)(32 * warp) << 16);
+  const int row = tid;  // TMEM lane = query row
+  const bool warp_busy = 32 * warp < nq;
+
+  constexpr uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+  constexpr uint32_t idesc_s = tc05::instr_desc_f16(fmt, S::kRows, S::kStep, 0, 0);
+  constexpr uint32_t idesc_o = tc05::instr_desc_f16(fmt, S::kRows, D, 0, 1);
+
+  float m_use = -INFINITY;  // reference max of O and l (base-2 scores)
+  float l = 0.f;
+  int err = 0;
+  for (int i = 0; i < S::kSteps; ++i) {
+    const int stage = i & 1;
+    if (i > 0) {
+      // MMA2 of step i-1 is done: O is current, P and the other stage are free.
+      if (!tc05::mbar_wait_bounded(bar_o, (i - 1) & 1, kWaitCycles)) err = 1;
+      tc05::fence_after();
+    }
+    if (i + 1 < S::kSteps && !err) load_step(i + 1, (i + 1) & 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    tc05::fence_proxy_async_smem();
+    tc05::fence_before();
+    err = __syncthreads_or(err);
+    if (err) break;
+    const uint32_t kst = st_smem + stage * S::kStageBytes;
+    const uint32_t vst = kst + S::kTileBytes;
+    if (tid == 0) {
+      tc05::fence_after();
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t blk = ks >> 2, koff = (ks & 3) * 32;
+        const uint64_t adesc = tc05::smem_desc_sw128(q_smem + blk * S::kQBlockBytes + koff, 16, 1024);
+        const uint64_t bdesc = tc05::smem_desc_sw128(kst + blk * S::kKVBlockBytes + koff, 16, 1024);
+        tc05::mma_ss(tmem + S::kSCol, adesc, bdesc, idesc_s, ks > 0 ? 1u : 0u);
+      }
+      tc05::commit(bar_s);
+    }
+    if (!tc05::mbar_wait_bounded(bar_s, i & 1, kWaitCycles)) err = 1;
+    tc05::fence_after();
+    if (warp_busy && !err) {
+      // Validity of the step's 64 tokens: one bit per 16 tokens (block_size >= 16).
+      const int tok0 = tok_begin + i * S::kStep;
+      uint32_t sreg[2][32];
+      tc05::ld32(row_taddr + S::kSCol, sreg[0]);
+      tc05::ld32(row_taddr + S::kSCol + 32, sreg[1]);
+      tc05::wait_ld();
+      float mx = -INFINITY;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int q4 = 0; q4 < 2; ++q4) {
+          const int tk = tok0 + 32 * h + 16 * q4;
+          const bool ok = (unsigned)__shfl_sync(kFull, lane_page, tk / bs - first_block) < (unsigned)a.num_blocks;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float v = ok ? __uint_as_float(sreg[h][16 * q4 + j]) * a.qk_scale_log2 : -INFINITY;
+            sreg[h][16 * q4 + j] = __float_as_uint(v);
+            mx = fmaxf(mx, v);
+          }
+        }
+      }
+      // Lazy rescaling: keep the reference max unless the new max exceeds it by 8.
+      float alpha = 1.f;
+      if (mx > m_use + 8.f) {
+        alpha = m_use == -INFINITY ? 0.f : exp2f(m_use - mx);
+        m_use = mx;
+      }
+      const float ref = m_use == -INFINITY ? 0.f : m_use;
+      float lsum = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float p0 = exp2f(__uint_as_float(sreg[h][2 * j]) - ref);
+          const float p1 = exp2f(__uint_as_float(sreg[h][2 * j + 1]) - ref);
+          lsum += p0 + p1;
+          pk[16 * h + j] = pack2<T>(p0, p1);
+        }
+      }
+      l = l * alpha + lsum;
+      if (i > 0 && __any_sync(kFull, alpha != 1.f)) {
+#pragma unroll
+        for (int cb = 0; cb < D / 32; ++cb) {
+          uint32_t ov[32];
+          tc05::ld32(row_taddr + S::kOCol + 32 * cb, ov);
+          tc05::wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+          tc05::st32(row_taddr + S::kOCol + 32 * cb, ov);
+        }
+      }
+      tc05::st32(row_taddr + S::kPCol, pk);
+      tc05::wait_st();
+    }
+    tc05::fence_before();
+    err = __syncthreads_or(err);
+    if (err) break;
+    if (tid == 0) {
+      tc05::fence_after();
+#pragma unroll
+      for (int kt = 0; kt < S::kStep / 16; ++kt) {
+        const uint64_t bdesc = tc05::smem_desc_sw128(vst + kt * 16 * 128, S::kKVBlockBytes, 1024);
+        tc05::mma_ts(tmem + S::kOCol, tmem + S::kPCol + 8 * kt, bdesc, idesc_o, (i > 0 || kt > 0) ? 1u : 0u);
+      }
+      tc05::commit(bar_o);
+    }
+  }
+  if (!err && !tc05::mbar_wait_bounded(bar_o, (S::kSteps - 1) & 1, kWaitCycles)) err = 1;
+  err = __syncthreads_or(err);
+  tc05::fence_after();
+  if (!err && warp_busy) {
+    const int64_t qrow = query_row(row);
+    uint32_t ov[32];
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const int64_t part = qrow * a.max_partitions + p;
+#pragma unroll
+    for (int cb = 0; cb < D / 32; ++cb) {
+      tc05::ld32(row_taddr + S::kOCol + 32 * cb, ov);
+      tc05::wait_ld();
+      if (qrow >= 0) {
+        float4* dst = reinterpret_cast<float4*>(a.o_part + part * D + 32 * cb);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          dst[j] = make_float4(__uint_as_float(ov[4 * j]) * inv, __uint_as_float(ov[4 * j + 1]) * inv,
+                               __uint_as_float(ov[4 * j + 2]) * inv, __uint_as_float(ov[4 * j + 3]) * inv);
+      }
+    }
+    if (qrow >= 0) {
+      a.m_part[part] = m_use == -INFINITY ? -INFINITY : m_use * kLn2;
+      a.l_part[part] = l;
+    }
+  }
+  if (err && tid == 0) flag_status(a.status, PA_DEV_TIMEOUT);
+  cp_async_wait<0>();
+  tc05::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc05::fence_after();
+    tc05::dealloc(tmem, S::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Log-sum-exp merge of the partitions.  A CTA of 4 warps serves 4 / WPI
 // (sequence, query head) items with WPI warps each (WPI grows with the
 // partition count).  Warp w of an item merges partitions w, w + WPI, ... with
@@ -950,12 +1241,31 @@ cudaError_t launch_shared(const DecodeArgs& a, dim3 grid, const int32_t* chunks,
   return cudaGetLastError();
 }
 
+template <typename T, int D>
+cudaError_t launch_shared_tc05(const DecodeArgs& a, dim3 grid, const int32_t* chunks, const int32_t* members,
+                               int num_members, int num_seqs, cudaStream_t stream) {
+  using S = Tc05Shape<D>;
+  static std::atomic<uint64_t> done{0};
+  auto kernel = decode_shared_tc05_kernel<T, D>;
+  cudaError_t err = ensure_smem(kernel, S::kSmemBytes, done);
+  if (err != cudaSuccess) return err;
+  kernel<<<grid, S::kThreads, S::kSmemBytes, stream>>>(a, chunks, members, num_members, num_seqs);
+  return cudaGetLastError();
+}
+
+std::atomic<int> g_shared_kernel{PA_SHARED_PREFIX_AUTO};
+
 template <typename T>
 cudaError_t launch_shared_dim(const DecodeArgs& a, int head_dim, dim3 grid, const int32_t* chunks,
                               const int32_t* members, int num_members, int num_seqs, cudaStream_t stream) {
+  const bool tc05 = g_shared_kernel.load() != PA_SHARED_PREFIX_MMA_SYNC;
   switch (head_dim) {
-    case 64: return launch_shared<T, 64>(a, grid, chunks, members, num_members, num_seqs, stream);
-    case 128: return launch_shared<T, 128>(a, grid, chunks, members, num_members, num_seqs, stream);
+    case 64:
+      return tc05 ? launch_shared_tc05<T, 64>(a, grid, chunks, members, num_members, num_seqs, stream)
+                  : launch_shared<T, 64>(a, grid, chunks, members, num_members, num_seqs, stream);
+    case 128:
+      return tc05 ? launch_shared_tc05<T, 128>(a, grid, chunks, members, num_members, num_seqs, stream)
+                  : launch_shared<T, 128>(a, grid, chunks, members, num_members, num_seqs, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -1014,6 +1324,13 @@ extern "C" pa_status pa_set_decode_kernel(pa_decode_kernel k) {
   if (k != PA_DECODE_AUTO && k != PA_DECODE_CUDA_CORES && k != PA_DECODE_TENSOR_CORES)
     return fail(PA_ERR_INVALID, "pa_set_decode_kernel: unknown kernel %d", (int)k);
   g_kernel_choice.store((int)k);
+  return PA_OK;
+}
+
+extern "C" pa_status pa_set_shared_prefix_kernel(pa_shared_prefix_kernel k) {
+  if (k != PA_SHARED_PREFIX_AUTO && k != PA_SHARED_PREFIX_TCGEN05 && k != PA_SHARED_PREFIX_MMA_SYNC)
+    return fail(PA_ERR_INVALID, "pa_set_shared_prefix_kernel: unknown kernel %d", (int)k);
+  g_shared_kernel.store((int)k);
   return PA_OK;
 }
 

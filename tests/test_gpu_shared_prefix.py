@@ -11,6 +11,15 @@ from tests.parity import assert_decode_close, bits_of, host_bits
 
 pytestmark = pytest.mark.gpu
 
+JOINT = {"tcgen05": pa.PA_SHARED_PREFIX_TCGEN05, "mma_sync": pa.PA_SHARED_PREFIX_MMA_SYNC}
+
+
+@pytest.fixture(params=list(JOINT))
+def joint(request):
+    pa.pa_set_shared_prefix_kernel(JOINT[request.param])
+    yield request.param
+    pa.pa_set_shared_prefix_kernel(pa.PA_SHARED_PREFIX_AUTO)
+
 
 @pytest.mark.parametrize("make", [
     lambda: workloads.prefix(num_seqs=5, prefix_len=1700, max_tail=90),
@@ -18,7 +27,7 @@ pytestmark = pytest.mark.gpu
     lambda: workloads.beam32k(num_beams=3, prompt_len=2100, own=40),
     lambda: workloads.beam32k(num_beams=8, prompt_len=1536, own=1),               # prompt = 3 whole partitions
 ], ids=["prefix-5", "prefix-40", "beam-3", "beam-8-exact"])
-def test_shared_flows_match_oracle(make):
+def test_shared_flows_match_oracle(make, joint):
     w = make()
     run = TraceRunner(w, shared_prefix=True)
     out = run.run()
@@ -31,8 +40,8 @@ def test_shared_flows_match_oracle(make):
 
 
 @pytest.mark.parametrize("hq,hkv,d,bs", [(8, 8, 128, 16), (16, 8, 128, 32), (64, 8, 64, 16), (32, 2, 128, 16),
-                                         (64, 4, 128, 64)])
-def test_shared_shapes(hq, hkv, d, bs):
+                                         (64, 4, 128, 64), (128, 8, 128, 16), (32, 8, 64, 32)])
+def test_shared_shapes(hq, hkv, d, bs, joint):
     """G = 1, 2, 8, 16, 16 with head_dim 64 / 128 and several block sizes."""
     import math
     import torch
@@ -69,7 +78,7 @@ def test_shared_shapes(hq, hkv, d, bs):
     assert_decode_close(out, ref, "bf16", f"shared hq{hq} hkv{hkv} d{d} bs{bs}")
 
 
-def test_bad_plan_entries_are_skipped_and_flagged():
+def test_bad_plan_entries_are_skipped_and_flagged(joint):
     """Out-of-range leader / member ranges / partitions are flagged, never dereferenced."""
     import math
     import torch

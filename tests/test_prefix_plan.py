@@ -29,7 +29,7 @@ def _check_plan(a, seqs, group_size, plan):
     bs = a.block_size
     tables = [a.block_table(s) for s in seqs]
     tokens = [a.num_tokens(s) for s in seqs]
-    per_chunk = max(1, 64 // group_size)
+    per_chunk = max(1, 128 // group_size)
     seen = set()
     first = plan["first_partition"]
     for leader, off, count, sp in plan["chunks"][:plan["num_chunks"]]:
@@ -49,7 +49,7 @@ def _check_plan(a, seqs, group_size, plan):
             assert first[i] == 0
 
 
-@pytest.mark.parametrize("name,chunks,sp", [("prefix", 7, 19), ("beam32k", 1, 64), ("llama70b", 0, 0),
+@pytest.mark.parametrize("name,chunks,sp", [("prefix", 4, 19), ("beam32k", 1, 64), ("llama70b", 0, 0),
                                             ("tiny", 0, 0)])
 def test_workload_plans(name, chunks, sp):
     w = workloads.by_name(name)
