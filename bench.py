@@ -52,6 +52,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true", help="skip the nvidia-smi clock record (profiler runs)")
+    ap.add_argument("--micro", action="store_true",
+                    help="instead of the decode step, time the cache write (65,536 tokens) and the page copy "
+                         "(4,096 pairs of 16-token pages) and print one JSON line each")
     ap.add_argument("--shared-prefix", choices=["auto", "on", "off"], default="auto",
                     help="decode shared leading pages once per group (auto: on for prefix/beam32k)")
     return ap.parse_args(argv)
@@ -279,6 +282,95 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------------------------
+# ranks
+# ---------------------------------------------------------------------------------------------
+
+def reduce_over_ranks(step_ms: float, per_rank_units, world: int, device):
+    """Max of the step time and sums of the per-rank unit counts over all ranks.
+
+    Used with NCCL on GPUs by the benchmark; any torch.distributed backend
+    works (the tests run it with gloo on CPU).
+    """
+    import torch
+    import torch.distributed as dist
+    if world <= 1:
+        return float(step_ms), [float(u) for u in per_rank_units]
+    t = torch.tensor([float(step_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    u = torch.tensor([float(x) for x in per_rank_units], dtype=torch.float64, device=device)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t[0]), [float(x) for x in u.tolist()]
+
+
+def rank_workload(name: str, rank: int):
+    """The batch a rank decodes: the named workload, reseeded per rank (weak scaling)."""
+    from paged_kv_cache_356_b200 import workloads
+    base = workloads.by_name(name)
+    return base if rank == 0 else workloads.by_name(name, seed=base.seed + 1000 * rank)
+
+
+# ---------------------------------------------------------------------------------------------
+# cache write / page copy bandwidth
+# ---------------------------------------------------------------------------------------------
+
+def run_micro(args):
+    import torch
+    from paged_kv_cache_356_b200 import binding as pa
+    from paged_kv_cache_356_b200 import build as pa_build
+    pa_build.build()
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    peak, peak_kind = measured_peak()
+    g = torch.Generator(device="cuda").manual_seed(7)
+    hkv, d, bs = 8, 128, 16
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, iters):
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / iters
+
+    # cache write: 65,536 tokens into a shuffled 4,160-page pool
+    t = 65536
+    nb = t // bs + 64
+    key = torch.randn(t, hkv, d, generator=g, device="cuda").to(torch.bfloat16)
+    value = torch.randn(t, hkv, d, generator=g, device="cuda").to(torch.bfloat16)
+    slots = torch.randperm(nb * bs, generator=g, device="cuda")[:t].to(torch.int64)
+    kc = torch.zeros(nb, hkv, bs, d, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    ms = timed(lambda: pa.pa_reshape_and_cache(key, value, slots, kc, vc), args.steps)
+    nbytes = 2 * 2 * t * hkv * d * 2
+    print(json.dumps({"metric": "reshape_and_cache GB/s", "value": nbytes / ms / 1e6, "unit": "GB/s",
+                      "ms_per_call": ms, "bytes_per_call": nbytes, "frac_of_hbm": nbytes / ms / 1e6 / peak,
+                      "peak": peak, "peak_kind": peak_kind,
+                      "config": {"tokens": t, "num_kv_heads": hkv, "head_dim": d, "block_size": bs,
+                                 "dtype": "bf16", "l2": "no flush: 1.07 GB moved per call"}}), flush=True)
+    del key, value, slots, kc, vc
+
+    # page copy: 4,096 (src, dst) pairs of 16-token pages
+    pairs = 4096
+    nb = 2 * pairs + 64
+    kc = torch.randn(nb, hkv, bs, d, generator=g, device="cuda").to(torch.bfloat16)
+    vc = torch.randn(nb, hkv, bs, d, generator=g, device="cuda").to(torch.bfloat16)
+    perm = torch.randperm(nb, generator=g, device="cuda")
+    mapping = torch.stack([perm[:pairs], perm[pairs:2 * pairs]], dim=1).to(torch.int64).contiguous()
+    ms = timed(lambda: pa.pa_copy_blocks(kc, vc, mapping), args.steps)
+    nbytes = 2 * 2 * pairs * hkv * bs * d * 2
+    print(json.dumps({"metric": "copy_blocks GB/s", "value": nbytes / ms / 1e6, "unit": "GB/s",
+                      "ms_per_call": ms, "bytes_per_call": nbytes, "frac_of_hbm": nbytes / ms / 1e6 / peak,
+                      "peak": peak, "peak_kind": peak_kind,
+                      "config": {"pairs": pairs, "num_kv_heads": hkv, "head_dim": d, "block_size": bs,
+                                 "dtype": "bf16", "l2": "no flush: 537 MB moved per call"}}), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------------------------
 
@@ -304,8 +396,7 @@ def run_ours(args):
     warps, stages = (int(x) for x in args.tiling.split("x"))
     pa.pa_set_decode_tiling(warps, stages)
 
-    seed_shift = 1000 * rank
-    w = workloads.by_name(args.workload, seed=workloads.by_name(args.workload).seed + seed_shift)
+    w = rank_workload(args.workload, rank)
     shared = args.shared_prefix == "on" or (args.shared_prefix == "auto" and w.kind in ("prefix", "beam"))
     run = TraceRunner(w, shared_prefix=shared)
     run.run(decode=False)
@@ -374,15 +465,7 @@ def run_ours(args):
     part_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
     reduce_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
 
-    t = torch.tensor([total_ms, float(unique), float(w.num_seqs)], dtype=torch.float64, device="cuda")
-    if world > 1:
-        tmax = t[:1].clone()
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-        tsum = t[1:].clone()
-        dist.all_reduce(tsum, op=dist.ReduceOp.SUM)
-        total_ms_max, all_unique, all_seqs = float(tmax[0]), float(tsum[0]), float(tsum[1])
-    else:
-        total_ms_max, all_unique, all_seqs = total_ms, float(unique), float(w.num_seqs)
+    total_ms_max, (all_unique, all_seqs) = reduce_over_ranks(total_ms, [unique, w.num_seqs], world, "cuda")
     seconds = total_ms_max / 1000.0
     value = all_unique * args.steps / seconds / 1e9
     seqs_per_s = all_seqs * args.steps / seconds
@@ -482,13 +565,7 @@ def end_to_end(args, torch, pa, run, w, unique, max_ctx, world, dist):
     for _ in range(args.steps):
         e2e_step()
     elapsed = time.perf_counter() - t0
-    el = torch.tensor([elapsed, float(unique)], dtype=torch.float64, device="cuda")
-    if world > 1:
-        mx = el[:1].clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        sm = el[1:].clone()
-        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
-        elapsed, unique = float(mx[0]), float(sm[0])
+    elapsed, (unique,) = reduce_over_ranks(elapsed, [unique], world, "cuda")
     h2d = sum(x.numel() * x.element_size() for x in (h_q, h_k, h_v, h_s, h_tab, h_ctx))
     d2h = h_out.numel() * h_out.element_size()
     return {"value": unique * args.steps / elapsed / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -501,6 +578,8 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.micro:
+        return run_micro(args)
     return run_ours(args)
 
 
