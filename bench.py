@@ -57,6 +57,8 @@ def parse_args(argv=None):
                          "(4,096 pairs of 16-token pages) and print one JSON line each")
     ap.add_argument("--shared-prefix", choices=["auto", "on", "off"], default="auto",
                     help="decode shared leading pages once per group (auto: on for prefix/beam32k)")
+    ap.add_argument("--joint-kernel", choices=["auto", "tcgen05", "tcgen05_serial", "mma_sync"], default="auto",
+                    help="kernel for the shared partitions of a prefix group")
     return ap.parse_args(argv)
 
 
@@ -395,6 +397,9 @@ def run_ours(args):
                              "cc": pa.PA_DECODE_CUDA_CORES}[args.kernel])
     warps, stages = (int(x) for x in args.tiling.split("x"))
     pa.pa_set_decode_tiling(warps, stages)
+    pa.pa_set_shared_prefix_kernel({"auto": pa.PA_SHARED_PREFIX_AUTO, "tcgen05": pa.PA_SHARED_PREFIX_TCGEN05,
+                                    "tcgen05_serial": pa.PA_SHARED_PREFIX_TCGEN05_SERIAL,
+                                    "mma_sync": pa.PA_SHARED_PREFIX_MMA_SYNC}[args.joint_kernel])
 
     w = rank_workload(args.workload, rank)
     shared = args.shared_prefix == "on" or (args.shared_prefix == "auto" and w.kind in ("prefix", "beam"))
@@ -489,6 +494,8 @@ def run_ours(args):
         cfg.update({"parallelism": f"dp{world} (independent batches per GPU, no collective)",
                     "l2": "no flush: each step reads the whole KV cache, far larger than the 126 MB L2",
                     "kernel": args.kernel, "tiling": args.tiling, "global_batch": w.num_seqs * world})
+        if run.plan is not None:
+            cfg["joint_kernel"] = args.joint_kernel
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,

@@ -263,13 +263,17 @@ PA_API pa_status pa_decode_shared_prefix(const void* q, const void* key_cache, c
                                          int32_t* dev_status, void* stream);
 
 /* Which joint kernel pa_decode_shared_prefix runs (process-wide; default
- * AUTO = TCGEN05): the 5th-generation tensor-core kernel (tcgen05.mma with
- * Tensor Memory accumulators) or the mma.sync kernel.  Both compute the same
- * partials; the switch exists for testing and measurement. */
+ * AUTO = TCGEN05): TCGEN05 is the pipelined persistent kernel on the 5th-
+ * generation tensor cores (TMA loads, tcgen05.mma with Tensor Memory
+ * accumulators, one CTA per SM); TCGEN05_SERIAL the one-partition-per-CTA
+ * tcgen05 kernel without the software pipeline; MMA_SYNC the mma.sync
+ * kernel.  All compute the same partials; the switch exists for testing and
+ * measurement. */
 typedef enum pa_shared_prefix_kernel {
   PA_SHARED_PREFIX_AUTO = 0,
   PA_SHARED_PREFIX_TCGEN05 = 1,
-  PA_SHARED_PREFIX_MMA_SYNC = 2
+  PA_SHARED_PREFIX_MMA_SYNC = 2,
+  PA_SHARED_PREFIX_TCGEN05_SERIAL = 3
 } pa_shared_prefix_kernel;
 PA_API pa_status pa_set_shared_prefix_kernel(pa_shared_prefix_kernel kernel);
 

@@ -36,6 +36,9 @@
 #include <type_traits>
 #include <mutex>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "device.cuh"
 #include "pa_internal.h"
 #include "tcgen05.cuh"
@@ -1035,6 +1038,463 @@ __global__ void __launch_bounds__(128, 1) decode_shared_tc05_kernel(const Decode
 }
 
 // ---------------------------------------------------------------------------
+// Warp-specialised, persistent shared-prefix kernel on tcgen05 (the default
+// joint kernel).  One CTA per SM walks work items (chunk, kv head, shared
+// partition) with stride gridDim.x; an item is 8 steps of 64 tokens.  Roles:
+//   warps 0-3  softmax: thread r owns query row r; per step it reads its S row
+//              from TMEM, keeps the running max / sum (lazy rescaling of O),
+//              writes P (16-bit) to TMEM; at the end of an item it writes the
+//              partials.
+//   warp 4     producer: K/V pages by TMA (16 lanes issue the step's 16 boxes
+//              at once) into a ring of STAGES buffers, as far ahead as the
+//              ring allows; three steps before an item ends it starts the
+//              next item's queries (cp.async) and table slice into the other
+//              query buffer, so the ring keeps filling across item boundaries.
+//   warp 5     MMA issuer (one lane): S(g) = Q.K^T into S[g & 1], then
+//              O += P(g-1).V(g-1), so the tensor cores work on step g while
+//              the softmax warps finish step g-1; an item's last O += P.V is
+//              issued before the next item starts.
+// Hand-offs are mbarriers, one per buffer, each waited at most one phase
+// behind its next completion: s_full / s_free (S), p_full (P), o_done (MMA2,
+// frees P, makes O current), kv_full / kv_empty (ring), q_full (queries and
+// table slice), item_free (O and Q of an item read out).  Every wait is
+// bounded; a timeout raises an abort flag that every role polls, then the CTA
+// flags PA_DEV_TIMEOUT, lets its TMA loads land, frees TMEM and returns.
+// ---------------------------------------------------------------------------
+template <int D, int STAGES>
+struct Tc05pShape {
+  static constexpr int kThreads = 192;
+  static constexpr int kRows = 128;
+  static constexpr int kStep = 64;
+  static constexpr int kStepsPerItem = kPartition / kStep;  // 8
+  static constexpr int kBlocks = D / 64;
+  static constexpr int kQBlockBytes = kRows * 128;
+  static constexpr int kQBytes = kBlocks * kQBlockBytes;
+  static constexpr int kKVBlockBytes = kStep * 128;
+  static constexpr int kTileBytes = kBlocks * kKVBlockBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kBoxBytes = 16 * 128;                 // one TMA box: 16 rows x 64 elements
+  static constexpr int kBoxesPerStep = 2 * (kStep / 16) * kBlocks;
+  static constexpr int kQOff = 0;
+  static constexpr int kStageOff = 2 * kQBytes;
+  static constexpr int kSliceOff = kStageOff + STAGES * kStageBytes;  // int32 [2][32]
+  static constexpr int kBarOff = kSliceOff + 256;
+  static constexpr int kNumBars = 2 * 5 + 2 * STAGES;         // s_full, s_free, p_full, o_done, q_full/item_free x2; kv x STAGES
+  static constexpr int kTaddrOff = kBarOff + 8 * (kNumBars + 2);
+  static constexpr int kSmemBytes = kTaddrOff + 16 + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kSCol = 0, kPCol = 128, kOCol = 256;  // S[b] at 64b, P[b] at 128 + 32b, O[b] at 256 + 128b
+  static_assert(D <= 128, "O double buffer needs D <= 128");
+  static_assert(kBoxesPerStep <= 32, "one lane per box");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+struct SharedItem {
+  int c, kvh, p, leader, moff, mcount;
+  bool valid;
+};
+
+// The next usable work item at or after `cursor` (stride gridDim.x), in the
+// order (partition, kv head, chunk) so concurrent CTAs share pages through L2.
+// Entries that would index outside an array are reported and skipped.
+__device__ __forceinline__ SharedItem next_shared_item(int64_t& cursor, int64_t total, int num_chunks,
+                                                       const DecodeArgs& a, const int32_t* __restrict__ chunks,
+                                                       int num_members, int num_seqs, bool report) {
+  SharedItem it{};
+  it.valid = false;
+  while (cursor < total) {
+    const int64_t w = cursor;
+    cursor += gridDim.x;
+    const int c = (int)(w % num_chunks);
+    const int64_t rest = w / num_chunks;
+    const int kvh = (int)(rest % a.num_kv_heads);
+    const int p = (int)(rest / a.num_kv_heads);
+    if (p >= __ldg(chunks + 4 * c + 3)) continue;
+    it.c = c;
+    it.kvh = kvh;
+    it.p = p;
+    it.leader = __ldg(chunks + 4 * c);
+    it.moff = __ldg(chunks + 4 * c + 1);
+    it.mcount = __ldg(chunks + 4 * c + 2);
+    const bool ok = (unsigned)it.leader < (unsigned)num_seqs && it.moff >= 0 && it.mcount >= 0 &&
+                    (int64_t)it.moff + it.mcount <= num_members && (int64_t)it.mcount * a.group <= 128 &&
+                    (int64_t)(p + 1) * kPartition <= (int64_t)a.max_blocks_per_seq * a.block_size &&
+                    p < a.max_partitions;
+    if (!ok) {
+      if (report) flag_status(a.status, PA_DEV_BAD_PLAN);
+      continue;
+    }
+    it.valid = true;
+    return it;
+  }
+  return it;
+}
+
+template <typename T, int D, int STAGES>
+__global__ void __launch_bounds__(192, 1)
+    decode_shared_tc05p_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
+                               const __grid_constant__ CUtensorMap tmap_v, const int32_t* __restrict__ chunks,
+                               int num_chunks, const int32_t* __restrict__ members, int num_members, int num_seqs,
+                               int max_shared_partitions) {
+  using S = Tc05pShape<D, STAGES>;
+  constexpr int SPI = S::kStepsPerItem;
+  static_assert(SPI >= 3, "the next item's queries are loaded three steps before the item ends");
+  extern __shared__ uint8_t smem_raw[];
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int bs = a.block_size;
+  const int G = a.group;
+  const int64_t total_rows = (int64_t)a.num_blocks * a.num_kv_heads * bs;
+  const int64_t total_items = (int64_t)max_shared_partitions * a.num_kv_heads * num_chunks;
+
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  int32_t* tslice = reinterpret_cast<int32_t*>(base_ptr + S::kSliceOff);  // [2][32]
+  const uint32_t bar0 = base + S::kBarOff;
+  auto s_full = [&](int b) { return bar0 + 8u * b; };
+  auto s_free = [&](int b) { return bar0 + 16u + 8u * b; };
+  auto p_full = [&](int b) { return bar0 + 32u + 8u * b; };
+  auto o_done = [&](int b) { return bar0 + 48u + 8u * b; };
+  auto q_full = [&](int b) { return bar0 + 64u + 8u * b; };
+  auto item_free = [&](int b) { return bar0 + 80u + 8u * b; };
+  auto kv_full = [&](int st) { return bar0 + 96u + 8u * st; };
+  auto kv_empty = [&](int st) { return bar0 + 96u + 8u * STAGES + 8u * st; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + S::kTaddrOff + 8);
+  const uint32_t taddr_slot = base + S::kTaddrOff;
+
+  // Bounded wait that also gives up once another role has aborted.
+  auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    const long long t0 = clock64();
+    while (!tc05::mbar_try_wait(bar, parity)) {
+      if (*abort_flag) return false;
+      if (clock64() - t0 > kWaitCycles) {
+        *abort_flag = 1;
+        return false;
+      }
+    }
+    return true;
+  };
+
+  // Warp-uniform form of `wait` for the softmax and producer warps: every lane
+  // waits (bounded) and the warp agrees on the outcome, so a break is taken by
+  // all 32 lanes together and no lane is left behind at a __syncwarp.
+  auto wwait = [&](uint32_t bar, uint32_t parity) -> bool { return __all_sync(kFull, wait(bar, parity)); };
+
+  // -- set-up -----------------------------------------------------------------------------------
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b) {
+      tc05::mbar_init(s_full(b), 1);
+      tc05::mbar_init(s_free(b), 4);     // one arrival per softmax warp
+      tc05::mbar_init(p_full(b), 4);
+      tc05::mbar_init(o_done(b), 1);
+      tc05::mbar_init(q_full(b), 1);     // the producer warp's lane 0
+      tc05::mbar_init(item_free(b), 4);
+    }
+    for (int st = 0; st < STAGES; ++st) {
+      tc05::mbar_init(kv_full(st), 1);
+      tc05::mbar_init(kv_empty(st), 1);
+    }
+    *abort_flag = 0;
+    tc05::fence_mbar_init();
+    tc05::prefetch_tensormap(&tmap_k);
+    tc05::prefetch_tensormap(&tmap_v);
+  }
+  if (warp == 0) {
+    tc05::alloc(taddr_slot, S::kTmemCols);
+    tc05::relinquish();
+  }
+  tc05::fence_before();
+  __syncthreads();
+  tc05::fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base_ptr + S::kTaddrOff);
+
+  int64_t cursor = blockIdx.x;
+  int64_t prod_g = 0;  // producer: steps whose loads have been issued
+  if (warp == 4) {
+    // ---------------------------------------------------------------- producer
+    const T* qbase = reinterpret_cast<const T*>(a.q);
+    // Queries (rows past mcount * G are zero) and table slice of `it` into buffer qb.
+    // Each lane owns rows lane + 32k: one member lookup per row, then its chunks.
+    auto load_q = [&](const SharedItem& it, int qb) {
+      const uint32_t qs = base + S::kQOff + qb * S::kQBytes;
+#pragma unroll
+      for (int k = 0; k < S::kRows / 32; ++k) {
+        const int r = lane + 32 * k;
+        int64_t row = -1;
+        if (r < it.mcount * G) {
+          const int mi = r / G;
+          const int b = __ldg(members + it.moff + mi);
+          if ((unsigned)b < (unsigned)num_seqs) row = (int64_t)b * a.num_q_heads + it.kvh * G + (r - mi * G);
+        }
+        const T* src = qbase + (row < 0 ? 0 : row) * D;
+#pragma unroll
+        for (int ck = 0; ck < D / 8; ++ck)
+          cp_async_16(qs + (ck >> 3) * S::kQBlockBytes + r * 128 + (((ck & 7) ^ (r & 7)) << 4), src + ck * 8,
+                      row < 0 ? 0u : 16u);
+      }
+      const int fb = it.p * kPartition / bs;
+      const int nblk = (it.p * kPartition + kPartition - 1) / bs - fb + 1;
+      tslice[qb * 32 + lane] =
+          lane < nblk ? __ldg(a.block_tables + (int64_t)it.leader * a.max_blocks_per_seq + fb + lane) : -1;
+      cp_async_commit();
+    };
+    auto publish_q = [&](int qb) {  // after load_q: make it visible, then signal
+      cp_async_wait<0>();
+      tc05::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(q_full(qb)) : "memory");
+    };
+    SharedItem it = next_shared_item(cursor, total_items, num_chunks, a, chunks, num_members, num_seqs, lane == 0);
+    if (it.valid) {
+      load_q(it, 0);
+      publish_q(0);
+    }
+    int64_t g = 0;
+    for (int j = 0; it.valid; ++j) {
+      const int qb = j & 1;
+      const SharedItem nxt =
+          next_shared_item(cursor, total_items, num_chunks, a, chunks, num_members, num_seqs, lane == 0);
+      const int fb = it.p * kPartition / bs;
+      const int my_page = tslice[qb * 32 + lane];
+      bool stop = false;
+      for (int i = 0; i < SPI; ++i, ++g) {
+        const int st = (int)(g % STAGES);
+        if (g >= STAGES && !wwait(kv_empty(st), (uint32_t)(((g - STAGES) / STAGES) & 1))) { stop = true; break; }
+        if (lane == 0) tc05::mbar_arrive_expect_tx(kv_full(st), S::kStageBytes);
+        // lane -> (row box rb, 64-wide block blk, K or V); lanes past the boxes idle
+        const int kv = lane & 1;
+        const int blk = (lane >> 1) % S::kBlocks;
+        const int rb = ((lane >> 1) / S::kBlocks) % (S::kStep / 16);
+        const int tok = it.p * kPartition + i * S::kStep + 16 * rb;
+        const int page = __shfl_sync(kFull, my_page, tok / bs - fb);
+        __syncwarp();
+        if (lane < S::kBoxesPerStep) {
+          const int64_t y = (unsigned)page < (unsigned)a.num_blocks
+                                ? ((int64_t)page * a.num_kv_heads + it.kvh) * bs + tok % bs
+                                : total_rows;  // out of range: the box is filled with zeros
+          const uint32_t dst = base + S::kStageOff + st * S::kStageBytes + kv * S::kTileBytes +
+                               blk * S::kKVBlockBytes + rb * S::kBoxBytes;
+          tc05::tma_load_2d(dst, kv ? (const void*)&tmap_v : (const void*)&tmap_k, kv_full(st), 64 * blk, (int32_t)y);
+        }
+        __syncwarp();
+        prod_g = g + 1;
+        // Mid-item: the next item's queries go into the other buffer once the
+        // item that last used it (j - 1) has been read out.
+        if (i == SPI - 3 && nxt.valid) {
+          if (j >= 1 && !wwait(item_free(qb ^ 1), (uint32_t)(((j - 1) >> 1) & 1))) { stop = true; break; }
+          load_q(nxt, qb ^ 1);
+        }
+      }
+      if (stop || __any_sync(kFull, *abort_flag != 0)) break;
+      if (nxt.valid) publish_q(qb ^ 1);
+      it = nxt;
+    }
+    cp_async_wait<0>();  // nothing may land in shared memory after the CTA leaves
+  } else if (warp == 5) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+      constexpr uint32_t idesc_s = tc05::instr_desc_f16(fmt, S::kRows, S::kStep, 0, 0);
+      constexpr uint32_t idesc_o = tc05::instr_desc_f16(fmt, S::kRows, D, 0, 1);
+      auto mma2 = [&](int64_t gp) -> bool {  // O[item of gp] += P(gp) . V(gp)
+        if (!wait(p_full((int)(gp & 1)), (uint32_t)((gp >> 1) & 1))) return false;
+        tc05::fence_after();
+        const int st = (int)(gp % STAGES);
+        const uint32_t vs = base + S::kStageOff + st * S::kStageBytes + S::kTileBytes;
+        const uint32_t ocol = S::kOCol + 128u * (uint32_t)((gp / SPI) & 1);
+        const int ip = (int)(gp % SPI);
+#pragma unroll
+        for (int kt = 0; kt < S::kStep / 16; ++kt)
+          tc05::mma_ts(tmem + ocol, tmem + S::kPCol + 32 * (uint32_t)(gp & 1) + 8 * kt,
+                       tc05::smem_desc_sw128(vs + kt * 16 * 128, S::kKVBlockBytes, 1024), idesc_o,
+                       (ip > 0 || kt > 0) ? 1u : 0u);
+        tc05::commit(o_done((int)(gp & 1)));
+        tc05::commit(kv_empty(st));
+        return true;
+      };
+      int64_t g = 0;
+      bool ok = true;
+      for (int j = 0; ok; ++j) {
+        const SharedItem it = next_shared_item(cursor, total_items, num_chunks, a, chunks, num_members, num_seqs,
+                                               false);
+        if (!it.valid) break;
+        const int qb = j & 1;
+        if (!wait(q_full(qb), (uint32_t)((j >> 1) & 1))) break;
+        tc05::fence_after();
+        tc05::fence_proxy_async_smem();
+        const uint32_t qs = base + S::kQOff + qb * S::kQBytes;
+        for (int i = 0; i < SPI; ++i, ++g) {
+          const int st = (int)(g % STAGES);
+          if (!wait(kv_full(st), (uint32_t)((g / STAGES) & 1))) { ok = false; break; }
+          if (g >= 2 && !wait(s_free((int)(g & 1)), (uint32_t)(((g - 2) >> 1) & 1))) { ok = false; break; }
+          tc05::fence_after();
+          const uint32_t ks = base + S::kStageOff + st * S::kStageBytes;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t blk = k >> 2, koff = (k & 3) * 32;
+            tc05::mma_ss(tmem + S::kSCol + 64 * (uint32_t)(g & 1),
+                         tc05::smem_desc_sw128(qs + blk * S::kQBlockBytes + koff, 16, 1024),
+                         tc05::smem_desc_sw128(ks + blk * S::kKVBlockBytes + koff, 16, 1024), idesc_s,
+                         k > 0 ? 1u : 0u);
+          }
+          tc05::commit(s_full((int)(g & 1)));
+          if (i >= 1 && !mma2(g - 1)) { ok = false; break; }
+        }
+        // Close the item (its epilogue must not wait for the next item's queries).
+        if (ok && !mma2(g - 1)) ok = false;
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax warps 0-3
+    const uint32_t row_t = tmem + ((uint32_t)(32 * warp) << 16);
+    int64_t g = 0;
+    for (int j = 0;; ++j) {
+      const SharedItem it = next_shared_item(cursor, total_items, num_chunks, a, chunks, num_members, num_seqs,
+                                             false);
+      if (!it.valid) break;
+      const int qb = j & 1;
+      const bool busy = 32 * warp < it.mcount * G;
+      if (!wwait(q_full(qb), (uint32_t)((j >> 1) & 1))) break;  // table slice of the item
+      float m_use = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int i = 0; i < SPI; ++i, ++g) {
+        if (!wwait(s_full((int)(g & 1)), (uint32_t)((g >> 1) & 1))) { ok = false; break; }
+        tc05::fence_after();
+        uint32_t sreg[2][32];
+        if (busy) {
+          tc05::ld32(row_t + S::kSCol + 64 * (uint32_t)(g & 1), sreg[0]);
+          tc05::ld32(row_t + S::kSCol + 64 * (uint32_t)(g & 1) + 32, sreg[1]);
+          tc05::wait_ld();
+        }
+        tc05::fence_before();
+        __syncwarp();
+        if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(s_free((int)(g & 1))) : "memory");
+        uint32_t pk[32];
+        float alpha = 1.f;
+        if (busy) {
+          const int tok0 = it.p * kPartition + i * S::kStep;
+          const int fb = it.p * kPartition / bs;
+          float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int page = tslice[qb * 32 + (tok0 + 16 * q4) / bs - fb];
+            const bool okp = (unsigned)page < (unsigned)a.num_blocks;
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              const int e = 16 * q4 + jj;
+              const float v = okp ? __uint_as_float(sreg[e >> 5][e & 31]) * a.qk_scale_log2 : -INFINITY;
+              sreg[e >> 5][e & 31] = __float_as_uint(v);
+              mx4[jj & 3] = fmaxf(mx4[jj & 3], v);
+            }
+          }
+          const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+          if (mx > m_use + 8.f) {
+            alpha = m_use == -INFINITY ? 0.f : exp2f(m_use - mx);
+            m_use = mx;
+          }
+          const float ref = m_use == -INFINITY ? 0.f : m_use;
+          float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) {
+            const int e0 = 2 * jj, e1 = 2 * jj + 1;
+            const float p0 = exp2f(__uint_as_float(sreg[e0 >> 5][e0 & 31]) - ref);
+            const float p1 = exp2f(__uint_as_float(sreg[e1 >> 5][e1 & 31]) - ref);
+            ls[jj & 3] += p0 + p1;
+            pk[jj] = pack2<T>(p0, p1);
+          }
+          l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+        }
+        if (busy && i > 0 && __any_sync(kFull, alpha != 1.f)) {
+          // O is current once O += P.V of step g - 1 has completed.
+          if (!wwait(o_done((int)((g - 1) & 1)), (uint32_t)(((g - 1) >> 1) & 1))) { ok = false; break; }
+          tc05::fence_after();
+          const uint32_t ocol = S::kOCol + 128u * (uint32_t)qb;
+#pragma unroll
+          for (int cb = 0; cb < D / 32; ++cb) {
+            uint32_t ov[32];
+            tc05::ld32(row_t + ocol + 32 * cb, ov);
+            tc05::wait_ld();
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) ov[jj] = __float_as_uint(__uint_as_float(ov[jj]) * alpha);
+            tc05::st32(row_t + ocol + 32 * cb, ov);
+          }
+        }
+        // P buffer g & 1 was last read by O += P.V of step g - 2.
+        if (g >= 2 && !wwait(o_done((int)(g & 1)), (uint32_t)(((g - 2) >> 1) & 1))) { ok = false; break; }
+        tc05::fence_after();
+        if (busy) {
+          tc05::st32(row_t + S::kPCol + 32 * (uint32_t)(g & 1), pk);
+          tc05::wait_st();
+        }
+        tc05::fence_before();
+        __syncwarp();
+        if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(p_full((int)(g & 1))) : "memory");
+      }
+      if (!ok) break;
+      // Epilogue: the item's last O += P.V (step g - 1) has to complete.
+      const int64_t gl = g - 1;
+      if (!wwait(o_done((int)(gl & 1)), (uint32_t)((gl >> 1) & 1))) break;
+      tc05::fence_after();
+      if (busy) {
+        int64_t qrow = -1;
+        if (tid < it.mcount * G) {
+          const int mi = tid / G;
+          const int b = __ldg(members + it.moff + mi);
+          if ((unsigned)b < (unsigned)num_seqs) qrow = (int64_t)b * a.num_q_heads + it.kvh * G + (tid - mi * G);
+        }
+        const int64_t part = qrow * a.max_partitions + it.p;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const uint32_t ocol = S::kOCol + 128u * (uint32_t)qb;
+#pragma unroll
+        for (int cb = 0; cb < D / 32; ++cb) {
+          uint32_t ov[32];
+          tc05::ld32(row_t + ocol + 32 * cb, ov);
+          tc05::wait_ld();
+          if (qrow >= 0) {
+            float4* dst = reinterpret_cast<float4*>(a.o_part + part * D + 32 * cb);
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+              dst[jj] = make_float4(__uint_as_float(ov[4 * jj]) * inv, __uint_as_float(ov[4 * jj + 1]) * inv,
+                                    __uint_as_float(ov[4 * jj + 2]) * inv, __uint_as_float(ov[4 * jj + 3]) * inv);
+          }
+        }
+        if (qrow >= 0) {
+          a.m_part[part] = m_use == -INFINITY ? -INFINITY : m_use * kLn2;
+          a.l_part[part] = l;
+        }
+      }
+      tc05::fence_before();
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(item_free(qb)) : "memory");
+    }
+  }
+
+  // -- teardown ---------------------------------------------------------------------------------
+  __syncthreads();
+  if (*abort_flag) {
+    if (tid == 0) flag_status(a.status, PA_DEV_TIMEOUT);
+    // Let the TMA loads still in the ring land before the shared memory is released
+    // (the last STAGES issued steps; each stage's latest phase is at most one behind).
+    if (warp == 4 && lane == 0)
+      for (int64_t gl = prod_g > STAGES ? prod_g - STAGES : 0; gl < prod_g; ++gl) {
+        const long long t0 = clock64();
+        while (!tc05::mbar_try_wait(kv_full((int)(gl % STAGES)), (uint32_t)((gl / STAGES) & 1)) &&
+               clock64() - t0 < kWaitCycles) {
+        }
+      }
+  }
+  cp_async_wait<0>();
+  tc05::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc05::fence_after();
+    tc05::dealloc(tmem, S::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Log-sum-exp merge of the partitions.  A CTA of 4 warps serves 4 / WPI
 // (sequence, query head) items with WPI warps each (WPI grows with the
 // partition count).  Warp w of an item merges partitions w, w + WPI, ... with
@@ -1253,12 +1713,85 @@ cudaError_t launch_shared_tc05(const DecodeArgs& a, dim3 grid, const int32_t* ch
   return cudaGetLastError();
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
+  PFN_cuTensorMapEncodeTiled_v12000 f = fn.load();
+  if (!f) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess && ptr) {
+      f = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+      fn.store(f);
+    }
+  }
+  return f;
+}
+
+// 2-D map of a cache viewed as [num_blocks * num_kv_heads * block_size rows][head_dim],
+// boxes of 16 rows x 64 elements (one 128-byte-swizzle block of 16 tokens).
+bool encode_cache_map(CUtensorMap* map, const void* cache, pa_dtype dtype, int64_t rows, int head_dim) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+  const cuuint32_t box[2] = {64, 16};
+  const cuuint32_t elem[2] = {1, 1};
+  return encode(map, dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                const_cast<void*>(cache), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  int n = cached[dev].load();
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev].store(n);
+  }
+  return n;
+}
+
+template <typename T, int D>
+cudaError_t launch_shared_tc05p(const DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, int num_chunks,
+                                const int32_t* chunks, const int32_t* members, int num_members, int num_seqs,
+                                int max_sp, cudaStream_t stream) {
+  constexpr int kStages = 4;
+  using S = Tc05pShape<D, kStages>;
+  static std::atomic<uint64_t> done{0};
+  auto kernel = decode_shared_tc05p_kernel<T, D, kStages>;
+  cudaError_t err = ensure_smem(kernel, S::kSmemBytes, done);
+  if (err != cudaSuccess) return err;
+  const int64_t items = (int64_t)max_sp * a.num_kv_heads * num_chunks;
+  const int grid = (int)(items < sm_count() ? items : sm_count());
+  kernel<<<grid, S::kThreads, S::kSmemBytes, stream>>>(a, mk, mv, chunks, num_chunks, members, num_members, num_seqs,
+                                                       max_sp);
+  return cudaGetLastError();
+}
+
 std::atomic<int> g_shared_kernel{PA_SHARED_PREFIX_AUTO};
 
 template <typename T>
 cudaError_t launch_shared_dim(const DecodeArgs& a, int head_dim, dim3 grid, const int32_t* chunks,
-                              const int32_t* members, int num_members, int num_seqs, cudaStream_t stream) {
-  const bool tc05 = g_shared_kernel.load() != PA_SHARED_PREFIX_MMA_SYNC;
+                              const int32_t* members, int num_members, int num_seqs, pa_dtype dtype,
+                              cudaStream_t stream) {
+  const int choice = g_shared_kernel.load();
+  if (choice == PA_SHARED_PREFIX_AUTO || choice == PA_SHARED_PREFIX_TCGEN05) {
+    const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * a.block_size;
+    CUtensorMap mk, mv;
+    if (rows < (1ll << 31) && encode_cache_map(&mk, a.key_cache, dtype, rows, head_dim) &&
+        encode_cache_map(&mv, a.value_cache, dtype, rows, head_dim)) {
+      if (head_dim == 64)
+        return launch_shared_tc05p<T, 64>(a, mk, mv, grid.x, chunks, members, num_members, num_seqs, grid.z, stream);
+      if (head_dim == 128)
+        return launch_shared_tc05p<T, 128>(a, mk, mv, grid.x, chunks, members, num_members, num_seqs, grid.z, stream);
+    }
+  }
+  const bool tc05 = choice != PA_SHARED_PREFIX_MMA_SYNC;
   switch (head_dim) {
     case 64:
       return tc05 ? launch_shared_tc05<T, 64>(a, grid, chunks, members, num_members, num_seqs, stream)
@@ -1328,7 +1861,8 @@ extern "C" pa_status pa_set_decode_kernel(pa_decode_kernel k) {
 }
 
 extern "C" pa_status pa_set_shared_prefix_kernel(pa_shared_prefix_kernel k) {
-  if (k != PA_SHARED_PREFIX_AUTO && k != PA_SHARED_PREFIX_TCGEN05 && k != PA_SHARED_PREFIX_MMA_SYNC)
+  if (k != PA_SHARED_PREFIX_AUTO && k != PA_SHARED_PREFIX_TCGEN05 && k != PA_SHARED_PREFIX_MMA_SYNC &&
+      k != PA_SHARED_PREFIX_TCGEN05_SERIAL)
     return fail(PA_ERR_INVALID, "pa_set_shared_prefix_kernel: unknown kernel %d", (int)k);
   g_shared_kernel.store((int)k);
   return PA_OK;
@@ -1592,8 +2126,9 @@ extern "C" pa_status pa_decode_shared_prefix(const void* q, const void* key_cach
     if (!aligned16(chunks)) return fail(PA_ERR_INVALID, "decode_shared_prefix: chunks must be 16-byte aligned");
     dim3 grid(num_chunks, num_kv_heads, max_shared_partitions < partitions ? max_shared_partitions : partitions);
     const cudaError_t err =
-        dtype == PA_BF16 ? launch_shared_dim<__nv_bfloat16>(a, head_dim, grid, chunks, members, num_members, num_seqs, s)
-                         : launch_shared_dim<__half>(a, head_dim, grid, chunks, members, num_members, num_seqs, s);
+        dtype == PA_BF16
+            ? launch_shared_dim<__nv_bfloat16>(a, head_dim, grid, chunks, members, num_members, num_seqs, dtype, s)
+            : launch_shared_dim<__half>(a, head_dim, grid, chunks, members, num_members, num_seqs, dtype, s);
     if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode shared-prefix kernel: %s", cudaGetErrorString(err));
     a.first_partition = first_partition;
     // Partitions below every sequence's first_partition need no per-sequence CTA.
