@@ -1040,17 +1040,19 @@ __global__ void __launch_bounds__(128, 1) decode_shared_tc05_kernel(const Decode
 // ---------------------------------------------------------------------------
 // Warp-specialised, persistent shared-prefix kernel on tcgen05 (the default
 // joint kernel).  One CTA per SM walks work items (chunk, kv head, shared
-// partition) with stride gridDim.x; an item is 8 steps of 64 tokens.  Roles:
+// partition) with stride gridDim.x; an item is 8 steps of 64 tokens.  Roles
+// (9 warps):
 //   warps 0-3  softmax: thread r owns query row r; per step it reads its S row
 //              from TMEM, keeps the running max / sum (lazy rescaling of O),
 //              writes P (16-bit) to TMEM; at the end of an item it writes the
 //              partials.
-//   warp 4     producer: K/V pages by TMA (16 lanes issue the step's 16 boxes
-//              at once) into a ring of STAGES buffers, as far ahead as the
-//              ring allows; three steps before an item ends it starts the
-//              next item's queries (cp.async) and table slice into the other
-//              query buffer, so the ring keeps filling across item boundaries.
-//   warp 5     MMA issuer (one lane): S(g) = Q.K^T into S[g & 1], then
+//   warps 4-7  producers: K/V pages by TMA into a ring of STAGES buffers, as
+//              far ahead as the ring allows, each warp a quarter of a step's
+//              16-row boxes (one warp alone cannot issue boxes fast enough to
+//              keep up with HBM); three steps before an item ends they start
+//              the next item's queries (cp.async, one row per lane) into the
+//              other query buffer, so the ring keeps filling across items.
+//   warp 8     MMA issuer (one lane): S(g) = Q.K^T into S[g & 1], then
 //              O += P(g-1).V(g-1), so the tensor cores work on step g while
 //              the softmax warps finish step g-1; an item's last O += P.V is
 //              issued before the next item starts.
@@ -1063,7 +1065,9 @@ __global__ void __launch_bounds__(128, 1) decode_shared_tc05_kernel(const Decode
 // ---------------------------------------------------------------------------
 template <int D, int STAGES>
 struct Tc05pShape {
-  static constexpr int kThreads = 192;
+  static constexpr int kProducerWarps = 4;  // TMA issue from one warp tops out near 41 GB/s per SM
+  static constexpr int kMmaWarp = 4 + kProducerWarps;
+  static constexpr int kThreads = 32 * (kMmaWarp + 1);
   static constexpr int kRows = 128;
   static constexpr int kStep = 64;
   static constexpr int kStepsPerItem = kPartition / kStep;  // 8
@@ -1077,15 +1081,20 @@ struct Tc05pShape {
   static constexpr int kBoxesPerStep = 2 * (kStep / 16) * kBlocks;
   static constexpr int kQOff = 0;
   static constexpr int kStageOff = 2 * kQBytes;
-  static constexpr int kSliceOff = kStageOff + STAGES * kStageBytes;  // int32 [2][32]
-  static constexpr int kBarOff = kSliceOff + 256;
+  static constexpr int kSliceOff = kStageOff + STAGES * kStageBytes;  // int32 [2][32] table slices
+  static constexpr int kDescOff = kSliceOff + 256;                     // int32 [2][4] item descriptors
+  static constexpr int kRowOff = kDescOff + 64;                        // int32 [2][kRows] workspace rows
+  static constexpr int kBarOff = kRowOff + 2 * kRows * 4;
   static constexpr int kNumBars = 2 * 5 + 2 * STAGES;         // s_full, s_free, p_full, o_done, q_full/item_free x2; kv x STAGES
   static constexpr int kTaddrOff = kBarOff + 8 * (kNumBars + 2);
   static constexpr int kSmemBytes = kTaddrOff + 16 + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kSCol = 0, kPCol = 128, kOCol = 256;  // S[b] at 64b, P[b] at 128 + 32b, O[b] at 256 + 128b
   static_assert(D <= 128, "O double buffer needs D <= 128");
-  static_assert(kBoxesPerStep <= 32, "one lane per box");
+  static constexpr int kBoxesPerWarp = kBoxesPerStep / kProducerWarps;
+  static_assert(kBoxesPerStep % kProducerWarps == 0 && kBoxesPerWarp <= 32, "one lane per box");
+  static_assert(kRows == 32 * kProducerWarps, "one query row per producer lane");
+  static_assert(kQBytes >= 4 * 32 * 20 * 4, "the epilogue's four 32-row float tiles fit in a query buffer");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -1093,6 +1102,15 @@ struct SharedItem {
   int c, kvh, p, leader, moff, mcount;
   bool valid;
 };
+
+// Whether a plan entry names a work item whose arrays are all in range.
+__device__ __forceinline__ bool shared_item_ok(const SharedItem& it, const DecodeArgs& a, int num_members,
+                                               int num_seqs) {
+  return (unsigned)it.leader < (unsigned)num_seqs && it.moff >= 0 && it.mcount >= 0 &&
+         (int64_t)it.moff + it.mcount <= num_members && (int64_t)it.mcount * a.group <= 128 &&
+         (int64_t)(it.p + 1) * kPartition <= (int64_t)a.max_blocks_per_seq * a.block_size &&
+         it.p < a.max_partitions;
+}
 
 // The next usable work item at or after `cursor` (stride gridDim.x), in the
 // order (partition, kv head, chunk) so concurrent CTAs share pages through L2.
@@ -1107,20 +1125,14 @@ __device__ __forceinline__ SharedItem next_shared_item(int64_t& cursor, int64_t 
     cursor += gridDim.x;
     const int c = (int)(w % num_chunks);
     const int64_t rest = w / num_chunks;
-    const int kvh = (int)(rest % a.num_kv_heads);
-    const int p = (int)(rest / a.num_kv_heads);
-    if (p >= __ldg(chunks + 4 * c + 3)) continue;
     it.c = c;
-    it.kvh = kvh;
-    it.p = p;
+    it.kvh = (int)(rest % a.num_kv_heads);
+    it.p = (int)(rest / a.num_kv_heads);
+    if (it.p >= __ldg(chunks + 4 * c + 3)) continue;
     it.leader = __ldg(chunks + 4 * c);
     it.moff = __ldg(chunks + 4 * c + 1);
     it.mcount = __ldg(chunks + 4 * c + 2);
-    const bool ok = (unsigned)it.leader < (unsigned)num_seqs && it.moff >= 0 && it.mcount >= 0 &&
-                    (int64_t)it.moff + it.mcount <= num_members && (int64_t)it.mcount * a.group <= 128 &&
-                    (int64_t)(p + 1) * kPartition <= (int64_t)a.max_blocks_per_seq * a.block_size &&
-                    p < a.max_partitions;
-    if (!ok) {
+    if (!shared_item_ok(it, a, num_members, num_seqs)) {
       if (report) flag_status(a.status, PA_DEV_BAD_PLAN);
       continue;
     }
@@ -1130,8 +1142,56 @@ __device__ __forceinline__ SharedItem next_shared_item(int64_t& cursor, int64_t 
   return it;
 }
 
+// The same walk split in two, so that the plan loads of the next item overlap
+// the current one: `prefetch_shared_item` takes the next work index and starts
+// loading its chunk's entries; `resolve_shared_item` uses them once they are
+// needed, continuing the walk where the index is not a usable item.
+struct SharedItemPrefetch {
+  int64_t w;  // work index, -1 past the end
+  int sp, leader, moff, mcount;
+};
+
+__device__ __forceinline__ SharedItemPrefetch prefetch_shared_item(int64_t& cursor, int64_t total, int num_chunks,
+                                                                   const int32_t* __restrict__ chunks) {
+  SharedItemPrefetch f{-1, 0, 0, 0, 0};
+  if (cursor < total) {
+    f.w = cursor;
+    cursor += gridDim.x;
+    const int c = (int)(f.w % num_chunks);
+    f.sp = __ldg(chunks + 4 * c + 3);
+    f.leader = __ldg(chunks + 4 * c);
+    f.moff = __ldg(chunks + 4 * c + 1);
+    f.mcount = __ldg(chunks + 4 * c + 2);
+  }
+  return f;
+}
+
+__device__ __forceinline__ SharedItem resolve_shared_item(const SharedItemPrefetch& f, int64_t& cursor, int64_t total,
+                                                          int num_chunks, const DecodeArgs& a,
+                                                          const int32_t* __restrict__ chunks, int num_members,
+                                                          int num_seqs, bool report) {
+  SharedItem it{};
+  it.valid = false;
+  if (f.w < 0) return it;
+  const int64_t rest = f.w / num_chunks;
+  it.c = (int)(f.w % num_chunks);
+  it.kvh = (int)(rest % a.num_kv_heads);
+  it.p = (int)(rest / a.num_kv_heads);
+  if (it.p < f.sp) {
+    it.leader = f.leader;
+    it.moff = f.moff;
+    it.mcount = f.mcount;
+    if (shared_item_ok(it, a, num_members, num_seqs)) {
+      it.valid = true;
+      return it;
+    }
+    if (report) flag_status(a.status, PA_DEV_BAD_PLAN);
+  }
+  return next_shared_item(cursor, total, num_chunks, a, chunks, num_members, num_seqs, report);
+}
+
 template <typename T, int D, int STAGES>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(Tc05pShape<D, STAGES>::kThreads, 1)
     decode_shared_tc05p_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
                                const __grid_constant__ CUtensorMap tmap_v, const int32_t* __restrict__ chunks,
                                int num_chunks, const int32_t* __restrict__ members, int num_members, int num_seqs,
@@ -1152,6 +1212,11 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* base_ptr = smem_raw + (base - raw);
   int32_t* tslice = reinterpret_cast<int32_t*>(base_ptr + S::kSliceOff);  // [2][32]
+  // Written by the producers, published with q_full: the item in buffer b
+  // (valid, partition, kv head, member count; valid 0 ends the walk) and the
+  // workspace row of each of its query rows (-1: none).
+  volatile int32_t* desc = reinterpret_cast<volatile int32_t*>(base_ptr + S::kDescOff);  // [2][4]
+  int32_t* prow_s = reinterpret_cast<int32_t*>(base_ptr + S::kRowOff);                   // [2][kRows]
   const uint32_t bar0 = base + S::kBarOff;
   auto s_full = [&](int b) { return bar0 + 8u * b; };
   auto s_free = [&](int b) { return bar0 + 16u + 8u * b; };
@@ -1164,10 +1229,13 @@ __global__ void __launch_bounds__(192, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + S::kTaddrOff + 8);
   const uint32_t taddr_slot = base + S::kTaddrOff;
 
-  // Bounded wait that also gives up once another role has aborted.
+  // Bounded wait that also gives up once another role has aborted.  A waiting
+  // thread sleeps until the phase completes (woken by the completion, or
+  // after 20 us to look at the abort flag), so waiting warps leave the issue
+  // slots to the softmax warps they share a scheduler with.
   auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
     const long long t0 = clock64();
-    while (!tc05::mbar_try_wait(bar, parity)) {
+    while (!tc05::mbar_try_wait_sleep(bar, parity, 20000u)) {
       if (*abort_flag) return false;
       if (clock64() - t0 > kWaitCycles) {
         *abort_flag = 1;
@@ -1189,11 +1257,11 @@ __global__ void __launch_bounds__(192, 1)
       tc05::mbar_init(s_free(b), 4);     // one arrival per softmax warp
       tc05::mbar_init(p_full(b), 4);
       tc05::mbar_init(o_done(b), 1);
-      tc05::mbar_init(q_full(b), 1);     // the producer warp's lane 0
+      tc05::mbar_init(q_full(b), S::kProducerWarps);  // lane 0 of each producer warp
       tc05::mbar_init(item_free(b), 4);
     }
     for (int st = 0; st < STAGES; ++st) {
-      tc05::mbar_init(kv_full(st), 1);
+      tc05::mbar_init(kv_full(st), S::kProducerWarps);
       tc05::mbar_init(kv_empty(st), 1);
     }
     *abort_flag = 0;
@@ -1212,33 +1280,46 @@ __global__ void __launch_bounds__(192, 1)
 
   int64_t cursor = blockIdx.x;
   int64_t prod_g = 0;  // producer: steps whose loads have been issued
-  if (warp == 4) {
-    // ---------------------------------------------------------------- producer
+  if (warp >= 4 && warp < S::kMmaWarp) {
+    // ---------------------------------------------------------------- producers
+    const int pw = warp - 4;
     const T* qbase = reinterpret_cast<const T*>(a.q);
-    // Queries (rows past mcount * G are zero) and table slice of `it` into buffer qb.
-    // Each lane owns rows lane + 32k: one member lookup per row, then its chunks.
-    auto load_q = [&](const SharedItem& it, int qb) {
-      const uint32_t qs = base + S::kQOff + qb * S::kQBytes;
-#pragma unroll
-      for (int k = 0; k < S::kRows / 32; ++k) {
-        const int r = lane + 32 * k;
-        int64_t row = -1;
-        if (r < it.mcount * G) {
-          const int mi = r / G;
-          const int b = __ldg(members + it.moff + mi);
-          if ((unsigned)b < (unsigned)num_seqs) row = (int64_t)b * a.num_q_heads + it.kvh * G + (r - mi * G);
-        }
-        const T* src = qbase + (row < 0 ? 0 : row) * D;
-#pragma unroll
-        for (int ck = 0; ck < D / 8; ++ck)
-          cp_async_16(qs + (ck >> 3) * S::kQBlockBytes + r * 128 + (((ck & 7) ^ (r & 7)) << 4), src + ck * 8,
-                      row < 0 ? 0u : 16u);
-      }
+    // Table entries of `it` (lane l holds page l of the partition; -1 past its end).
+    auto load_pages = [&](const SharedItem& it) -> int {
       const int fb = it.p * kPartition / bs;
       const int nblk = (it.p * kPartition + kPartition - 1) / bs - fb + 1;
-      tslice[qb * 32 + lane] =
-          lane < nblk ? __ldg(a.block_tables + (int64_t)it.leader * a.max_blocks_per_seq + fb + lane) : -1;
+      return lane < nblk ? __ldg(a.block_tables + (int64_t)it.leader * a.max_blocks_per_seq + fb + lane) : -1;
+    };
+    // Query row pw * 32 + lane of `it` (zero past mcount * G) into buffer qb; the
+    // first producer warp also stores the table slice for the softmax warps.
+    auto load_q = [&](const SharedItem& it, int qb, int pages) {
+      const uint32_t qs = base + S::kQOff + qb * S::kQBytes;
+      const int r = pw * 32 + lane;
+      int64_t row = -1;
+      if (r < it.mcount * G) {
+        const int mi = r / G;
+        const int b = __ldg(members + it.moff + mi);
+        if ((unsigned)b < (unsigned)num_seqs) row = (int64_t)b * a.num_q_heads + it.kvh * G + (r - mi * G);
+      }
+      const T* src = qbase + (row < 0 ? 0 : row) * D;
+#pragma unroll
+      for (int ck = 0; ck < D / 8; ++ck)
+        cp_async_16(qs + (ck >> 3) * S::kQBlockBytes + r * 128 + (((ck & 7) ^ (r & 7)) << 4), src + ck * 8,
+                    row < 0 ? 0u : 16u);
+      prow_s[qb * S::kRows + r] = row < 0 ? -1 : (int32_t)(row * a.max_partitions + it.p);
+      if (pw == 0) {
+        tslice[qb * 32 + lane] = pages;
+        if (lane == 0) {
+          desc[qb * 4 + 1] = it.p;
+          desc[qb * 4 + 2] = it.kvh;
+          desc[qb * 4 + 3] = it.mcount;
+          desc[qb * 4 + 0] = 1;
+        }
+      }
       cp_async_commit();
+    };
+    auto end_walk = [&](int qb) {  // buffer qb holds no item: the other roles stop there
+      if (pw == 0 && lane == 0) desc[qb * 4 + 0] = 0;
     };
     auto publish_q = [&](int qb) {  // after load_q: make it visible, then signal
       cp_async_wait<0>();
@@ -1246,31 +1327,38 @@ __global__ void __launch_bounds__(192, 1)
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(q_full(qb)) : "memory");
     };
-    SharedItem it = next_shared_item(cursor, total_items, num_chunks, a, chunks, num_members, num_seqs, lane == 0);
+    SharedItem it = next_shared_item(cursor, total_items, num_chunks, a, chunks, num_members, num_seqs,
+                                     pw == 0 && lane == 0);
+    int my_page = -1;
     if (it.valid) {
-      load_q(it, 0);
-      publish_q(0);
+      my_page = load_pages(it);
+      load_q(it, 0, my_page);
+    } else {
+      end_walk(0);
     }
+    publish_q(0);
     int64_t g = 0;
     for (int j = 0; it.valid; ++j) {
       const int qb = j & 1;
-      const SharedItem nxt =
-          next_shared_item(cursor, total_items, num_chunks, a, chunks, num_members, num_seqs, lane == 0);
+      const SharedItemPrefetch pf = prefetch_shared_item(cursor, total_items, num_chunks, chunks);
+      SharedItem nxt{};
+      nxt.valid = false;
       const int fb = it.p * kPartition / bs;
-      const int my_page = tslice[qb * 32 + lane];
+      int nxt_page = -1;
       bool stop = false;
       for (int i = 0; i < SPI; ++i, ++g) {
         const int st = (int)(g % STAGES);
         if (g >= STAGES && !wwait(kv_empty(st), (uint32_t)(((g - STAGES) / STAGES) & 1))) { stop = true; break; }
-        if (lane == 0) tc05::mbar_arrive_expect_tx(kv_full(st), S::kStageBytes);
-        // lane -> (row box rb, 64-wide block blk, K or V); lanes past the boxes idle
-        const int kv = lane & 1;
-        const int blk = (lane >> 1) % S::kBlocks;
-        const int rb = ((lane >> 1) / S::kBlocks) % (S::kStep / 16);
+        if (lane == 0) tc05::mbar_arrive_expect_tx(kv_full(st), S::kBoxesPerWarp * S::kBoxBytes);
+        // box -> (row box rb, 64-wide block blk, K or V)
+        const int box = pw * S::kBoxesPerWarp + lane;
+        const int kv = box & 1;
+        const int blk = (box >> 1) % S::kBlocks;
+        const int rb = ((box >> 1) / S::kBlocks) % (S::kStep / 16);
         const int tok = it.p * kPartition + i * S::kStep + 16 * rb;
         const int page = __shfl_sync(kFull, my_page, tok / bs - fb);
         __syncwarp();
-        if (lane < S::kBoxesPerStep) {
+        if (lane < S::kBoxesPerWarp) {
           const int64_t y = (unsigned)page < (unsigned)a.num_blocks
                                 ? ((int64_t)page * a.num_kv_heads + it.kvh) * bs + tok % bs
                                 : total_rows;  // out of range: the box is filled with zeros
@@ -1279,20 +1367,28 @@ __global__ void __launch_bounds__(192, 1)
           tc05::tma_load_2d(dst, kv ? (const void*)&tmap_v : (const void*)&tmap_k, kv_full(st), 64 * blk, (int32_t)y);
         }
         __syncwarp();
-        prod_g = g + 1;
-        // Mid-item: the next item's queries go into the other buffer once the
-        // item that last used it (j - 1) has been read out.
-        if (i == SPI - 3 && nxt.valid) {
+        if (pw == 0) prod_g = g + 1;
+        // Three steps before the end: the next item's queries go into the other
+        // buffer once the item that last used it (j - 1) has been read out.
+        if (i == SPI - 3) {
+          nxt = resolve_shared_item(pf, cursor, total_items, num_chunks, a, chunks, num_members, num_seqs,
+                                    pw == 0 && lane == 0);
           if (j >= 1 && !wwait(item_free(qb ^ 1), (uint32_t)(((j - 1) >> 1) & 1))) { stop = true; break; }
-          load_q(nxt, qb ^ 1);
+          if (nxt.valid) {
+            nxt_page = load_pages(nxt);
+            load_q(nxt, qb ^ 1, nxt_page);
+          } else {
+            end_walk(qb ^ 1);
+          }
         }
       }
       if (stop || __any_sync(kFull, *abort_flag != 0)) break;
-      if (nxt.valid) publish_q(qb ^ 1);
+      publish_q(qb ^ 1);
       it = nxt;
+      my_page = nxt_page;
     }
     cp_async_wait<0>();  // nothing may land in shared memory after the CTA leaves
-  } else if (warp == 5) {
+  } else if (warp == S::kMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
@@ -1317,11 +1413,9 @@ __global__ void __launch_bounds__(192, 1)
       int64_t g = 0;
       bool ok = true;
       for (int j = 0; ok; ++j) {
-        const SharedItem it = next_shared_item(cursor, total_items, num_chunks, a, chunks, num_members, num_seqs,
-                                               false);
-        if (!it.valid) break;
         const int qb = j & 1;
         if (!wait(q_full(qb), (uint32_t)((j >> 1) & 1))) break;
+        if (desc[qb * 4 + 0] == 0) break;  // the walk has ended
         tc05::fence_after();
         tc05::fence_proxy_async_smem();
         const uint32_t qs = base + S::kQOff + qb * S::kQBytes;
@@ -1351,12 +1445,13 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t row_t = tmem + ((uint32_t)(32 * warp) << 16);
     int64_t g = 0;
     for (int j = 0;; ++j) {
-      const SharedItem it = next_shared_item(cursor, total_items, num_chunks, a, chunks, num_members, num_seqs,
-                                             false);
-      if (!it.valid) break;
       const int qb = j & 1;
+      if (!wwait(q_full(qb), (uint32_t)((j >> 1) & 1))) break;  // item, table slice and rows
+      if (desc[qb * 4 + 0] == 0) break;                          // the walk has ended
+      SharedItem it{};
+      it.p = desc[qb * 4 + 1];
+      it.mcount = desc[qb * 4 + 3];
       const bool busy = 32 * warp < it.mcount * G;
-      if (!wwait(q_full(qb), (uint32_t)((j >> 1) & 1))) break;  // table slice of the item
       float m_use = -INFINITY, l = 0.f;
       bool ok = true;
       for (int i = 0; i < SPI; ++i, ++g) {
@@ -1376,49 +1471,75 @@ __global__ void __launch_bounds__(192, 1)
         if (busy) {
           const int tok0 = it.p * kPartition + i * S::kStep;
           const int fb = it.p * kPartition / bs;
+          int bad = 0;  // 16-token groups of the step whose page is out of range
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            bad |= (unsigned)tslice[qb * 32 + (tok0 + 16 * q4) / bs - fb] < (unsigned)a.num_blocks ? 0 : 1 << q4;
           float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          float nref;  // minus the reference score; weights are 2^(s * scale + nref)
+          if (bad == 0 && a.qk_scale_log2 > 0.f) {
+            // Every score is finite: max over the raw scores, one FMA per weight.
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int page = tslice[qb * 32 + (tok0 + 16 * q4) / bs - fb];
-            const bool okp = (unsigned)page < (unsigned)a.num_blocks;
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj) {
-              const int e = 16 * q4 + jj;
-              const float v = okp ? __uint_as_float(sreg[e >> 5][e & 31]) * a.qk_scale_log2 : -INFINITY;
-              sreg[e >> 5][e & 31] = __float_as_uint(v);
-              mx4[jj & 3] = fmaxf(mx4[jj & 3], v);
+            for (int e = 0; e < 64; ++e) mx4[e & 3] = fmaxf(mx4[e & 3], __uint_as_float(sreg[e >> 5][e & 31]));
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * a.qk_scale_log2;
+            if (mx > m_use + 8.f) {
+              alpha = m_use == -INFINITY ? 0.f : ex2_approx(m_use - mx);
+              m_use = mx;
             }
-          }
-          const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-          if (mx > m_use + 8.f) {
-            alpha = m_use == -INFINITY ? 0.f : exp2f(m_use - mx);
-            m_use = mx;
-          }
-          const float ref = m_use == -INFINITY ? 0.f : m_use;
-          float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            nref = -m_use;
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj) {
-            const int e0 = 2 * jj, e1 = 2 * jj + 1;
-            const float p0 = exp2f(__uint_as_float(sreg[e0 >> 5][e0 & 31]) - ref);
-            const float p1 = exp2f(__uint_as_float(sreg[e1 >> 5][e1 & 31]) - ref);
-            ls[jj & 3] += p0 + p1;
-            pk[jj] = pack2<T>(p0, p1);
+            for (int jj = 0; jj < 32; ++jj) {
+              const int e0 = 2 * jj, e1 = 2 * jj + 1;
+              const float p0 = ex2_approx(fmaf(__uint_as_float(sreg[e0 >> 5][e0 & 31]), a.qk_scale_log2, nref));
+              const float p1 = ex2_approx(fmaf(__uint_as_float(sreg[e1 >> 5][e1 & 31]), a.qk_scale_log2, nref));
+              ls[jj & 3] += p0 + p1;
+              pk[jj] = pack2<T>(p0, p1);
+            }
+            l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+          } else {
+            // Scores of tokens on an out-of-range page are -inf (weight 0).
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll
+              for (int jj = 0; jj < 16; ++jj) {
+                const int e = 16 * q4 + jj;
+                const float v = (bad >> q4) & 1 ? -INFINITY : __uint_as_float(sreg[e >> 5][e & 31]) * a.qk_scale_log2;
+                sreg[e >> 5][e & 31] = __float_as_uint(v);
+                mx4[jj & 3] = fmaxf(mx4[jj & 3], v);
+              }
+            }
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            if (mx > m_use + 8.f) {
+              alpha = m_use == -INFINITY ? 0.f : ex2_approx(m_use - mx);
+              m_use = mx;
+            }
+            nref = m_use == -INFINITY ? 0.f : -m_use;
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+              const int e0 = 2 * jj, e1 = 2 * jj + 1;
+              const float p0 = ex2_approx(__uint_as_float(sreg[e0 >> 5][e0 & 31]) + nref);
+              const float p1 = ex2_approx(__uint_as_float(sreg[e1 >> 5][e1 & 31]) + nref);
+              ls[jj & 3] += p0 + p1;
+              pk[jj] = pack2<T>(p0, p1);
+            }
+            l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
           }
-          l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
         }
         if (busy && i > 0 && __any_sync(kFull, alpha != 1.f)) {
           // O is current once O += P.V of step g - 1 has completed.
           if (!wwait(o_done((int)((g - 1) & 1)), (uint32_t)(((g - 1) >> 1) & 1))) { ok = false; break; }
           tc05::fence_after();
           const uint32_t ocol = S::kOCol + 128u * (uint32_t)qb;
-#pragma unroll
-          for (int cb = 0; cb < D / 32; ++cb) {
-            uint32_t ov[32];
-            tc05::ld32(row_t + ocol + 32 * cb, ov);
+#pragma unroll 1
+          for (int cb = 0; cb < D / 16; ++cb) {
+            uint32_t ov[16];
+            tc05::ld16(row_t + ocol + 16 * cb, ov);
             tc05::wait_ld();
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) ov[jj] = __float_as_uint(__uint_as_float(ov[jj]) * alpha);
-            tc05::st32(row_t + ocol + 32 * cb, ov);
+            for (int jj = 0; jj < 16; ++jj) ov[jj] = __float_as_uint(__uint_as_float(ov[jj]) * alpha);
+            tc05::st16(row_t + ocol + 16 * cb, ov);
           }
         }
         // P buffer g & 1 was last read by O += P.V of step g - 2.
@@ -1438,31 +1559,43 @@ __global__ void __launch_bounds__(192, 1)
       if (!wwait(o_done((int)(gl & 1)), (uint32_t)((gl >> 1) & 1))) break;
       tc05::fence_after();
       if (busy) {
-        int64_t qrow = -1;
-        if (tid < it.mcount * G) {
-          const int mi = tid / G;
-          const int b = __ldg(members + it.moff + mi);
-          if ((unsigned)b < (unsigned)num_seqs) qrow = (int64_t)b * a.num_q_heads + it.kvh * G + (tid - mi * G);
-        }
-        const int64_t part = qrow * a.max_partitions + it.p;
+        const int32_t prow = prow_s[qb * S::kRows + tid];  // workspace row of this thread's partial
         const float inv = l > 0.f ? 1.f / l : 0.f;
         const uint32_t ocol = S::kOCol + 128u * (uint32_t)qb;
-#pragma unroll
-        for (int cb = 0; cb < D / 32; ++cb) {
-          uint32_t ov[32];
-          tc05::ld32(row_t + ocol + 32 * cb, ov);
+        // O leaves through a 32-row tile per warp (rows 80 bytes apart: 16-byte
+        // accesses are conflict-free both ways) in this item's query buffer,
+        // idle once the item's MMAs are done and not refilled before item_free,
+        // 16 columns at a time.  Store instructions cost the most here, so each
+        // one writes 16 bytes per lane: 64 contiguous bytes of each of 8 rows.
+        constexpr int kTileStride = 20;  // floats
+        float* tile = reinterpret_cast<float*>(base_ptr + S::kQOff + qb * S::kQBytes) + warp * 32 * kTileStride;
+        float4* wr = reinterpret_cast<float4*>(tile + lane * kTileStride);  // this thread's row
+        const int rsub = lane >> 2, csub = lane & 3;                        // row 8i + rsub, 4 columns
+#pragma unroll 1
+        for (int cb = 0; cb < D / 16; ++cb) {
+          uint32_t ov[16];
+          tc05::ld16(row_t + ocol + 16 * cb, ov);
           tc05::wait_ld();
-          if (qrow >= 0) {
-            float4* dst = reinterpret_cast<float4*>(a.o_part + part * D + 32 * cb);
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
-              dst[jj] = make_float4(__uint_as_float(ov[4 * jj]) * inv, __uint_as_float(ov[4 * jj + 1]) * inv,
-                                    __uint_as_float(ov[4 * jj + 2]) * inv, __uint_as_float(ov[4 * jj + 3]) * inv);
+          for (int q4 = 0; q4 < 4; ++q4)
+            wr[q4] = make_float4(__uint_as_float(ov[4 * q4]) * inv, __uint_as_float(ov[4 * q4 + 1]) * inv,
+                                 __uint_as_float(ov[4 * q4 + 2]) * inv, __uint_as_float(ov[4 * q4 + 3]) * inv);
+          __syncwarp();
+          float4 v[4];
+          int32_t pr[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            pr[i] = __shfl_sync(kFull, prow, 8 * i + rsub);
+            v[i] = *reinterpret_cast<const float4*>(tile + (8 * i + rsub) * kTileStride + 4 * csub);
           }
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (pr[i] >= 0) *reinterpret_cast<float4*>(a.o_part + (int64_t)pr[i] * D + 16 * cb + 4 * csub) = v[i];
         }
-        if (qrow >= 0) {
-          a.m_part[part] = m_use == -INFINITY ? -INFINITY : m_use * kLn2;
-          a.l_part[part] = l;
+        if (prow >= 0) {
+          a.m_part[prow] = m_use == -INFINITY ? -INFINITY : m_use * kLn2;
+          a.l_part[prow] = l;
         }
       }
       tc05::fence_before();
@@ -1477,7 +1610,7 @@ __global__ void __launch_bounds__(192, 1)
     if (tid == 0) flag_status(a.status, PA_DEV_TIMEOUT);
     // Let the TMA loads still in the ring land before the shared memory is released
     // (the last STAGES issued steps; each stage's latest phase is at most one behind).
-    if (warp == 4 && lane == 0)
+    if (warp == 4 && lane == 0)  // (a phase another producer warp left short runs into the bound)
       for (int64_t gl = prod_g > STAGES ? prod_g - STAGES : 0; gl < prod_g; ++gl) {
         const long long t0 = clock64();
         while (!tc05::mbar_try_wait(kv_full((int)(gl % STAGES)), (uint32_t)((gl / STAGES) & 1)) &&
@@ -1507,7 +1640,7 @@ __global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeArgs a, 
   constexpr int VPL = D / 32;
   constexpr int NW = 4;
   constexpr int IPC = NW / WPI;  // items per CTA
-  constexpr int UNROLL = 4;
+  constexpr int UNROLL = VPL <= 4 ? 8 : 4;
   __shared__ float acc_w[NW][D];
   __shared__ float m_w[NW], l_w[NW];
   const int warp = threadIdx.x >> 5;
@@ -1524,9 +1657,45 @@ __global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeArgs a, 
   }
   const bool merge = live && np > 1;
 
-  float mx = -INFINITY;
+  // This warp's partitions are p = sub + WPI * (lane + 32 c), c = 0, 1, ...
+  // Lane `lane` holds m and l of its first one; the first UNROLL partial rows
+  // are requested before the max is known, and each group of rows is
+  // accumulated while the next group is in flight.
+  auto load_rows = [&](float (&x)[UNROLL][VPL], int p0, int k, int cnt) {
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      if (k + u < cnt) {
+        const float* src = a.o_part + (base + p0 + WPI * (k + u)) * D + lane * VPL;
+        if constexpr (VPL % 4 == 0) {
+#pragma unroll
+          for (int v = 0; v < VPL / 4; ++v) {
+            const float4 f = reinterpret_cast<const float4*>(src)[v];
+            x[u][4 * v] = f.x;
+            x[u][4 * v + 1] = f.y;
+            x[u][4 * v + 2] = f.z;
+            x[u][4 * v + 3] = f.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < VPL; ++i) x[u][i] = src[i];
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) x[u][i] = 0.f;
+      }
+    }
+  };
+  const int pf = sub + WPI * lane;
+  float m_first = -INFINITY, l_first = 0.f;
+  if (merge && pf < np) {
+    m_first = a.m_part[base + pf];
+    l_first = a.l_part[base + pf];
+  }
+  float x[UNROLL][VPL];
+  load_rows(x, sub, 0, merge ? min(32, (np - sub + WPI - 1) / WPI) : 0);
+  float mx = m_first;
   if (merge)
-    for (int p = sub + WPI * lane; p < np; p += WPI * 32) mx = fmaxf(mx, a.m_part[base + p]);
+    for (int p = pf + WPI * 32; p < np; p += WPI * 32) mx = fmaxf(mx, a.m_part[base + p]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
 
@@ -1535,43 +1704,33 @@ __global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeArgs a, 
   for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
   float lsum = 0.f;
   if (merge && mx != -INFINITY) {
-    for (int p0 = sub; p0 < np; p0 += WPI * 32) {
+    for (int p0 = sub, c = 0; p0 < np; p0 += WPI * 32, ++c) {
       const int p = p0 + WPI * lane;
       float wt = 0.f;
-      if (p < np) wt = a.l_part[base + p] * expf(a.m_part[base + p] - mx);
+      if (p < np) {
+        const float mp = c == 0 ? m_first : a.m_part[base + p];
+        const float lp = c == 0 ? l_first : a.l_part[base + p];
+        wt = lp * expf(mp - mx);
+      }
       lsum += wt;
       const int cnt = min(32, (np - p0 + WPI - 1) / WPI);
+      if (c > 0) load_rows(x, p0, 0, cnt);
       for (int k = 0; k < cnt; k += UNROLL) {
-        float x[UNROLL][VPL];
-        float wk[UNROLL];
+        float xn[UNROLL][VPL];
+        const bool more = k + UNROLL < cnt;
+        if (more) load_rows(xn, p0, k + UNROLL, cnt);
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
-          wk[u] = __shfl_sync(kFull, wt, min(k + u, 31));
-          if (k + u < cnt) {
-            const float* src = a.o_part + (base + p0 + WPI * (k + u)) * D + lane * VPL;
-            if constexpr (VPL % 4 == 0) {
+          const float wk = __shfl_sync(kFull, wt, min(k + u, 31));
 #pragma unroll
-              for (int v = 0; v < VPL / 4; ++v) {
-                const float4 f = reinterpret_cast<const float4*>(src)[v];
-                x[u][4 * v] = f.x;
-                x[u][4 * v + 1] = f.y;
-                x[u][4 * v + 2] = f.z;
-                x[u][4 * v + 3] = f.w;
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < VPL; ++i) x[u][i] = src[i];
-            }
-          } else {
-            wk[u] = 0.f;
-#pragma unroll
-            for (int i = 0; i < VPL; ++i) x[u][i] = 0.f;
-          }
+          for (int i = 0; i < VPL; ++i) acc[i] = fmaf(k + u < cnt ? wk : 0.f, x[u][i], acc[i]);
         }
+        if (more) {
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u)
+          for (int u = 0; u < UNROLL; ++u)
 #pragma unroll
-          for (int i = 0; i < VPL; ++i) acc[i] = fmaf(wk[u], x[u][i], acc[i]);
+            for (int i = 0; i < VPL; ++i) x[u][i] = xn[u][i];
+        }
       }
     }
   }
@@ -1760,7 +1919,9 @@ template <typename T, int D>
 cudaError_t launch_shared_tc05p(const DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, int num_chunks,
                                 const int32_t* chunks, const int32_t* members, int num_members, int num_seqs,
                                 int max_sp, cudaStream_t stream) {
-  constexpr int kStages = 4;
+  // As many ring stages as shared memory holds: a stage stays with the
+  // consumer for about two steps, the rest are loads in flight.
+  constexpr int kStages = D == 128 ? 5 : 8;
   using S = Tc05pShape<D, kStages>;
   static std::atomic<uint64_t> done{0};
   auto kernel = decode_shared_tc05p_kernel<T, D, kStages>;

@@ -88,6 +88,15 @@ __device__ __forceinline__ void load_floats(const T* __restrict__ p, float (&out
   }
 }
 
+// 2^x on the special-function unit (PTX ex2.approx.ftz.f32: subnormal results
+// flush to zero, 2^-inf = 0).  Softmax weights are rounded to 16 bits right
+// after, far coarser than the instruction's error.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---- async copies ---------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
