@@ -127,12 +127,25 @@ __device__ __forceinline__ void store_zero_rows(const DecodeArgs& a, int b, int 
     out[((int64_t)b * a.num_q_heads + h0) * D + i] = from_float<T>(0.f);
 }
 
+// A partition kernel launched as a programmatic dependent of the shared-prefix
+// kernel (so that its CTAs fill the SMs that kernel's last wave leaves idle)
+// must still finish after it, for the merge that follows: one thread waits for
+// the prerequisite grid on the way out.  On an ordinary launch the wait returns
+// at once.
+struct AfterPrerequisiteGrid {
+  bool on;
+  __device__ ~AfterPrerequisiteGrid() {
+    if (on) asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  }
+};
+
 // ---------------------------------------------------------------------------
 // CUDA-core partition kernel.  Grid (num_seqs, num_kv_heads * head_chunks, P);
 // a CTA serves up to GC query heads of one kv head.
 // ---------------------------------------------------------------------------
 template <typename T, int D, int GC, int NW>
 __global__ void __launch_bounds__(NW * 32) decode_cc_kernel(const DecodeArgs a) {
+  const AfterPrerequisiteGrid after{threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0};
   constexpr int VPL = D / 32;
   __shared__ float o_w[NW * GC * D];
   __shared__ float m_w[NW * GC];
@@ -257,6 +270,7 @@ struct TcShape {
 
 template <typename T, int D, int NW, int STAGES>
 __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(const DecodeArgs a) {
+  const AfterPrerequisiteGrid after{threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0};
   using S = TcShape<D, NW, STAGES>;
   constexpr int KSTEPS = D / 16;
   constexpr int MTILES = D / 16;
@@ -1278,6 +1292,9 @@ __global__ void __launch_bounds__(Tc05pShape<D, STAGES>::kThreads, 1)
   tc05::fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base_ptr + S::kTaddrOff);
 
+  // The per-sequence partition kernel that follows may start on SMs this grid
+  // leaves (its CTAs cannot share an SM with this one's).
+  if (tid == 0) asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   int64_t cursor = blockIdx.x;
   int64_t prod_g = 0;  // producer: steps whose loads have been issued
   if (warp >= 4 && warp < S::kMmaWarp) {
@@ -1452,6 +1469,11 @@ __global__ void __launch_bounds__(Tc05pShape<D, STAGES>::kThreads, 1)
       it.p = desc[qb * 4 + 1];
       it.mcount = desc[qb * 4 + 3];
       const bool busy = 32 * warp < it.mcount * G;
+      // Page validity of the item's 32 16-token groups (4 per step), one lane each.
+      static_assert(kPartition / 16 == 32 && S::kStep == 64, "one lane per 16-token group of an item");
+      const uint32_t page_ok = __ballot_sync(
+          kFull, (unsigned)tslice[qb * 32 + (it.p * kPartition + 16 * lane) / bs - it.p * kPartition / bs] <
+                     (unsigned)a.num_blocks);
       float m_use = -INFINITY, l = 0.f;
       bool ok = true;
       for (int i = 0; i < SPI; ++i, ++g) {
@@ -1469,12 +1491,7 @@ __global__ void __launch_bounds__(Tc05pShape<D, STAGES>::kThreads, 1)
         uint32_t pk[32];
         float alpha = 1.f;
         if (busy) {
-          const int tok0 = it.p * kPartition + i * S::kStep;
-          const int fb = it.p * kPartition / bs;
-          int bad = 0;  // 16-token groups of the step whose page is out of range
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            bad |= (unsigned)tslice[qb * 32 + (tok0 + 16 * q4) / bs - fb] < (unsigned)a.num_blocks ? 0 : 1 << q4;
+          const int bad = (int)(~page_ok >> (4 * i)) & 0xF;  // 16-token groups whose page is out of range
           float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
           float nref;  // minus the reference score; weights are 2^(s * scale + nref)
           if (bad == 0 && a.qk_scale_log2 > 0.f) {
@@ -1810,36 +1827,50 @@ cudaError_t ensure_smem(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
 }
 
 template <typename T, int D, int NW, int STAGES>
-cudaError_t launch_tc(const DecodeArgs& a, dim3 grid, cudaStream_t stream) {
+cudaError_t launch_tc(const DecodeArgs& a, dim3 grid, cudaStream_t stream, bool dependent) {
   using S = TcShape<D, NW, STAGES>;
   static std::atomic<uint64_t> done{0};
   auto kernel = decode_tc_kernel<T, D, NW, STAGES>;
   cudaError_t err = ensure_smem(kernel, S::kSmemBytes, done);
   if (err != cudaSuccess) return err;
-  kernel<<<grid, NW * 32, S::kSmemBytes, stream>>>(a);
-  return cudaGetLastError();
+  if (!dependent) {
+    kernel<<<grid, NW * 32, S::kSmemBytes, stream>>>(a);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(NW * 32);
+  cfg.dynamicSmemBytes = S::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
 template <typename T, int D>
-cudaError_t launch_tc_config(const DecodeArgs& a, dim3 grid, cudaStream_t stream, int warps, int stages) {
-  if (warps == 4 && stages == 3) return launch_tc<T, D, 4, 3>(a, grid, stream);
-  if (warps == 4 && stages == 2) return launch_tc<T, D, 4, 2>(a, grid, stream);
-  if (warps == 4 && stages == 4) return launch_tc<T, D, 4, 4>(a, grid, stream);
-  if (warps == 2 && stages == 4) return launch_tc<T, D, 2, 4>(a, grid, stream);
-  if (warps == 8 && stages == 2) return launch_tc<T, D, 8, 2>(a, grid, stream);
+cudaError_t launch_tc_config(const DecodeArgs& a, dim3 grid, cudaStream_t stream, int warps, int stages,
+                             bool dependent) {
+  if (warps == 4 && stages == 3) return launch_tc<T, D, 4, 3>(a, grid, stream, dependent);
+  if (warps == 4 && stages == 2) return launch_tc<T, D, 4, 2>(a, grid, stream, dependent);
+  if (warps == 4 && stages == 4) return launch_tc<T, D, 4, 4>(a, grid, stream, dependent);
+  if (warps == 2 && stages == 4) return launch_tc<T, D, 2, 4>(a, grid, stream, dependent);
+  if (warps == 8 && stages == 2) return launch_tc<T, D, 8, 2>(a, grid, stream, dependent);
   return cudaErrorInvalidValue;
 }
 
 template <typename T>
 cudaError_t launch_tc_dim(const DecodeArgs& a, int head_dim, dim3 grid, cudaStream_t stream, int warps,
-                          int stages) {
+                          int stages, bool dependent = false) {
   switch (head_dim) {
-    case 64: return launch_tc_config<T, 64>(a, grid, stream, warps, stages);
-    case 128: return launch_tc_config<T, 128>(a, grid, stream, warps, stages);
+    case 64: return launch_tc_config<T, 64>(a, grid, stream, warps, stages, dependent);
+    case 128: return launch_tc_config<T, 128>(a, grid, stream, warps, stages, dependent);
     case 256:
       // 256-wide rows: keep to configurations within the shared-memory limit.
       if (warps * stages * 16384 > 200 * 1024) return cudaErrorInvalidValue;
-      return launch_tc_config<T, 256>(a, grid, stream, warps, stages);
+      return launch_tc_config<T, 256>(a, grid, stream, warps, stages, dependent);
   }
   return cudaErrorInvalidValue;
 }
@@ -2103,8 +2134,10 @@ pa_status prepare_decode(const void* q, const void* key_cache, const void* value
   return PA_OK;
 }
 
+// `dependent`: launched as a programmatic dependent of the kernel before it on
+// the stream (tensor-core kernel only; the CUDA-core one launches as usual).
 pa_status launch_partitions(const DecodeArgs& a, pa_dtype dtype, int head_dim, int num_seqs, int partitions,
-                            cudaStream_t s) {
+                            cudaStream_t s, bool dependent = false) {
   const int choice = g_kernel_choice.load();
   const bool tc_ok = tc_supported(dtype, head_dim, a.group, a.block_size);
   if (choice == PA_DECODE_TENSOR_CORES && !tc_ok)
@@ -2113,8 +2146,8 @@ pa_status launch_partitions(const DecodeArgs& a, pa_dtype dtype, int head_dim, i
   if (tc_ok && choice != PA_DECODE_CUDA_CORES) {
     dim3 grid(num_seqs, a.num_kv_heads, partitions - a.partition_base);
     const int warps = g_tc_warps.load(), stages = g_tc_stages.load();
-    err = dtype == PA_BF16 ? launch_tc_dim<__nv_bfloat16>(a, head_dim, grid, s, warps, stages)
-                           : launch_tc_dim<__half>(a, head_dim, grid, s, warps, stages);
+    err = dtype == PA_BF16 ? launch_tc_dim<__nv_bfloat16>(a, head_dim, grid, s, warps, stages, dependent)
+                           : launch_tc_dim<__half>(a, head_dim, grid, s, warps, stages, dependent);
   } else {
     err = dtype == PA_F32    ? launch_cc<float>(a, head_dim, num_seqs, partitions, s)
           : dtype == PA_BF16 ? launch_cc<__nv_bfloat16>(a, head_dim, num_seqs, partitions, s)
@@ -2295,7 +2328,7 @@ extern "C" pa_status pa_decode_shared_prefix(const void* q, const void* key_cach
     // Partitions below every sequence's first_partition need no per-sequence CTA.
     a.partition_base = min_shared_partitions < partitions - 1 ? min_shared_partitions : partitions - 1;
   }
-  st = launch_partitions(a, dtype, head_dim, num_seqs, partitions, s);
+  st = launch_partitions(a, dtype, head_dim, num_seqs, partitions, s, /*dependent=*/joint);
   if (st != PA_OK || partitions <= 1) return st;
   return launch_reduce_any(a, dtype, head_dim, num_seqs, s);
 }
