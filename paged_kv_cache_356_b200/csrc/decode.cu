@@ -1060,13 +1060,13 @@ __global__ void __launch_bounds__(128, 1) decode_shared_tc05_kernel(const Decode
 //              from TMEM, keeps the running max / sum (lazy rescaling of O),
 //              writes P (16-bit) to TMEM; at the end of an item it writes the
 //              partials.
-//   warps 4-7  producers: K/V pages by TMA into a ring of STAGES buffers, as
+//   warps 4-6, 8  producers: K/V pages by TMA into a ring of STAGES buffers, as
 //              far ahead as the ring allows, each warp a quarter of a step's
 //              16-row boxes (one warp alone cannot issue boxes fast enough to
 //              keep up with HBM); three steps before an item ends they start
 //              the next item's queries (cp.async, one row per lane) into the
 //              other query buffer, so the ring keeps filling across items.
-//   warp 8     MMA issuer (one lane): S(g) = Q.K^T into S[g & 1], then
+//   warp 7     MMA issuer (one lane): S(g) = Q.K^T into S[g & 1], then
 //              O += P(g-1).V(g-1), so the tensor cores work on step g while
 //              the softmax warps finish step g-1; an item's last O += P.V is
 //              issued before the next item starts.
@@ -1080,8 +1080,10 @@ __global__ void __launch_bounds__(128, 1) decode_shared_tc05_kernel(const Decode
 template <int D, int STAGES>
 struct Tc05pShape {
   static constexpr int kProducerWarps = 4;  // TMA issue from one warp tops out near 41 GB/s per SM
-  static constexpr int kMmaWarp = 4 + kProducerWarps;
-  static constexpr int kThreads = 32 * (kMmaWarp + 1);
+  // Warp w runs on scheduler w % 4.  The MMA warp takes scheduler 3: softmax
+  // warp 0 (scheduler 0) has rows in every item, warp 3 only in full ones.
+  static constexpr int kMmaWarp = 7;
+  static constexpr int kThreads = 32 * (4 + kProducerWarps + 1);
   static constexpr int kRows = 128;
   static constexpr int kStep = 64;
   static constexpr int kStepsPerItem = kPartition / kStep;  // 8
@@ -1297,9 +1299,9 @@ __global__ void __launch_bounds__(Tc05pShape<D, STAGES>::kThreads, 1)
   if (tid == 0) asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   int64_t cursor = blockIdx.x;
   int64_t prod_g = 0;  // producer: steps whose loads have been issued
-  if (warp >= 4 && warp < S::kMmaWarp) {
+  if (warp >= 4 && warp != S::kMmaWarp) {
     // ---------------------------------------------------------------- producers
-    const int pw = warp - 4;
+    const int pw = warp < S::kMmaWarp ? warp - 4 : warp - 5;
     const T* qbase = reinterpret_cast<const T*>(a.q);
     // Table entries of `it` (lane l holds page l of the partition; -1 past its end).
     auto load_pages = [&](const SharedItem& it) -> int {

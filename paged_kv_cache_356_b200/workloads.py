@@ -221,17 +221,27 @@ def _independent_trace(context_lens) -> Tuple[tuple, ...]:
 def _shared_trace(prefix_len, tails) -> Tuple[tuple, ...]:
     """Sequence 0 holds the prefix; 1..B-1 fork from it; each appends its tail.
 
-    All appends run first (in sequence order), then the pending page copies,
-    then every tail write, then the decode step.
+    The tails but their last token are appended (in sequence order), the
+    pending page copies made and the tokens written; then every sequence
+    appends its new token, the pages that append forked are copied, the new
+    tokens are written (the decode step's own cache write) and the step
+    decodes.  A tail of one token is just the new token.
     """
     ops = [("allocate", 0, prefix_len), ("write", 0, 0, prefix_len)]
     for b in range(1, len(tails)):
         ops.append(("fork", 0, b))
     for b, t in enumerate(tails):
-        ops.append(("append", b, t))
+        if t > 1:
+            ops.append(("append", b, t - 1))
     ops.append(("copy_pending",))
     for b, t in enumerate(tails):
-        ops.append(("write", b, prefix_len, t))
+        if t > 1:
+            ops.append(("write", b, prefix_len, t - 1))
+    for b in range(len(tails)):
+        ops.append(("append", b, 1))
+    ops.append(("copy_pending",))
+    for b, t in enumerate(tails):
+        ops.append(("write", b, prefix_len + t - 1, 1))
     ops.append(("decode",))
     return tuple(ops)
 
