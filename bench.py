@@ -57,6 +57,8 @@ def parse_args(argv=None):
                          "(4,096 pairs of 16-token pages) and print one JSON line each")
     ap.add_argument("--shared-prefix", choices=["auto", "on", "off"], default="auto",
                     help="decode shared leading pages once per group (auto: on for prefix/beam32k)")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time eager launches instead of replaying the step as a CUDA graph")
     ap.add_argument("--joint-kernel", choices=["auto", "tcgen05", "tcgen05_serial", "mma_sync"], default="auto",
                     help="kernel for the shared partitions of a prefix group")
     return ap.parse_args(argv)
@@ -416,7 +418,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
     kd, vd, sd = run.step_write
 
-    def step(evs=None):
+    def step(evs=None, stream=stream):
         if evs is not None:
             evs[0].record(stream)
         pa.pa_reshape_and_cache(kd, vd, sd, run.key_cache, run.value_cache, stream=stream)
@@ -440,32 +442,69 @@ def run_ours(args):
         step()
     torch.cuda.synchronize()
 
+    # Per-kernel breakdown: one eager pass of the same steps with events between the kernels.
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+
+    # The timed region replays the step as a CUDA graph (as a decode loop would), unless disabled.
+    graph, launch_mode = None, "eager"
+    if not args.no_graph:
+        try:
+            side = torch.cuda.Stream()
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                step(stream=side)
+            stream.wait_stream(side)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step(stream=torch.cuda.current_stream())
+            for _ in range(3):
+                graph.replay()
+            torch.cuda.synchronize()
+            launch_mode = "CUDA graph of one step (write + decode), replayed"
+        except Exception as exc:  # capture unsupported here: time eager launches
+            graph = None
+            launch_mode = f"eager (graph capture failed: {type(exc).__name__})"
+            torch.cuda.synchronize()
+
+    def timed_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
+
     sampler = None
     if not args.no_clocks:
         sampler = ClockSampler(gpu_smi_id(torch, local))
         sampler.start()
         time.sleep(0.3)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    t0.record(stream)
     for i in range(args.steps):
-        step(evs[i])
+        timed_step()
+    t1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    total_ms = evs[0][0].elapsed_time(evs[-1][3])
+    total_ms = t0.elapsed_time(t1)
     clocks = None
     if sampler is not None:
         # keep identical steps running until the clock record spans at least ~1.5 s under load
         soak_until = time.perf_counter() + max(0.0, 1.5 - total_ms / 1000)
         while time.perf_counter() < soak_until:
             for _ in range(20):
-                step()
+                timed_step()
             torch.cuda.synchronize()
         clocks = sampler.stop()
         clocks["window"] = "timed region, extended by identical steps to >= 1.5 s of samples"
-
+    if graph is not None:
+        del graph
     write_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     part_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
     reduce_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
@@ -493,7 +532,8 @@ def run_ours(args):
         cfg = describe(w)
         cfg.update({"parallelism": f"dp{world} (independent batches per GPU, no collective)",
                     "l2": "no flush: each step reads the whole KV cache, far larger than the 126 MB L2",
-                    "kernel": args.kernel, "tiling": args.tiling, "global_batch": w.num_seqs * world})
+                    "kernel": args.kernel, "tiling": args.tiling, "global_batch": w.num_seqs * world,
+                    "launch": launch_mode})
         if run.plan is not None:
             cfg["joint_kernel"] = args.joint_kernel
         line = {
