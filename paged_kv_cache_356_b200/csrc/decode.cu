@@ -1647,17 +1647,17 @@ __global__ void __launch_bounds__(Tc05pShape<D, STAGES>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Log-sum-exp merge of the partitions.  A CTA of 4 warps serves 4 / WPI
-// (sequence, query head) items with WPI warps each (WPI grows with the
-// partition count).  Warp w of an item merges partitions w, w + WPI, ... with
-// its own running maximum (the lanes compute 32 weights per round; partials
-// are loaded four at a time), then the item's warps merge through shared
-// memory the same way.
+// Log-sum-exp merge of the partitions.  A CTA of max(4, WPI) warps serves
+// max(4, WPI) / WPI (sequence, query head) items with WPI warps each (WPI
+// grows with the partition count).  Warp w of an item merges partitions w,
+// w + WPI, ... with its own running maximum (the lanes compute 32 weights per
+// round; partial rows are loaded in prefetched groups), then the item's warps
+// merge through shared memory the same way.
 // ---------------------------------------------------------------------------
 template <typename T, int D, int WPI>
-__global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeArgs a, int num_seqs) {
+__global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel(const DecodeArgs a, int num_seqs) {
   constexpr int VPL = D / 32;
-  constexpr int NW = 4;
+  constexpr int NW = WPI > 4 ? WPI : 4;
   constexpr int IPC = NW / WPI;  // items per CTA
   constexpr int UNROLL = VPL <= 4 ? 8 : 4;
   __shared__ float acc_w[NW][D];
@@ -2017,6 +2017,8 @@ template <typename T, int D>
 cudaError_t launch_reduce_dim(const DecodeArgs& a, int num_seqs, cudaStream_t stream) {
   const int64_t items = (int64_t)num_seqs * a.num_q_heads;
   auto grid = [&](int ipc) { return (unsigned)((items + ipc - 1) / ipc); };
+  // Warps per (sequence, query head), by partition count (an 8-warp form,
+  // tried for more than 32 partitions, measured no faster).
   if (a.max_partitions <= 16)
     decode_reduce_kernel<T, D, 1><<<grid(4), 128, 0, stream>>>(a, num_seqs);
   else if (a.max_partitions <= 48)

@@ -148,11 +148,12 @@ def test_cuda_core_shapes(dtype, d, group, bs):
 
 
 @pytest.mark.parametrize("kernel", ["tc", "cc"])
-@pytest.mark.parametrize("ctx", [[9000, 20000, 700], [30000, 1, 513], [70000, 40000, 1, 513]],
-                         ids=["p40", "p59", "p137"])
+@pytest.mark.parametrize("ctx", [[9000, 15000, 700], [9000, 20000, 700], [30000, 1, 513],
+                                 [70000, 40000, 1, 513], [140000, 3, 2000]],
+                         ids=["p30", "p40", "p59", "p137", "p274"])
 def test_long_contexts_merge_many_partitions(kernel, ctx):
-    """Merges of 40, 59 and 137 partitions: the merge kernel's 2- and 4-warp forms,
-    the latter over more than one group of 128 partitions."""
+    """Merges of 30 to 274 partitions: the merge kernel's 2- and 4-warp forms, the
+    latter over more than one group of 128 partitions (32 per warp)."""
     case = _paged_case(31 + len(ctx), ctx, 4, 1, 128, 16, "bf16")
     assert_decode_close(_run_gpu(case, kernel), _oracle(case), "bf16", f"{kernel} ctx{ctx}")
 
