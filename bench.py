@@ -129,11 +129,22 @@ def profiled_traffic(kernel_hash):
 
 
 def kernel_source_hash():
+    """First 16 hex digits of sha256 over the tensor-core partition kernel's source: decode.cu's
+    argument and helper block (struct DecodeArgs up to the next section rule), its TcShape /
+    decode_tc_kernel section, and device.cuh."""
     import hashlib
+    csrc = os.path.join(ROOT, "paged_kv_cache_356_b200", "csrc")
+    with open(os.path.join(csrc, "decode.cu")) as fh:
+        src = fh.read()
+    a = src.index("struct DecodeArgs {")
+    b = src.index("// ----", a)
+    c = src.index("template <int D, int NW, int STAGES>\nstruct TcShape {")
+    d = src.index("// ----", src.index("decode_tc_kernel(const DecodeArgs a)"))
     h = hashlib.sha256()
-    for f in ("decode.cu", "device.cuh"):
-        with open(os.path.join(ROOT, "paged_kv_cache_356_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+    h.update(src[a:b].encode())
+    h.update(src[c:d].encode())
+    with open(os.path.join(csrc, "device.cuh"), "rb") as fh:
+        h.update(fh.read())
     return h.hexdigest()[:16]
 
 

@@ -277,6 +277,20 @@ typedef enum pa_shared_prefix_kernel {
 } pa_shared_prefix_kernel;
 PA_API pa_status pa_set_shared_prefix_kernel(pa_shared_prefix_kernel kernel);
 
+/* Test hook for the device-side failure path (process-wide; default off).
+ * The pages have no counterpart.  Waits inside the tcgen05 shared-prefix
+ * kernel are bounded (about one second); when one runs out the kernel raises
+ * PA_DEV_TIMEOUT in dev_status, lets its loads and MMAs finish, frees its
+ * tensor memory and returns, leaving the context usable.  Mode
+ * PA_FAULT_WITHHOLD_FIRST_ITEM makes that kernel's producer warps hold back
+ * the hand-off of each CTA's first work item, so the other roles' waits run
+ * out: the call completes after about one second with PA_DEV_TIMEOUT set and
+ * the shared partitions' partials unwritten.  PA_ERR_INVALID for an unknown
+ * mode. */
+#define PA_FAULT_NONE 0
+#define PA_FAULT_WITHHOLD_FIRST_ITEM 1
+PA_API pa_status pa_set_fault_injection(int32_t mode);
+
 /* Which partition kernel pa_decode runs (process-wide; default AUTO).
  * AUTO picks the tensor-core kernel whenever it supports the call (bf16/f16,
  * head_dim 64/128/256, G <= 8, block_size a multiple of 16 up to 256) and the

@@ -17,6 +17,7 @@ PA_PREFIX_QUERIES_PER_CTA = 128
 PA_DEV_TIMEOUT = 32
 PA_DECODE_AUTO, PA_DECODE_CUDA_CORES, PA_DECODE_TENSOR_CORES = 0, 1, 2
 PA_SHARED_PREFIX_AUTO, PA_SHARED_PREFIX_TCGEN05, PA_SHARED_PREFIX_MMA_SYNC, PA_SHARED_PREFIX_TCGEN05_SERIAL = 0, 1, 2, 3
+PA_FAULT_NONE, PA_FAULT_WITHHOLD_FIRST_ITEM = 0, 1
 PA_PARTITION_TOKENS = 512
 PA_FIXED_SCRATCH_BYTES = 32 * 1024 * 1024
 
@@ -43,6 +44,7 @@ SIGNATURES = {
                                        _vp, _i32, _vp, _sz, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _vp, _vp]),
     "pa_set_decode_kernel": (_i32, [_i32]),
     "pa_set_shared_prefix_kernel": (_i32, [_i32]),
+    "pa_set_fault_injection": (_i32, [_i32]),
     "pa_set_decode_tiling": (_i32, [_i32, _i32]),
     "pa_block_alloc_create": (_i32, [_i32, _i32, _pi32, _c.POINTER(_vp)]),
     "pa_block_alloc_destroy": (None, [_vp]),

@@ -1101,8 +1101,9 @@ struct Tc05pShape {
   static constexpr int kDescOff = kSliceOff + 256;                     // int32 [2][4] item descriptors
   static constexpr int kRowOff = kDescOff + 64;                        // int32 [2][kRows] workspace rows
   static constexpr int kBarOff = kRowOff + 2 * kRows * 4;
-  static constexpr int kNumBars = 2 * 5 + 2 * STAGES;         // s_full, s_free, p_full, o_done, q_full/item_free x2; kv x STAGES
-  static constexpr int kTaddrOff = kBarOff + 8 * (kNumBars + 2);
+  // s_full, s_free, p_full, o_done, q_full, item_free x2; kv_full, kv_empty x STAGES; mma_drain
+  static constexpr int kNumBars = 2 * 6 + 2 * STAGES + 1;
+  static constexpr int kTaddrOff = kBarOff + 8 * kNumBars;
   static constexpr int kSmemBytes = kTaddrOff + 16 + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kSCol = 0, kPCol = 128, kOCol = 256;  // S[b] at 64b, P[b] at 128 + 32b, O[b] at 256 + 128b
@@ -1211,7 +1212,7 @@ __global__ void __launch_bounds__(Tc05pShape<D, STAGES>::kThreads, 1)
     decode_shared_tc05p_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
                                const __grid_constant__ CUtensorMap tmap_v, const int32_t* __restrict__ chunks,
                                int num_chunks, const int32_t* __restrict__ members, int num_members, int num_seqs,
-                               int max_shared_partitions) {
+                               int max_shared_partitions, int fault) {
   using S = Tc05pShape<D, STAGES>;
   constexpr int SPI = S::kStepsPerItem;
   static_assert(SPI >= 3, "the next item's queries are loaded three steps before the item ends");
@@ -1242,6 +1243,7 @@ __global__ void __launch_bounds__(Tc05pShape<D, STAGES>::kThreads, 1)
   auto item_free = [&](int b) { return bar0 + 80u + 8u * b; };
   auto kv_full = [&](int st) { return bar0 + 96u + 8u * st; };
   auto kv_empty = [&](int st) { return bar0 + 96u + 8u * STAGES + 8u * st; };
+  const uint32_t mma_drain = bar0 + 96u + 16u * STAGES;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + S::kTaddrOff + 8);
   const uint32_t taddr_slot = base + S::kTaddrOff;
 
@@ -1280,6 +1282,7 @@ __global__ void __launch_bounds__(Tc05pShape<D, STAGES>::kThreads, 1)
       tc05::mbar_init(kv_full(st), S::kProducerWarps);
       tc05::mbar_init(kv_empty(st), 1);
     }
+    tc05::mbar_init(mma_drain, 1);
     *abort_flag = 0;
     tc05::fence_mbar_init();
     tc05::prefetch_tensormap(&tmap_k);
@@ -1355,7 +1358,8 @@ __global__ void __launch_bounds__(Tc05pShape<D, STAGES>::kThreads, 1)
     } else {
       end_walk(0);
     }
-    publish_q(0);
+    if (fault != PA_FAULT_WITHHOLD_FIRST_ITEM) publish_q(0);
+    else cp_async_wait<0>();  // test hook: the other roles' waits for this hand-off run out
     int64_t g = 0;
     for (int j = 0; it.valid; ++j) {
       const int qb = j & 1;
@@ -1457,6 +1461,14 @@ __global__ void __launch_bounds__(Tc05pShape<D, STAGES>::kThreads, 1)
         }
         // Close the item (its epilogue must not wait for the next item's queries).
         if (ok && !mma2(g - 1)) ok = false;
+      }
+      // Every MMA this thread issued has completed before the CTA frees TMEM and
+      // shared memory (on an abort some may still be running).
+      tc05::commit(mma_drain);
+      {
+        const long long t0 = clock64();
+        while (!tc05::mbar_try_wait(mma_drain, 0) && clock64() - t0 < kWaitCycles) {
+        }
       }
     }
   } else {
@@ -1796,6 +1808,7 @@ __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel
 // Host side.
 // ---------------------------------------------------------------------------
 std::atomic<int> g_kernel_choice{PA_DECODE_AUTO};
+std::atomic<int> g_fault{PA_FAULT_NONE};
 std::atomic<int> g_tc_warps{4};
 std::atomic<int> g_tc_stages{2};
 
@@ -1963,7 +1976,7 @@ cudaError_t launch_shared_tc05p(const DecodeArgs& a, const CUtensorMap& mk, cons
   const int64_t items = (int64_t)max_sp * a.num_kv_heads * num_chunks;
   const int grid = (int)(items < sm_count() ? items : sm_count());
   kernel<<<grid, S::kThreads, S::kSmemBytes, stream>>>(a, mk, mv, chunks, num_chunks, members, num_members, num_seqs,
-                                                       max_sp);
+                                                       max_sp, g_fault.load());
   return cudaGetLastError();
 }
 
@@ -2053,6 +2066,13 @@ extern "C" pa_status pa_set_decode_kernel(pa_decode_kernel k) {
   if (k != PA_DECODE_AUTO && k != PA_DECODE_CUDA_CORES && k != PA_DECODE_TENSOR_CORES)
     return fail(PA_ERR_INVALID, "pa_set_decode_kernel: unknown kernel %d", (int)k);
   g_kernel_choice.store((int)k);
+  return PA_OK;
+}
+
+extern "C" pa_status pa_set_fault_injection(int32_t mode) {
+  if (mode != PA_FAULT_NONE && mode != PA_FAULT_WITHHOLD_FIRST_ITEM)
+    return fail(PA_ERR_INVALID, "pa_set_fault_injection: unknown mode %d", (int)mode);
+  g_fault.store(mode);
   return PA_OK;
 }
 

@@ -99,3 +99,42 @@ def test_bad_plan_entries_are_skipped_and_flagged(joint):
                                dev_status=status)
     torch.cuda.synchronize()
     assert status.item() & pa.PA_DEV_BAD_PLAN
+
+
+def test_wait_that_runs_out_reports_timeout_and_the_context_stays_usable():
+    """Failure path of the tcgen05 joint kernel: with the first work item's hand-off withheld (test hook),
+    the other roles' bounded waits run out after about a second; the call completes with PA_DEV_TIMEOUT
+    instead of hanging, and the next ordinary call on the same context gives the oracle's result."""
+    import math
+    import time
+    import torch
+    pa.pa_set_shared_prefix_kernel(pa.PA_SHARED_PREFIX_TCGEN05)
+    w = workloads.beam32k(num_beams=3, prompt_len=2100, own=40)
+    run = TraceRunner(w, shared_prefix=True)
+    run.run(decode=False)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    try:
+        pa.pa_set_fault_injection(pa.PA_FAULT_WITHHOLD_FIRST_ITEM)
+        t0 = time.perf_counter()
+        pa.pa_decode_shared_prefix(run.q, run.key_cache, run.value_cache, run.block_tables, run.context_lens,
+                                   1 / math.sqrt(w.head_dim), run.plan, out=run.out, workspace=run.workspace,
+                                   dev_status=status)
+        torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
+    finally:
+        pa.pa_set_fault_injection(pa.PA_FAULT_NONE)
+        pa.pa_set_shared_prefix_kernel(pa.PA_SHARED_PREFIX_AUTO)
+    assert status.item() & pa.PA_DEV_TIMEOUT
+    assert 0.2 < elapsed < 30
+    status.zero_()
+    out = pa.pa_decode_shared_prefix(run.q, run.key_cache, run.value_cache, run.block_tables, run.context_lens,
+                                     1 / math.sqrt(w.head_dim), run.plan, out=run.out, workspace=run.workspace,
+                                     dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert_decode_close(out, scenario.run(w)["out"], w.dtype, "after a timed-out call")
+
+
+def test_fault_injection_rejects_unknown_modes():
+    with pytest.raises(pa.PagedAttentionError):
+        pa.pa_set_fault_injection(7)
