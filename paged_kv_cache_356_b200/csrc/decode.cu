@@ -30,6 +30,13 @@
 // (one partition) or the partition's (o_p / l_p, m_p, l_p).  decode_reduce
 // then merges partitions: M = max m_p, w_p = l_p e^(m_p - M),
 // out = sum w_p o_p / sum w_p.
+//
+// pa_decode_shared_prefix computes the same partials, but a whole partition
+// that a group of sequences shares (the same physical pages: forked beams, a
+// common prompt) is read once for the whole group by a joint kernel serving up
+// to PA_PREFIX_QUERIES_PER_CTA queries -- a dense contraction, run on the
+// fifth-generation tensor cores (decode_shared_tc05p_kernel) -- while the
+// per-sequence kernel covers the remaining partitions and the merge follows.
 #include <math.h>
 
 #include <atomic>
@@ -1066,6 +1073,10 @@ __global__ void __launch_bounds__(128, 1) decode_shared_tc05_kernel(const Decode
 //              keep up with HBM); three steps before an item ends they start
 //              the next item's queries (cp.async, one row per lane) into the
 //              other query buffer, so the ring keeps filling across items.
+//              Only they read the plan: each item's descriptor, table slice
+//              and workspace rows reach the other roles through shared memory
+//              with the queries (q_full); a descriptor marked invalid ends the
+//              walk.
 //   warp 7     MMA issuer (one lane): S(g) = Q.K^T into S[g & 1], then
 //              O += P(g-1).V(g-1), so the tensor cores work on step g while
 //              the softmax warps finish step g-1; an item's last O += P.V is
@@ -1075,7 +1086,8 @@ __global__ void __launch_bounds__(128, 1) decode_shared_tc05_kernel(const Decode
 // frees P, makes O current), kv_full / kv_empty (ring), q_full (queries and
 // table slice), item_free (O and Q of an item read out).  Every wait is
 // bounded; a timeout raises an abort flag that every role polls, then the CTA
-// flags PA_DEV_TIMEOUT, lets its TMA loads land, frees TMEM and returns.
+// flags PA_DEV_TIMEOUT, lets its TMA loads land and its MMAs finish, frees
+// TMEM and returns.
 // ---------------------------------------------------------------------------
 template <int D, int STAGES>
 struct Tc05pShape {
