@@ -40,10 +40,14 @@ def test_shared_flows_match_oracle(make, joint):
     assert_decode_close(out, ref["out"], w.dtype, w.name)
 
 
-@pytest.mark.parametrize("hq,hkv,d,bs", [(8, 8, 128, 16), (16, 8, 128, 32), (64, 8, 64, 16), (32, 2, 128, 16),
-                                         (64, 4, 128, 64), (128, 8, 128, 16), (32, 8, 64, 32)])
-def test_shared_shapes(hq, hkv, d, bs, joint):
-    """G = 1, 2, 8, 16, 16 with head_dim 64 / 128 and several block sizes."""
+@pytest.mark.parametrize("hq,hkv,d,bs,dtype", [(8, 8, 128, 16, "bf16"), (16, 8, 128, 32, "bf16"),
+                                               (64, 8, 64, 16, "bf16"), (32, 2, 128, 16, "bf16"),
+                                               (64, 4, 128, 64, "bf16"), (128, 8, 128, 16, "bf16"),
+                                               (32, 8, 64, 32, "bf16"), (32, 8, 128, 48, "bf16"),
+                                               (64, 8, 128, 16, "f16"), (16, 4, 64, 32, "f16")])
+def test_shared_shapes(hq, hkv, d, bs, dtype, joint):
+    """G = 1, 2, 4, 8, 16 with head_dim 64 / 128, block sizes 16 to 64 (48: pages not aligned to
+    partitions), bf16 and f16."""
     import math
     import torch
     from oracle import attention
@@ -64,10 +68,15 @@ def test_shared_shapes(hq, hkv, d, bs, joint):
     ctx = [prompt + o for o in own]
     mb = max(-(-c // bs) for c in ctx)
     tables, lens = a.block_tables(list(range(nseq)), mb, pad=-1)
-    kc = workloads.normal_values(rng, nb * hkv * bs * d, "bf16").reshape(nb, hkv, bs, d)
-    vc = workloads.normal_values(rng, nb * hkv * bs * d, "bf16").reshape(nb, hkv, bs, d)
-    q = workloads.normal_values(rng, nseq * hq * d, "bf16").reshape(nseq, hq, d)
-    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).cuda()  # noqa
+    def values(n):
+        if dtype == "f16":
+            return rng.standard_normal(n, dtype=np.float32).astype(np.float16).view(np.uint16)
+        return workloads.normal_values(rng, n, "bf16")
+    kc = values(nb * hkv * bs * d).reshape(nb, hkv, bs, d)
+    vc = values(nb * hkv * bs * d).reshape(nb, hkv, bs, d)
+    q = values(nseq * hq * d).reshape(nseq, hq, d)
+    tdt = torch.float16 if dtype == "f16" else torch.bfloat16
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(tdt).cuda()  # noqa
     plan = pa.prefix_plan_to_device(a.prefix_plan(list(range(nseq)), hq // hkv))
     assert plan["num_chunks"] >= 1
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -75,8 +84,8 @@ def test_shared_shapes(hq, hkv, d, bs, joint):
                                      torch.from_numpy(lens).cuda(), 1 / math.sqrt(d), plan, dev_status=status)
     torch.cuda.synchronize()
     assert status.item() == 0
-    ref = attention.decode_attention(q, kc, vc, tables, lens, 1 / math.sqrt(d), "bf16")
-    assert_decode_close(out, ref, "bf16", f"shared hq{hq} hkv{hkv} d{d} bs{bs}")
+    ref = attention.decode_attention(q, kc, vc, tables, lens, 1 / math.sqrt(d), dtype)
+    assert_decode_close(out, ref, dtype, f"shared {dtype} hq{hq} hkv{hkv} d{d} bs{bs}")
 
 
 def test_bad_plan_entries_are_skipped_and_flagged(joint):
