@@ -59,7 +59,8 @@ def parse_args(argv=None):
                     help="decode shared leading pages once per group (auto: on for prefix/beam32k)")
     ap.add_argument("--no-graph", action="store_true",
                     help="time eager launches instead of replaying the step as a CUDA graph")
-    ap.add_argument("--joint-kernel", choices=["auto", "tcgen05", "tcgen05_serial", "mma_sync"], default="auto",
+    ap.add_argument("--joint-kernel", choices=["auto", "tcgen05", "tcgen05_2cta", "tcgen05_serial", "mma_sync"],
+                    default="auto",
                     help="kernel for the shared partitions of a prefix group")
     return ap.parse_args(argv)
 
@@ -411,6 +412,7 @@ def run_ours(args):
     warps, stages = (int(x) for x in args.tiling.split("x"))
     pa.pa_set_decode_tiling(warps, stages)
     pa.pa_set_shared_prefix_kernel({"auto": pa.PA_SHARED_PREFIX_AUTO, "tcgen05": pa.PA_SHARED_PREFIX_TCGEN05,
+                                    "tcgen05_2cta": pa.PA_SHARED_PREFIX_TCGEN05_2CTA,
                                     "tcgen05_serial": pa.PA_SHARED_PREFIX_TCGEN05_SERIAL,
                                     "mma_sync": pa.PA_SHARED_PREFIX_MMA_SYNC}[args.joint_kernel])
 

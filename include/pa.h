@@ -265,7 +265,8 @@ PA_API pa_status pa_decode_shared_prefix(const void* q, const void* key_cache, c
 /* Which joint kernel pa_decode_shared_prefix runs (process-wide; default
  * AUTO = TCGEN05): TCGEN05 is the pipelined persistent kernel on the 5th-
  * generation tensor cores (TMA loads, tcgen05.mma with Tensor Memory
- * accumulators, one CTA per SM); TCGEN05_SERIAL the one-partition-per-CTA
+ * accumulators, one CTA per SM); TCGEN05_2CTA the same pipeline in a leaner
+ * form that runs two CTAs per SM; TCGEN05_SERIAL the one-partition-per-CTA
  * tcgen05 kernel without the software pipeline; MMA_SYNC the mma.sync
  * kernel.  All compute the same partials; the switch exists for testing and
  * measurement. */
@@ -273,7 +274,8 @@ typedef enum pa_shared_prefix_kernel {
   PA_SHARED_PREFIX_AUTO = 0,
   PA_SHARED_PREFIX_TCGEN05 = 1,
   PA_SHARED_PREFIX_MMA_SYNC = 2,
-  PA_SHARED_PREFIX_TCGEN05_SERIAL = 3
+  PA_SHARED_PREFIX_TCGEN05_SERIAL = 3,
+  PA_SHARED_PREFIX_TCGEN05_2CTA = 4
 } pa_shared_prefix_kernel;
 PA_API pa_status pa_set_shared_prefix_kernel(pa_shared_prefix_kernel kernel);
 

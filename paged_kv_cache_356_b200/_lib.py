@@ -17,6 +17,7 @@ PA_PREFIX_QUERIES_PER_CTA = 128
 PA_DEV_TIMEOUT = 32
 PA_DECODE_AUTO, PA_DECODE_CUDA_CORES, PA_DECODE_TENSOR_CORES = 0, 1, 2
 PA_SHARED_PREFIX_AUTO, PA_SHARED_PREFIX_TCGEN05, PA_SHARED_PREFIX_MMA_SYNC, PA_SHARED_PREFIX_TCGEN05_SERIAL = 0, 1, 2, 3
+PA_SHARED_PREFIX_TCGEN05_2CTA = 4
 PA_FAULT_NONE, PA_FAULT_WITHHOLD_FIRST_ITEM = 0, 1
 PA_PARTITION_TOKENS = 512
 PA_FIXED_SCRATCH_BYTES = 32 * 1024 * 1024

@@ -1671,6 +1671,448 @@ __global__ void __launch_bounds__(Tc05pShape<D, STAGES>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Two-CTAs-per-SM variant of the persistent tcgen05 shared-prefix kernel.  The
+// one-CTA kernel is bound by its own per-step chain (S MMA, softmax pass, O
+// MMA) while the SM's tensor pipe and its share of DRAM stay mostly idle; two
+// CTAs per SM run two such chains side by side.  To fit two per SM a CTA keeps
+// one query buffer, a STAGES-deep K/V ring (about 99 KB of shared memory at
+// D 128), 256 TMEM columns (S, two P buffers, O) and 7 warps:
+//   warps 0-3  softmax, as in the one-CTA kernel; the S row is read in two
+//              32-column halves, once for the maximum and once for the
+//              weights, to stay within the register budget of two CTAs
+//   warps 4-5  producers: 8 TMA boxes each per step; after an item's last step
+//              and once its epilogue has freed the query buffer, the next
+//              item's queries (two rows per lane), table slice, descriptor and
+//              workspace rows
+//   warp 6     MMA issuer (one lane): S(g) once the softmax has read S(g-1) out,
+//              then O += P(g-1).V(g-1)
+// Hand-offs, bounded waits, the abort path and the fault hook are those of the
+// one-CTA kernel.
+// ---------------------------------------------------------------------------
+template <int D, int STAGES>
+struct Tc05dShape {
+  static constexpr int kProducerWarps = 2;
+  static constexpr int kMmaWarp = 6;
+  static constexpr int kThreads = 32 * 7;
+  static constexpr int kRows = 128;
+  static constexpr int kStep = 64;
+  static constexpr int kStepsPerItem = kPartition / kStep;  // 8
+  static constexpr int kBlocks = D / 64;
+  static constexpr int kQBlockBytes = kRows * 128;
+  static constexpr int kQBytes = kBlocks * kQBlockBytes;
+  static constexpr int kKVBlockBytes = kStep * 128;
+  static constexpr int kTileBytes = kBlocks * kKVBlockBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kBoxBytes = 16 * 128;
+  static constexpr int kBoxesPerStep = 2 * (kStep / 16) * kBlocks;
+  static constexpr int kBoxesPerWarp = kBoxesPerStep / kProducerWarps;
+  static constexpr int kQOff = 0;
+  static constexpr int kStageOff = kQBytes;
+  static constexpr int kSliceOff = kStageOff + STAGES * kStageBytes;  // int32 [32] table slice
+  static constexpr int kDescOff = kSliceOff + 128;                     // int32 [4] item descriptor
+  static constexpr int kRowOff = kDescOff + 16;                        // int32 [kRows] workspace rows
+  static constexpr int kBarOff = kRowOff + kRows * 4;
+  // s_full, s_free, q_full, item_free, mma_drain; p_full, o_done x2; kv_full, kv_empty x STAGES
+  static constexpr int kNumBars = 5 + 4 + 2 * STAGES;
+  static constexpr int kTaddrOff = kBarOff + 8 * kNumBars;
+  static constexpr int kSmemBytes = kTaddrOff + 16 + 1024;
+  static constexpr uint32_t kTmemCols = 256;
+  static constexpr uint32_t kSCol = 0, kPCol = 64, kOCol = 128;  // S at 0, P[b] at 64 + 32b, O at 128
+  static_assert(D <= 128, "O needs D <= 128 columns");
+  static_assert(kBoxesPerStep % kProducerWarps == 0 && kBoxesPerWarp <= 32, "one lane per box");
+  static_assert(kRows == 2 * 32 * kProducerWarps, "two query rows per producer lane");
+  static_assert(kQBytes >= 4 * 32 * 20 * 4, "the epilogue's four 32-row float tiles fit in the query buffer");
+  static_assert(2 * (kSmemBytes + 1024) <= 228 * 1024, "two CTAs per SM");
+};
+
+template <typename T, int D, int STAGES>
+__global__ void __launch_bounds__(Tc05dShape<D, STAGES>::kThreads, 2)
+    decode_shared_tc05d_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
+                               const __grid_constant__ CUtensorMap tmap_v, const int32_t* __restrict__ chunks,
+                               int num_chunks, const int32_t* __restrict__ members, int num_members, int num_seqs,
+                               int max_shared_partitions, int fault) {
+  using S = Tc05dShape<D, STAGES>;
+  constexpr int SPI = S::kStepsPerItem;
+  extern __shared__ uint8_t smem_raw[];
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int bs = a.block_size;
+  const int G = a.group;
+  const int64_t total_rows = (int64_t)a.num_blocks * a.num_kv_heads * bs;
+  const int64_t total_items = (int64_t)max_shared_partitions * a.num_kv_heads * num_chunks;
+
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  int32_t* tslice = reinterpret_cast<int32_t*>(base_ptr + S::kSliceOff);
+  volatile int32_t* desc = reinterpret_cast<volatile int32_t*>(base_ptr + S::kDescOff);
+  int32_t* prow_s = reinterpret_cast<int32_t*>(base_ptr + S::kRowOff);
+  const uint32_t bar0 = base + S::kBarOff;
+  const uint32_t s_full = bar0, s_free = bar0 + 8u, q_full = bar0 + 16u, item_free = bar0 + 24u,
+                 mma_drain = bar0 + 32u;
+  auto p_full = [&](int b) { return bar0 + 40u + 8u * b; };
+  auto o_done = [&](int b) { return bar0 + 56u + 8u * b; };
+  auto kv_full = [&](int st) { return bar0 + 72u + 8u * st; };
+  auto kv_empty = [&](int st) { return bar0 + 72u + 8u * STAGES + 8u * st; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + S::kTaddrOff + 8);
+  const uint32_t taddr_slot = base + S::kTaddrOff;
+
+  auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    const long long t0 = clock64();
+    while (!tc05::mbar_try_wait_sleep(bar, parity, 20000u)) {
+      if (*abort_flag) return false;
+      if (clock64() - t0 > kWaitCycles) {
+        *abort_flag = 1;
+        return false;
+      }
+    }
+    return true;
+  };
+  auto wwait = [&](uint32_t bar, uint32_t parity) -> bool { return __all_sync(kFull, wait(bar, parity)); };
+
+  if (tid == 0) {
+    tc05::mbar_init(s_full, 1);
+    tc05::mbar_init(s_free, 4);      // one arrival per softmax warp
+    tc05::mbar_init(q_full, S::kProducerWarps);
+    tc05::mbar_init(item_free, 4);
+    tc05::mbar_init(mma_drain, 1);
+    for (int b = 0; b < 2; ++b) {
+      tc05::mbar_init(p_full(b), 4);
+      tc05::mbar_init(o_done(b), 1);
+    }
+    for (int st = 0; st < STAGES; ++st) {
+      tc05::mbar_init(kv_full(st), S::kProducerWarps);
+      tc05::mbar_init(kv_empty(st), 1);
+    }
+    *abort_flag = 0;
+    tc05::fence_mbar_init();
+    tc05::prefetch_tensormap(&tmap_k);
+    tc05::prefetch_tensormap(&tmap_v);
+  }
+  if (warp == 0) {
+    tc05::alloc(taddr_slot, S::kTmemCols);
+    tc05::relinquish();
+  }
+  tc05::fence_before();
+  __syncthreads();
+  tc05::fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base_ptr + S::kTaddrOff);
+  if (tid == 0) asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  int64_t cursor = blockIdx.x;
+  int64_t prod_g = 0;
+  const uint32_t qs = base + S::kQOff;
+
+  if (warp == 4 || warp == 5) {
+    // ---------------------------------------------------------------- producers
+    const int pw = warp - 4;
+    const T* qbase = reinterpret_cast<const T*>(a.q);
+    auto load_pages = [&](const SharedItem& it) -> int {
+      const int fb = it.p * kPartition / bs;
+      const int nblk = (it.p * kPartition + kPartition - 1) / bs - fb + 1;
+      return lane < nblk ? __ldg(a.block_tables + (int64_t)it.leader * a.max_blocks_per_seq + fb + lane) : -1;
+    };
+    auto load_q = [&](const SharedItem& it, int pages) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int r = pw * 64 + 32 * k + lane;
+        int64_t row = -1;
+        if (r < it.mcount * G) {
+          const int mi = r / G;
+          const int b = __ldg(members + it.moff + mi);
+          if ((unsigned)b < (unsigned)num_seqs) row = (int64_t)b * a.num_q_heads + it.kvh * G + (r - mi * G);
+        }
+        const T* src = qbase + (row < 0 ? 0 : row) * D;
+#pragma unroll
+        for (int ck = 0; ck < D / 8; ++ck)
+          cp_async_16(qs + (ck >> 3) * S::kQBlockBytes + r * 128 + (((ck & 7) ^ (r & 7)) << 4), src + ck * 8,
+                      row < 0 ? 0u : 16u);
+        prow_s[r] = row < 0 ? -1 : (int32_t)(row * a.max_partitions + it.p);
+      }
+      if (pw == 0) {
+        tslice[lane] = pages;
+        if (lane == 0) {
+          desc[1] = it.p;
+          desc[2] = it.kvh;
+          desc[3] = it.mcount;
+          desc[0] = 1;
+        }
+      }
+      cp_async_commit();
+    };
+    auto end_walk = [&]() {
+      if (pw == 0 && lane == 0) desc[0] = 0;
+    };
+    auto publish_q = [&]() {
+      cp_async_wait<0>();
+      tc05::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(q_full) : "memory");
+    };
+    SharedItem it = next_shared_item(cursor, total_items, num_chunks, a, chunks, num_members, num_seqs,
+                                     pw == 0 && lane == 0);
+    int my_page = it.valid ? load_pages(it) : -1;
+    if (it.valid) load_q(it, my_page);
+    else end_walk();
+    if (fault != PA_FAULT_WITHHOLD_FIRST_ITEM) publish_q();
+    else cp_async_wait<0>();  // test hook: the other roles' waits for this hand-off run out
+    int64_t g = 0;
+    for (int j = 0; it.valid; ++j) {
+      const SharedItemPrefetch pf = prefetch_shared_item(cursor, total_items, num_chunks, chunks);
+      SharedItem nxt{};
+      nxt.valid = false;
+      const int fb = it.p * kPartition / bs;
+      int nxt_page = -1;
+      bool stop = false;
+      for (int i = 0; i < SPI; ++i, ++g) {
+        const int st = (int)(g % STAGES);
+        if (g >= STAGES && !wwait(kv_empty(st), (uint32_t)(((g - STAGES) / STAGES) & 1))) { stop = true; break; }
+        if (lane == 0) tc05::mbar_arrive_expect_tx(kv_full(st), S::kBoxesPerWarp * S::kBoxBytes);
+        const int box = pw * S::kBoxesPerWarp + lane;
+        const int kv = box & 1;
+        const int blk = (box >> 1) % S::kBlocks;
+        const int rb = ((box >> 1) / S::kBlocks) % (S::kStep / 16);
+        const int tok = it.p * kPartition + i * S::kStep + 16 * rb;
+        const int page = __shfl_sync(kFull, my_page, tok / bs - fb);
+        __syncwarp();
+        if (lane < S::kBoxesPerWarp) {
+          const int64_t y = (unsigned)page < (unsigned)a.num_blocks
+                                ? ((int64_t)page * a.num_kv_heads + it.kvh) * bs + tok % bs
+                                : total_rows;  // out of range: the box is filled with zeros
+          const uint32_t dst = base + S::kStageOff + st * S::kStageBytes + kv * S::kTileBytes +
+                               blk * S::kKVBlockBytes + rb * S::kBoxBytes;
+          tc05::tma_load_2d(dst, kv ? (const void*)&tmap_v : (const void*)&tmap_k, kv_full(st), 64 * blk, (int32_t)y);
+        }
+        __syncwarp();
+        prod_g = g + 1;
+        if (i == SPI - 3) {
+          nxt = resolve_shared_item(pf, cursor, total_items, num_chunks, a, chunks, num_members, num_seqs,
+                                    pw == 0 && lane == 0);
+          if (nxt.valid) nxt_page = load_pages(nxt);
+        }
+      }
+      if (stop || __any_sync(kFull, *abort_flag != 0)) break;
+      // The query buffer is free once item j's epilogue has read it out.
+      if (!wwait(item_free, (uint32_t)(j & 1))) break;
+      if (nxt.valid) load_q(nxt, nxt_page);
+      else end_walk();
+      publish_q();
+      it = nxt;
+      my_page = nxt_page;
+    }
+    cp_async_wait<0>();  // nothing may land in shared memory after the CTA leaves
+  } else if (warp == S::kMmaWarp) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+      constexpr uint32_t idesc_s = tc05::instr_desc_f16(fmt, S::kRows, S::kStep, 0, 0);
+      constexpr uint32_t idesc_o = tc05::instr_desc_f16(fmt, S::kRows, D, 0, 1);
+      auto mma2 = [&](int64_t gp) -> bool {  // O += P(gp) . V(gp)
+        if (!wait(p_full((int)(gp & 1)), (uint32_t)((gp >> 1) & 1))) return false;
+        tc05::fence_after();
+        const int st = (int)(gp % STAGES);
+        const uint32_t vs = base + S::kStageOff + st * S::kStageBytes + S::kTileBytes;
+        const int ip = (int)(gp % SPI);
+#pragma unroll
+        for (int kt = 0; kt < S::kStep / 16; ++kt)
+          tc05::mma_ts(tmem + S::kOCol, tmem + S::kPCol + 32 * (uint32_t)(gp & 1) + 8 * kt,
+                       tc05::smem_desc_sw128(vs + kt * 16 * 128, S::kKVBlockBytes, 1024), idesc_o,
+                       (ip > 0 || kt > 0) ? 1u : 0u);
+        tc05::commit(o_done((int)(gp & 1)));
+        tc05::commit(kv_empty(st));
+        return true;
+      };
+      int64_t g = 0;
+      bool ok = true;
+      for (int j = 0; ok; ++j) {
+        if (!wait(q_full, (uint32_t)(j & 1))) break;
+        if (desc[0] == 0) break;  // the walk has ended
+        tc05::fence_after();
+        tc05::fence_proxy_async_smem();
+        for (int i = 0; i < SPI; ++i, ++g) {
+          const int st = (int)(g % STAGES);
+          if (!wait(kv_full(st), (uint32_t)((g / STAGES) & 1))) { ok = false; break; }
+          if (g >= 1 && !wait(s_free, (uint32_t)((g - 1) & 1))) { ok = false; break; }  // S(g-1) read out
+          tc05::fence_after();
+          const uint32_t ks = base + S::kStageOff + st * S::kStageBytes;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t blk = k >> 2, koff = (k & 3) * 32;
+            tc05::mma_ss(tmem + S::kSCol, tc05::smem_desc_sw128(qs + blk * S::kQBlockBytes + koff, 16, 1024),
+                         tc05::smem_desc_sw128(ks + blk * S::kKVBlockBytes + koff, 16, 1024), idesc_s,
+                         k > 0 ? 1u : 0u);
+          }
+          tc05::commit(s_full);
+          if (i >= 1 && !mma2(g - 1)) { ok = false; break; }
+        }
+        if (ok && !mma2(g - 1)) ok = false;  // close the item
+      }
+      tc05::commit(mma_drain);
+      {
+        const long long t0 = clock64();
+        while (!tc05::mbar_try_wait(mma_drain, 0) && clock64() - t0 < kWaitCycles) {
+        }
+      }
+    }
+  } else if (warp < 4) {
+    // ---------------------------------------------------------------- softmax warps 0-3
+    const uint32_t row_t = tmem + ((uint32_t)(32 * warp) << 16);
+    int64_t g = 0;
+    for (int j = 0;; ++j) {
+      if (!wwait(q_full, (uint32_t)(j & 1))) break;  // item, table slice and rows
+      if (desc[0] == 0) break;                        // the walk has ended
+      const int ip = desc[1];
+      const int mcount = desc[3];
+      const bool busy = 32 * warp < mcount * G;
+      const uint32_t page_ok = __ballot_sync(
+          kFull, (unsigned)tslice[(ip * kPartition + 16 * lane) / bs - ip * kPartition / bs] < (unsigned)a.num_blocks);
+      float m_use = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int i = 0; i < SPI; ++i, ++g) {
+        if (!wwait(s_full, (uint32_t)(g & 1))) { ok = false; break; }
+        tc05::fence_after();
+        if (!busy && lane == 0)  // nothing to read: S is free at once
+          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(s_free) : "memory");
+        const int bad = (int)(~page_ok >> (4 * i)) & 0xF;  // 16-token groups whose page is out of range
+        float alpha = 1.f, ref = 0.f;
+        if (busy) {
+          // Pass 1: the step's maximum, 32 columns at a time.
+          float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t sr[32];
+            tc05::ld32(row_t + S::kSCol + 32 * h, sr);
+            tc05::wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const bool okg = !((bad >> (2 * h + (e >> 4))) & 1);
+              mx4[e & 3] = fmaxf(mx4[e & 3], okg ? __uint_as_float(sr[e]) * a.qk_scale_log2 : -INFINITY);
+            }
+          }
+          const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+          if (mx > m_use + 8.f) {
+            alpha = m_use == -INFINITY ? 0.f : ex2_approx(m_use - mx);
+            m_use = mx;
+          }
+          ref = m_use == -INFINITY ? 0.f : m_use;
+        }
+        // O is rescaled before this step's P . V is added (MMA2 of step g waits for p_full(g)).
+        if (busy && i > 0 && __any_sync(kFull, alpha != 1.f)) {
+          if (!wwait(o_done((int)((g - 1) & 1)), (uint32_t)(((g - 1) >> 1) & 1))) { ok = false; break; }
+          tc05::fence_after();
+#pragma unroll 1
+          for (int cb = 0; cb < D / 16; ++cb) {
+            uint32_t ov[16];
+            tc05::ld16(row_t + S::kOCol + 16 * cb, ov);
+            tc05::wait_ld();
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) ov[jj] = __float_as_uint(__uint_as_float(ov[jj]) * alpha);
+            tc05::st16(row_t + S::kOCol + 16 * cb, ov);
+          }
+        }
+        // P buffer g & 1 was last read by O += P.V of step g - 2.
+        if (g >= 2 && !wwait(o_done((int)(g & 1)), (uint32_t)(((g - 2) >> 1) & 1))) { ok = false; break; }
+        tc05::fence_after();
+        // Pass 2: weights, 32 columns at a time, stored as 16-bit pairs.
+        if (busy) {
+          float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t sr[32];
+            tc05::ld32(row_t + S::kSCol + 32 * h, sr);
+            tc05::wait_ld();
+            if (h == 1) {  // S has been read out: the next S may be computed
+              tc05::fence_before();
+              __syncwarp();
+              if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(s_free) : "memory");
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              const int e0 = 2 * jj, e1 = 2 * jj + 1;
+              const bool okg = !((bad >> (2 * h + (e0 >> 4))) & 1);
+              const float p0 = okg ? ex2_approx(__uint_as_float(sr[e0]) * a.qk_scale_log2 - ref) : 0.f;
+              const float p1 = okg ? ex2_approx(__uint_as_float(sr[e1]) * a.qk_scale_log2 - ref) : 0.f;
+              ls[jj & 3] += p0 + p1;
+              pk[jj] = pack2<T>(p0, p1);
+            }
+            tc05::st16(row_t + S::kPCol + 32 * (uint32_t)(g & 1) + 16 * h, pk);
+          }
+          l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+          tc05::wait_st();
+        }
+        // P of step g is in TMEM.
+        tc05::fence_before();
+        __syncwarp();
+        if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(p_full((int)(g & 1))) : "memory");
+      }
+      if (!ok) break;
+      // Epilogue: the item's last O += P.V (step g - 1) has to complete.
+      const int64_t gl = g - 1;
+      if (!wwait(o_done((int)(gl & 1)), (uint32_t)((gl >> 1) & 1))) break;
+      tc05::fence_after();
+      if (busy) {
+        const int32_t prow = prow_s[tid];
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        constexpr int kTileStride = 20;  // floats; 16-byte accesses conflict-free both ways
+        float* tile = reinterpret_cast<float*>(base_ptr + S::kQOff) + warp * 32 * kTileStride;
+        float4* wr = reinterpret_cast<float4*>(tile + lane * kTileStride);
+        const int rsub = lane >> 2, csub = lane & 3;
+#pragma unroll 1
+        for (int cb = 0; cb < D / 16; ++cb) {
+          uint32_t ov[16];
+          tc05::ld16(row_t + S::kOCol + 16 * cb, ov);
+          tc05::wait_ld();
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            wr[q4] = make_float4(__uint_as_float(ov[4 * q4]) * inv, __uint_as_float(ov[4 * q4 + 1]) * inv,
+                                 __uint_as_float(ov[4 * q4 + 2]) * inv, __uint_as_float(ov[4 * q4 + 3]) * inv);
+          __syncwarp();
+          float4 v[4];
+          int32_t pr[4];
+#pragma unroll
+          for (int ii = 0; ii < 4; ++ii) {
+            pr[ii] = __shfl_sync(kFull, prow, 8 * ii + rsub);
+            v[ii] = *reinterpret_cast<const float4*>(tile + (8 * ii + rsub) * kTileStride + 4 * csub);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int ii = 0; ii < 4; ++ii)
+            if (pr[ii] >= 0) *reinterpret_cast<float4*>(a.o_part + (int64_t)pr[ii] * D + 16 * cb + 4 * csub) = v[ii];
+        }
+        if (prow >= 0) {
+          a.m_part[prow] = m_use == -INFINITY ? -INFINITY : m_use * kLn2;
+          a.l_part[prow] = l;
+        }
+      }
+      tc05::fence_before();
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(item_free) : "memory");
+    }
+  }
+
+  // -- teardown ---------------------------------------------------------------------------------
+  __syncthreads();
+  if (*abort_flag) {
+    if (tid == 0) flag_status(a.status, PA_DEV_TIMEOUT);
+    if (warp == 4 && lane == 0)
+      for (int64_t gl = prod_g > STAGES ? prod_g - STAGES : 0; gl < prod_g; ++gl) {
+        const long long t0 = clock64();
+        while (!tc05::mbar_try_wait(kv_full((int)(gl % STAGES)), (uint32_t)((gl / STAGES) & 1)) &&
+               clock64() - t0 < kWaitCycles) {
+        }
+      }
+  }
+  cp_async_wait<0>();
+  tc05::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc05::fence_after();
+    tc05::dealloc(tmem, S::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Log-sum-exp merge of the partitions.  A CTA of max(4, WPI) warps serves
 // max(4, WPI) / WPI (sequence, query head) items with WPI warps each (WPI
 // grows with the partition count).  Warp w of an item merges partitions w,
@@ -1992,6 +2434,32 @@ cudaError_t launch_shared_tc05p(const DecodeArgs& a, const CUtensorMap& mk, cons
   return cudaGetLastError();
 }
 
+template <typename T, int D>
+cudaError_t launch_shared_tc05d(const DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, int num_chunks,
+                                const int32_t* chunks, const int32_t* members, int num_members, int num_seqs,
+                                int max_sp, cudaStream_t stream) {
+  constexpr int kStages = D == 128 ? 2 : 4;
+  using S = Tc05dShape<D, kStages>;
+  static std::atomic<uint64_t> done{0};
+  auto kernel = decode_shared_tc05d_kernel<T, D, kStages>;
+  cudaError_t err = ensure_smem(kernel, S::kSmemBytes, done);
+  if (err != cudaSuccess) return err;
+  // Two CTAs per SM need the largest shared-memory carveout.
+  static std::atomic<uint64_t> carve{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev < 64 && !(carve.load() & (1ull << dev))) {
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (err != cudaSuccess) return err;
+    carve.fetch_or(1ull << dev);
+  }
+  const int64_t items = (int64_t)max_sp * a.num_kv_heads * num_chunks;
+  const int64_t slots = 2 * (int64_t)sm_count();
+  const int grid = (int)(items < slots ? items : slots);
+  kernel<<<grid, S::kThreads, S::kSmemBytes, stream>>>(a, mk, mv, chunks, num_chunks, members, num_members, num_seqs,
+                                                       max_sp, g_fault.load());
+  return cudaGetLastError();
+}
+
 std::atomic<int> g_shared_kernel{PA_SHARED_PREFIX_AUTO};
 
 template <typename T>
@@ -1999,15 +2467,23 @@ cudaError_t launch_shared_dim(const DecodeArgs& a, int head_dim, dim3 grid, cons
                               const int32_t* members, int num_members, int num_seqs, pa_dtype dtype,
                               cudaStream_t stream) {
   const int choice = g_shared_kernel.load();
-  if (choice == PA_SHARED_PREFIX_AUTO || choice == PA_SHARED_PREFIX_TCGEN05) {
+  if (choice == PA_SHARED_PREFIX_AUTO || choice == PA_SHARED_PREFIX_TCGEN05 ||
+      choice == PA_SHARED_PREFIX_TCGEN05_2CTA) {
     const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * a.block_size;
     CUtensorMap mk, mv;
     if (rows < (1ll << 31) && encode_cache_map(&mk, a.key_cache, dtype, rows, head_dim) &&
         encode_cache_map(&mv, a.value_cache, dtype, rows, head_dim)) {
+      const bool two = choice == PA_SHARED_PREFIX_TCGEN05_2CTA;
       if (head_dim == 64)
-        return launch_shared_tc05p<T, 64>(a, mk, mv, grid.x, chunks, members, num_members, num_seqs, grid.z, stream);
+        return two ? launch_shared_tc05d<T, 64>(a, mk, mv, grid.x, chunks, members, num_members, num_seqs, grid.z,
+                                                stream)
+                   : launch_shared_tc05p<T, 64>(a, mk, mv, grid.x, chunks, members, num_members, num_seqs, grid.z,
+                                                stream);
       if (head_dim == 128)
-        return launch_shared_tc05p<T, 128>(a, mk, mv, grid.x, chunks, members, num_members, num_seqs, grid.z, stream);
+        return two ? launch_shared_tc05d<T, 128>(a, mk, mv, grid.x, chunks, members, num_members, num_seqs, grid.z,
+                                                 stream)
+                   : launch_shared_tc05p<T, 128>(a, mk, mv, grid.x, chunks, members, num_members, num_seqs, grid.z,
+                                                 stream);
     }
   }
   const bool tc05 = choice != PA_SHARED_PREFIX_MMA_SYNC;
@@ -2090,7 +2566,7 @@ extern "C" pa_status pa_set_fault_injection(int32_t mode) {
 
 extern "C" pa_status pa_set_shared_prefix_kernel(pa_shared_prefix_kernel k) {
   if (k != PA_SHARED_PREFIX_AUTO && k != PA_SHARED_PREFIX_TCGEN05 && k != PA_SHARED_PREFIX_MMA_SYNC &&
-      k != PA_SHARED_PREFIX_TCGEN05_SERIAL)
+      k != PA_SHARED_PREFIX_TCGEN05_SERIAL && k != PA_SHARED_PREFIX_TCGEN05_2CTA)
     return fail(PA_ERR_INVALID, "pa_set_shared_prefix_kernel: unknown kernel %d", (int)k);
   g_shared_kernel.store((int)k);
   return PA_OK;
