@@ -1062,13 +1062,13 @@ __global__ void __launch_bounds__(128, 1) decode_shared_tc05_kernel(const Decode
 // Warp-specialised, persistent shared-prefix kernel on tcgen05 (the default
 // joint kernel).  One CTA per SM walks work items (chunk, kv head, shared
 // partition) with stride gridDim.x; an item is 8 steps of 64 tokens.  Roles
-// (9 warps):
+// (8 warps):
 //   warps 0-3  softmax: thread r owns query row r; per step it reads its S row
 //              from TMEM, keeps the running max / sum (lazy rescaling of O),
 //              writes P (16-bit) to TMEM; at the end of an item it writes the
 //              partials.
-//   warps 4-6, 8  producers: K/V pages by TMA into a ring of STAGES buffers, as
-//              far ahead as the ring allows, each warp a quarter of a step's
+//   warps 4-6  producers: K/V pages by TMA into a ring of STAGES buffers, as
+//              far ahead as the ring allows, each warp a third of a step's
 //              16-row boxes (one warp alone cannot issue boxes fast enough to
 //              keep up with HBM); three steps before an item ends they start
 //              the next item's queries (cp.async, one row per lane) into the
@@ -1091,11 +1091,14 @@ __global__ void __launch_bounds__(128, 1) decode_shared_tc05_kernel(const Decode
 // ---------------------------------------------------------------------------
 template <int D, int STAGES>
 struct Tc05pShape {
-  static constexpr int kProducerWarps = 4;  // TMA issue from one warp tops out near 41 GB/s per SM
+  // TMA issue from one warp tops out near 41 GB/s per SM; three keep up with the step chain, and 8
+  // warps in all (two per scheduler) leave each thread up to 255 registers.
+  static constexpr int kProducerWarps = 3;
   // Warp w runs on scheduler w % 4.  The MMA warp takes scheduler 3: softmax
   // warp 0 (scheduler 0) has rows in every item, warp 3 only in full ones.
   static constexpr int kMmaWarp = 7;
   static constexpr int kThreads = 32 * (4 + kProducerWarps + 1);
+  static_assert(kMmaWarp == 4 + kProducerWarps, "producers are warps 4 .. kMmaWarp - 1");
   static constexpr int kRows = 128;
   static constexpr int kStep = 64;
   static constexpr int kStepsPerItem = kPartition / kStep;  // 8
@@ -1120,9 +1123,10 @@ struct Tc05pShape {
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kSCol = 0, kPCol = 128, kOCol = 256;  // S[b] at 64b, P[b] at 128 + 32b, O[b] at 256 + 128b
   static_assert(D <= 128, "O double buffer needs D <= 128");
-  static constexpr int kBoxesPerWarp = kBoxesPerStep / kProducerWarps;
-  static_assert(kBoxesPerStep % kProducerWarps == 0 && kBoxesPerWarp <= 32, "one lane per box");
-  static_assert(kRows == 32 * kProducerWarps, "one query row per producer lane");
+  // Producer pw issues boxes pw, pw + 3, ... and loads query rows pw * 32 + lane (+ 96).
+  __host__ __device__ static constexpr int boxes_of(int pw) { return (kBoxesPerStep - pw + kProducerWarps - 1) / kProducerWarps; }
+  static_assert(kBoxesPerStep <= 32 * kProducerWarps, "one lane per box");
+  static_assert(kRows <= 64 * kProducerWarps && kRows > 32 * kProducerWarps, "one or two query rows per lane");
   static_assert(kQBytes >= 4 * 32 * 20 * 4, "the epilogue's four 32-row float tiles fit in a query buffer");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -1324,23 +1328,27 @@ __global__ void __launch_bounds__(Tc05pShape<D, STAGES>::kThreads, 1)
       const int nblk = (it.p * kPartition + kPartition - 1) / bs - fb + 1;
       return lane < nblk ? __ldg(a.block_tables + (int64_t)it.leader * a.max_blocks_per_seq + fb + lane) : -1;
     };
-    // Query row pw * 32 + lane of `it` (zero past mcount * G) into buffer qb; the
-    // first producer warp also stores the table slice for the softmax warps.
+    // Query rows pw * 32 + lane (+ 96) of `it` (zero past mcount * G) into buffer qb;
+    // the first producer warp also stores the table slice for the softmax warps.
     auto load_q = [&](const SharedItem& it, int qb, int pages) {
       const uint32_t qs = base + S::kQOff + qb * S::kQBytes;
-      const int r = pw * 32 + lane;
-      int64_t row = -1;
-      if (r < it.mcount * G) {
-        const int mi = r / G;
-        const int b = __ldg(members + it.moff + mi);
-        if ((unsigned)b < (unsigned)num_seqs) row = (int64_t)b * a.num_q_heads + it.kvh * G + (r - mi * G);
-      }
-      const T* src = qbase + (row < 0 ? 0 : row) * D;
 #pragma unroll
-      for (int ck = 0; ck < D / 8; ++ck)
-        cp_async_16(qs + (ck >> 3) * S::kQBlockBytes + r * 128 + (((ck & 7) ^ (r & 7)) << 4), src + ck * 8,
-                    row < 0 ? 0u : 16u);
-      prow_s[qb * S::kRows + r] = row < 0 ? -1 : (int32_t)(row * a.max_partitions + it.p);
+      for (int k = 0; k < 2; ++k) {
+        const int r = pw * 32 + lane + 32 * S::kProducerWarps * k;
+        if (r >= S::kRows) break;
+        int64_t row = -1;
+        if (r < it.mcount * G) {
+          const int mi = r / G;
+          const int b = __ldg(members + it.moff + mi);
+          if ((unsigned)b < (unsigned)num_seqs) row = (int64_t)b * a.num_q_heads + it.kvh * G + (r - mi * G);
+        }
+        const T* src = qbase + (row < 0 ? 0 : row) * D;
+#pragma unroll
+        for (int ck = 0; ck < D / 8; ++ck)
+          cp_async_16(qs + (ck >> 3) * S::kQBlockBytes + r * 128 + (((ck & 7) ^ (r & 7)) << 4), src + ck * 8,
+                      row < 0 ? 0u : 16u);
+        prow_s[qb * S::kRows + r] = row < 0 ? -1 : (int32_t)(row * a.max_partitions + it.p);
+      }
       if (pw == 0) {
         tslice[qb * 32 + lane] = pages;
         if (lane == 0) {
@@ -1384,16 +1392,16 @@ __global__ void __launch_bounds__(Tc05pShape<D, STAGES>::kThreads, 1)
       for (int i = 0; i < SPI; ++i, ++g) {
         const int st = (int)(g % STAGES);
         if (g >= STAGES && !wwait(kv_empty(st), (uint32_t)(((g - STAGES) / STAGES) & 1))) { stop = true; break; }
-        if (lane == 0) tc05::mbar_arrive_expect_tx(kv_full(st), S::kBoxesPerWarp * S::kBoxBytes);
+        if (lane == 0) tc05::mbar_arrive_expect_tx(kv_full(st), S::boxes_of(pw) * S::kBoxBytes);
         // box -> (row box rb, 64-wide block blk, K or V)
-        const int box = pw * S::kBoxesPerWarp + lane;
+        const int box = pw + S::kProducerWarps * lane;
         const int kv = box & 1;
         const int blk = (box >> 1) % S::kBlocks;
         const int rb = ((box >> 1) / S::kBlocks) % (S::kStep / 16);
         const int tok = it.p * kPartition + i * S::kStep + 16 * rb;
         const int page = __shfl_sync(kFull, my_page, tok / bs - fb);
         __syncwarp();
-        if (lane < S::kBoxesPerWarp) {
+        if (box < S::kBoxesPerStep) {
           const int64_t y = (unsigned)page < (unsigned)a.num_blocks
                                 ? ((int64_t)page * a.num_kv_heads + it.kvh) * bs + tok % bs
                                 : total_rows;  // out of range: the box is filled with zeros
