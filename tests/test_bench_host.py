@@ -1,0 +1,30 @@
+"""Host-side pieces of bench.py that need no GPU: the partition kernel's source hash resolves its
+anchors, the committed ncu summary parses and still matches the sources, and the byte accounting of a
+decode step counts shared pages once."""
+import numpy as np
+
+import bench
+from paged_kv_cache_356_b200 import workloads
+
+
+def test_kernel_hash_and_committed_traffic_are_consistent():
+    h = bench.kernel_source_hash()
+    assert len(h) == 16 and int(h, 16) >= 0
+    traffic, committed = bench.profiled_traffic(h)
+    assert committed is not None and len(committed) == 16
+    if committed == h:   # counters taken on these sources: a plausible DRAM figure for the full batch
+        assert traffic is not None and 0.9 < traffic / 2965942736 < 1.1
+    else:                # the kernel changed since: the bench must report no traffic
+        assert traffic is None
+
+
+def test_unique_and_logical_kv_bytes():
+    w = workloads.beam32k(num_beams=3, prompt_len=64, own=16)
+    bs = w.block_size
+    # three sequences sharing 4 pages of prompt, each with one page of its own
+    tables = np.array([[0, 1, 2, 3, 4], [0, 1, 2, 3, 5], [0, 1, 2, 3, 6]], dtype=np.int32)
+    ctx = np.array([80, 80, 80], dtype=np.int32)
+    unique, logical = bench.kv_bytes(w, tables, ctx)
+    per_token = 2 * w.num_kv_heads * w.head_dim * w.elem_bytes
+    assert unique == (4 * bs + 3 * 16) * per_token
+    assert logical == 3 * 80 * per_token
