@@ -17,7 +17,8 @@ Modules
   allocator  ref-counted free-page pool, block tables, fork, copy-on-write
   cache_ops  writing tokens into page slots; whole-page copies
   attention  block-table gather + textbook softmax attention (fp64); the
-             split-context partials and their log-sum-exp merge
+             split-context partials and their log-sum-exp merge; several
+             causal query tokens per sequence (draft verification)
   formulas   block counts, KV bytes per token, internal waste
   scenario   runs a workload trace through the pieces above
 

@@ -22,6 +22,10 @@ decode path uses for long sequences: per 512-token partition the normalised
 partial output ``o_p``, the partition's score maximum ``m_p`` and
 ``l_p = sum exp(s_j - m_p)``; merging them with weights ``l_p * exp(m_p - M)``
 reproduces the unsplit softmax exactly (up to rounding).
+
+``verify_attention`` is the same attention for several query tokens per
+sequence (draft-token verification), each seeing the keys up to its own
+position.
 """
 from __future__ import annotations
 
@@ -97,3 +101,40 @@ def lse_merge(parts) -> np.ndarray:
     m_all = max(m for _, m, _ in parts)
     weights = [l * np.exp(m - m_all) for _, m, l in parts]
     return sum(w * o for w, (o, _, _) in zip(weights, parts)) / sum(weights)
+
+
+def visible_keys(context_len: int, num_tokens: int, t: int) -> int:
+    """Keys that query token t of ``num_tokens`` sees: positions ``0 .. context_len - num_tokens + t``."""
+    return max(0, context_len - num_tokens + t + 1)
+
+
+def verify_attention(q, key_cache, value_cache, block_tables, context_lens, scale: float,
+                     dtype: str, seqs=None) -> np.ndarray:
+    """fp64 output ``[B, T, H_q, D]`` for T query tokens per sequence (draft verification).
+
+    Internals, "The Mathematical Cause of KV Cache Fragmentation", points to
+    speculative-decoding kernels that check several draft tokens of a sequence
+    at once against its paged memory.  Reading (the page gives no formula):
+    the T query tokens of sequence b are the last T positions of its context,
+    ``pos_t = context_lens[b] - T + t``, their own K/V already written; token
+    t attends causally, i.e. to the keys ``j <= pos_t``, and to nothing else.
+    A token with ``pos_t < 0`` sees no key and yields zeros.  With T = 1 this
+    is ``decode_attention``.
+
+    ``q`` is ``[B, T, H_q, D]``; the other arguments are as in ``decode_attention``.
+    """
+    q64 = to_float64(q, dtype)
+    num_seqs, num_tokens, num_q_heads, head_dim = q64.shape
+    num_kv_heads = key_cache.shape[1]
+    group = num_q_heads // num_kv_heads
+    out = np.zeros(q64.shape, dtype=np.float64)
+    for b in (range(num_seqs) if seqs is None else seqs):
+        ctx = int(context_lens[b])
+        keys = to_float64(gather_sequence(key_cache, block_tables[b], ctx), dtype)
+        values = to_float64(gather_sequence(value_cache, block_tables[b], ctx), dtype)
+        for t in range(num_tokens):
+            visible = visible_keys(ctx, num_tokens, t)
+            for h in range(num_q_heads):
+                out[b, t, h] = softmax_attention(q64[b, t, h], keys[:visible, h // group, :],
+                                                 values[:visible, h // group, :], scale)
+    return out
