@@ -63,6 +63,11 @@ def parse_args(argv=None):
     ap.add_argument("--joint-kernel", choices=["auto", "tcgen05", "tcgen05_2cta", "tcgen05_serial", "mma_sync"],
                     default="auto",
                     help="kernel for the shared partitions of a prefix group")
+    ap.add_argument("--verify-tokens", type=int, default=0,
+                    help="T > 0: each step writes T draft tokens per sequence and runs pa_decode_verify "
+                         "(T causal query tokens per sequence) instead of a one-token decode step")
+    ap.add_argument("--verify-path", choices=["auto", "per_sequence", "joint"], default="auto",
+                    help="with --verify-tokens: joint kernel for the partitions all tokens see (auto: when T*G > 16)")
     return ap.parse_args(argv)
 
 
@@ -92,6 +97,19 @@ def partition_kernel_bytes(w, ctx, unique_kv):
     partials = sum(n for n in nparts if n > 1) * w.num_q_heads * (w.head_dim + 2) * 4
     rows = sum(1 for n in nparts if n <= 1) * w.num_q_heads * w.head_dim * eb
     return unique_kv + q + tables + lens + partials + rows
+
+
+def verify_call_bytes(w, ctx, unique_kv, num_tokens):
+    """Algorithmic bytes of one pa_decode_verify call (partition kernel + merge): KV + q + tables +
+    lengths, the partials written and read back, and every output row written once."""
+    eb = w.elem_bytes
+    nparts = [-(-int(c) // 512) for c in ctx]
+    rows = w.num_seqs * num_tokens * w.num_q_heads
+    q = rows * w.head_dim * eb
+    tables = 4 * sum(-(-int(c) // w.block_size) for c in ctx)
+    lens = 4 * w.num_seqs
+    partials = sum(n for n in nparts if n > 1) * num_tokens * w.num_q_heads * (w.head_dim + 2) * 4
+    return unique_kv + q + tables + lens + 2 * partials + rows * w.head_dim * eb
 
 
 def describe(w):
@@ -229,7 +247,7 @@ class OracleSample:
     this host; setup (allocator, cache writes of the prefill) is not timed.
     """
 
-    def __init__(self, name, seconds_per_step, max_seqs=256):
+    def __init__(self, name, seconds_per_step, max_seqs=256, verify_tokens=0):
         from oracle import attention, scenario
         from paged_kv_cache_356_b200 import workloads
 
@@ -246,6 +264,7 @@ class OracleSample:
         attention.decode_attention(probe.query(), res["key_cache"], res["value_cache"], res["block_tables"],
                                    res["context_lens"], probe.scale, probe.dtype)
         per_seq = max(time.perf_counter() - t0, 1e-3) * (np.mean(full.context_lens) / probe.context_lens[0])
+        per_seq *= max(1, verify_tokens)
         n = int(max(1, min(max_seqs, full.num_seqs, seconds_per_step / per_seq)))
         self.w = w = workloads.by_name(name, **{key: n})
         self.res = res = scenario.run(w)
@@ -254,21 +273,34 @@ class OracleSample:
         self.k_new, self.v_new = w.batched_token_kv(step_writes)
         self.slots = res["write_slots"][-sum(op[3] for op in step_writes):]
         self.unique, _ = kv_bytes(w, res["block_tables"], res["context_lens"])
+        self.verify_tokens = t = verify_tokens
+        if t > 0:      # draft tokens at the last t positions of each sequence
+            mgr = res["manager"]
+            self.slots = np.array([mgr.slot(b, p) for b in range(w.num_seqs)
+                                   for p in range(int(res["context_lens"][b]) - t, int(res["context_lens"][b]))],
+                                  dtype=np.int64)
+            self.k_new, self.v_new = w.draft_kv(t)
+            self.q = w.draft_query(t)
         self.desc = (f"first {w.num_seqs} of {full.num_seqs} sequences of the {name} batch "
-                     f"({int(np.sum(w.context_lens))} context tokens, {self.unique / 1e6:.1f} MB of KV)")
+                     f"({int(np.sum(w.context_lens))} context tokens, {self.unique / 1e6:.1f} MB of KV"
+                     + (f", {t} query tokens each" if t > 0 else "") + ")")
 
     def step(self):
         from oracle import attention, cache_ops
         r, w = self.res, self.w
         t0 = time.perf_counter()
         cache_ops.reshape_and_cache(self.k_new, self.v_new, self.slots, r["key_cache"], r["value_cache"])
-        attention.decode_attention(self.q, r["key_cache"], r["value_cache"], r["block_tables"], r["context_lens"],
-                                   w.scale, w.dtype)
+        if self.verify_tokens > 0:
+            attention.verify_attention(self.q, r["key_cache"], r["value_cache"], r["block_tables"],
+                                       r["context_lens"], w.scale, w.dtype)
+        else:
+            attention.decode_attention(self.q, r["key_cache"], r["value_cache"], r["block_tables"],
+                                       r["context_lens"], w.scale, w.dtype)
         return time.perf_counter() - t0
 
 
-def cpu_baseline(name, seconds):
-    sample = OracleSample(name, seconds / 4)
+def cpu_baseline(name, seconds, verify_tokens=0):
+    sample = OracleSample(name, seconds / 4, verify_tokens=verify_tokens)
     times = []
     while not times or sum(times) < seconds * 0.75:
         times.append(sample.step())
@@ -283,7 +315,8 @@ def run_reference(args):
         return 0
     from paged_kv_cache_356_b200 import workloads
     w = workloads.by_name(args.workload)
-    sample = OracleSample(args.workload, max(0.05, 90.0 / max(1, args.steps + args.warmup)))
+    sample = OracleSample(args.workload, max(0.05, 90.0 / max(1, args.steps + args.warmup)),
+                          verify_tokens=args.verify_tokens)
     for _ in range(args.warmup):
         sample.step()
     times = [sample.step() for _ in range(args.steps)]
@@ -293,7 +326,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": describe(w),
+            "config": dict(describe(w), **({"query_tokens": args.verify_tokens} if args.verify_tokens else {})),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": sample.cores, "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "note": "fp64 NumPy CPU oracle, as it stands, on the host cores; each step is a bounded sample"}
@@ -415,6 +448,8 @@ def run_ours(args):
                              "cc": pa.PA_DECODE_CUDA_CORES}[args.kernel])
     warps, stages = (int(x) for x in args.tiling.split("x"))
     pa.pa_set_decode_tiling(warps, stages)
+    pa.pa_set_verify_path({"auto": pa.PA_VERIFY_AUTO, "per_sequence": pa.PA_VERIFY_PER_SEQUENCE,
+                           "joint": pa.PA_VERIFY_JOINT}[args.verify_path])
     pa.pa_set_shared_prefix_kernel({"auto": pa.PA_SHARED_PREFIX_AUTO, "tcgen05": pa.PA_SHARED_PREFIX_TCGEN05,
                                     "tcgen05_2cta": pa.PA_SHARED_PREFIX_TCGEN05_2CTA,
                                     "tcgen05_serial": pa.PA_SHARED_PREFIX_TCGEN05_SERIAL,
@@ -434,6 +469,27 @@ def run_ours(args):
     max_ctx = w.max_blocks_per_seq * w.block_size
     stream = torch.cuda.current_stream()
     kd, vd, sd = run.step_write
+    q_step, out_step, ws_step = run.q, run.out, run.workspace
+    T = args.verify_tokens
+    verify_joint = False
+    if T > 0:
+        # draft verification: the step overwrites each sequence's last T positions with the draft
+        # tokens' K/V, then attends with T causal query tokens per sequence
+        if run.plan is not None or int(ctx_np.min()) < T:
+            raise SystemExit("--verify-tokens needs a workload without a shared-prefix plan and contexts >= T")
+        slots = np.concatenate([run.alloc.slot_mapping(b, int(ctx_np[b]) - T, T) for b in range(w.num_seqs)])
+        dk, dv = w.draft_kv(T)
+        kd, vd = run._to_device(dk), run._to_device(dv)
+        sd = torch.from_numpy(slots.astype(np.int64)).cuda()
+        q_step = run._to_device(w.draft_query(T))
+        out_step = torch.empty_like(q_step)
+        need = pa.pa_decode_verify_workspace_size(w.num_seqs, T, w.num_q_heads, w.head_dim, max_ctx)
+        ws_step = torch.empty(need, dtype=torch.uint8, device="cuda") if need > 0 else None
+        part_bytes = verify_call_bytes(w, ctx_np, unique, T)
+        verify_joint = (args.verify_path == "joint" or
+                        (args.verify_path == "auto" and T * w.group_size > 16 and args.kernel != "cc" and
+                         w.dtype in ("bf16", "f16") and w.head_dim in (64, 128) and w.block_size % 16 == 0 and
+                         max_ctx > 512))
 
     def step(evs=None, stream=stream):
         if evs is not None:
@@ -441,7 +497,12 @@ def run_ours(args):
         pa.pa_reshape_and_cache(kd, vd, sd, run.key_cache, run.value_cache, stream=stream)
         if evs is not None:
             evs[1].record(stream)
-        if run.plan is not None:     # joint + per-sequence partition kernels and the merge, one call
+        if T > 0:                    # partition kernel and merge, one call
+            pa.pa_decode_verify(q_step, run.key_cache, run.value_cache, run.block_tables, run.context_lens,
+                                w.scale, out=out_step, workspace=ws_step, stream=stream)
+            if evs is not None:
+                evs[2].record(stream)
+        elif run.plan is not None:   # joint + per-sequence partition kernels and the merge, one call
             pa.pa_decode_shared_prefix(run.q, run.key_cache, run.value_cache, run.block_tables, run.context_lens,
                                        w.scale, run.plan, out=run.out, workspace=run.workspace, stream=stream)
             if evs is not None:
@@ -550,7 +611,17 @@ def run_ours(args):
     # end to end through the API, host buffers: export tables, copy inputs in, decode, read the output back
     e2e = None
     if not args.no_e2e:
-        e2e = end_to_end(args, torch, pa, run, w, unique, max_ctx, world, dist)
+        if T > 0:
+            decode = lambda d_q, d_tab, d_ctx, d_out: pa.pa_decode_verify(
+                d_q, run.key_cache, run.value_cache, d_tab, d_ctx, w.scale, out=d_out, workspace=ws_step)
+        elif run.plan is not None:
+            decode = lambda d_q, d_tab, d_ctx, d_out: pa.pa_decode_shared_prefix(
+                d_q, run.key_cache, run.value_cache, d_tab, d_ctx, w.scale, run.plan, out=d_out,
+                workspace=run.workspace)
+        else:
+            decode = lambda d_q, d_tab, d_ctx, d_out: pa.pa_decode(
+                d_q, run.key_cache, run.value_cache, d_tab, d_ctx, w.scale, out=d_out, workspace=run.workspace)
+        e2e = end_to_end(args, torch, pa, run, w, unique, world, dist, (q_step, kd, vd, sd, out_step), decode)
 
     peak, peak_kind = measured_peak()
     achieved = part_bytes / (part_ms / 1000.0) / 1e9
@@ -559,7 +630,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(args.workload, args.cpu_seconds)
+        cpu = cpu_baseline(args.workload, args.cpu_seconds, verify_tokens=T)
 
     if rank == 0:
         cfg = describe(w)
@@ -571,34 +642,48 @@ def run_ours(args):
                     "launch": launch_mode})
         if run.plan is not None:
             cfg["joint_kernel"] = args.joint_kernel
+        if T > 0:
+            cfg["query_tokens"] = T
+            cfg["verify_path"] = f"{args.verify_path} ({'joint + per-sequence' if verify_joint else 'per-sequence'})"
+            cfg["workload"] += f"; {T} draft tokens per sequence verified per step (causal)"
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else w.dtype,
             "data": "synthetic", "config": cfg,
             "seqs_per_s": seqs_per_s,
+            **({"query_tokens_per_s": seqs_per_s * T} if T > 0 else {}),
             "eager": {"ms_per_step": eager_ms, "seqs_per_s": w.num_seqs * 1000.0 / eager_ms,
                       "note": "same steps launched one call at a time, events between the kernels"},
             "kv_bytes_per_step": {"unique": unique, "logical": logical},
             "frac_of_hbm": {"measured": value / world / peak, "nominal_8000": value / world / NOMINAL_HBM_GBS},
-            "kernel_ms": ({"reshape_and_cache": write_ms, "decode_partitions": part_ms, "decode_reduce": reduce_ms}
+            "kernel_ms": ({"reshape_and_cache": write_ms, "decode_verify (partition kernel + merge)": part_ms}
+                          if T > 0 else
+                          {"reshape_and_cache": write_ms, "decode_partitions": part_ms, "decode_reduce": reduce_ms}
                           if run.plan is None else
                           {"reshape_and_cache": write_ms, "decode_shared_prefix (joint + per-sequence + merge)": part_ms}),
             "shared_prefix_plan": (None if run.plan is None else
                                    {"chunks": run.plan["num_chunks"], "members": run.plan["num_members"],
                                     "shared_partitions": run.plan["max_shared_partitions"]}),
             "roofline": {"bound": "hbm",
-                         "kernel": ("decode_tc_kernel (pa_decode_partitions)" if run.plan is None else
+                         "kernel": (("pa_decode_verify call: plan kernel + joint tcgen05 kernel (partitions all "
+                                     "tokens see) + decode_verify_tc_kernel (the rest) + merge, timed together"
+                                     if verify_joint else
+                                     "pa_decode_verify call: decode_verify_tc_kernel + merge (timed together)")
+                                    if T > 0 else
+                                    "decode_tc_kernel (pa_decode_partitions)" if run.plan is None else
                                     "pa_decode_shared_prefix call: decode_shared_tc05p_kernel + per-sequence "
                                     "decode_tc_kernel + merge (timed together)"),
                          "achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} (copy bandwidth)",
                          "unit": "GB/s", "frac": achieved / peak,
                          # the committed counters are per launch of the Llama-3-70B-shaped batch
-                         "traffic": traffic if (args.workload == "llama70b" and run.plan is None) else None,
+                         "traffic": (traffic if (args.workload == "llama70b" and run.plan is None and T == 0)
+                                     else None),
                          "algorithmic_bytes_per_launch": part_bytes, "kernel_source_sha256": khash},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": (4 if run.plan is not None and run.plan["num_chunks"] > 0 else 3) * args.steps,
+            "gpu_launches": ((4 if run.plan is not None and run.plan["num_chunks"] > 0 else 3) if T == 0 else
+                             2 + (max_ctx > 512) + 2 * verify_joint) * args.steps,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -608,12 +693,15 @@ def run_ours(args):
     return 0
 
 
-def end_to_end(args, torch, pa, run, w, unique, max_ctx, world, dist):
-    """Same steps through the public API from pinned host buffers; wall clock, result read back each step."""
-    kd, vd, sd = run.step_write
+def end_to_end(args, torch, pa, run, w, unique, world, dist, inputs, decode):
+    """Same steps through the public API from pinned host buffers; wall clock, result read back each step.
+
+    ``inputs`` = (q, new K, new V, slots, out) of the device-resident step; ``decode(q, tables, lens, out)``
+    is its attention call."""
+    q_dev, kd, vd, sd, out_dev = inputs
     pin = dict(pin_memory=True)
-    h_q = torch.empty(run.q.shape, dtype=run.q.dtype, **pin)
-    h_q.copy_(run.q)
+    h_q = torch.empty(q_dev.shape, dtype=q_dev.dtype, **pin)
+    h_q.copy_(q_dev)
     h_k = torch.empty(kd.shape, dtype=kd.dtype, **pin)
     h_k.copy_(kd)
     h_v = torch.empty(vd.shape, dtype=vd.dtype, **pin)
@@ -622,11 +710,11 @@ def end_to_end(args, torch, pa, run, w, unique, max_ctx, world, dist):
     h_s.copy_(sd)
     h_tab = torch.empty(run.block_tables.shape, dtype=torch.int32, **pin)
     h_ctx = torch.empty(run.context_lens.shape, dtype=torch.int32, **pin)
-    h_out = torch.empty(run.out.shape, dtype=run.out.dtype, **pin)
+    h_out = torch.empty(out_dev.shape, dtype=out_dev.dtype, **pin)
     d_q, d_k, d_v, d_s = (torch.empty_like(x, device="cuda") for x in (h_q, h_k, h_v, h_s))
     d_tab = torch.empty_like(run.block_tables)
     d_ctx = torch.empty_like(run.context_lens)
-    d_out = torch.empty_like(run.out)
+    d_out = torch.empty_like(out_dev)
     seqs = list(range(w.num_seqs))
     tab_np, ctx_np = h_tab.numpy(), h_ctx.numpy()
 
@@ -635,18 +723,13 @@ def end_to_end(args, torch, pa, run, w, unique, max_ctx, world, dist):
         for dst, src in ((d_q, h_q), (d_k, h_k), (d_v, h_v), (d_s, h_s), (d_tab, h_tab), (d_ctx, h_ctx)):
             dst.copy_(src, non_blocking=True)
         pa.pa_reshape_and_cache(d_k, d_v, d_s, run.key_cache, run.value_cache)
-        if run.plan is not None:
-            pa.pa_decode_shared_prefix(d_q, run.key_cache, run.value_cache, d_tab, d_ctx, w.scale, run.plan,
-                                       out=d_out, workspace=run.workspace)
-        else:
-            pa.pa_decode(d_q, run.key_cache, run.value_cache, d_tab, d_ctx, w.scale, out=d_out,
-                         workspace=run.workspace)
+        decode(d_q, d_tab, d_ctx, d_out)
         h_out.copy_(d_out, non_blocking=True)
         torch.cuda.current_stream().synchronize()
 
     for _ in range(3):
         e2e_step()
-    if not torch.equal(h_out.view(torch.int16), run.out.cpu().view(torch.int16)):
+    if not torch.equal(h_out.view(torch.int16), out_dev.cpu().view(torch.int16)):
         raise RuntimeError("end-to-end output differs from the device-resident step")
     if world > 1:
         dist.barrier()

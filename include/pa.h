@@ -186,6 +186,59 @@ PA_API pa_status pa_decode_reduce(const int32_t* context_lens, int32_t num_seqs,
                                   const void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * pa_decode_verify -- several query tokens per sequence (checking draft
+ * tokens of speculative decoding against the paged cache in one pass).
+ *
+ * [Internals] "The Mathematical Cause of KV Cache Fragmentation" points to
+ * speculative-decoding kernels that verify parallel draft tokens across
+ * paged memory; it gives no formula.  Reading: the T = num_query_tokens
+ * query tokens of sequence b are the last T positions of its context, their
+ * K/V already written (pa_reshape_and_cache); token t sits at position
+ * pos_t = context_lens[b] - T + t and attends causally:
+ *     s_j   = scale * <q[b][t][h], K_b[j][h / G]>,   j <= pos_t
+ *     out[b][t][h] = sum_j softmax(s)_j * V_b[j][h / G]
+ * A token with pos_t < 0 (T above the context length) sees no key and gets a
+ * zero row.  T = 1 is pa_decode.
+ *
+ * q               device [num_seqs][num_query_tokens][num_q_heads][head_dim], dtype.
+ * out             device, same shape and dtype as q.
+ * workspace       device scratch of at least
+ *                 pa_decode_verify_workspace_size(num_seqs, num_query_tokens,
+ *                 num_q_heads, head_dim, max_blocks_per_seq * block_size)
+ *                 bytes, 256-byte aligned: the pa_decode partials layout
+ *                 with num_query_tokens * num_q_heads query heads per
+ *                 sequence, then room for the joint kernel's work plan
+ *                 (20 bytes per query token, each array 256-byte aligned).
+ * Everything else, including the supported sizes, the device status bits
+ * and the error returns, is as for pa_decode; in addition
+ * num_query_tokens >= 1 and num_query_tokens * num_q_heads <= 2^24.
+ * bf16 / f16 caches with block_size a multiple of 16 run on tensor cores:
+ * when T * G > 16 (head_dim 64 or 128), the partitions that all T tokens see
+ * in full go to the shared-prefix joint kernel (the T tokens of a sequence
+ * are members of one group: each page is read once for all T * G rows; the
+ * plan is built on the device from context_lens, inside the workspace), and
+ * the rest -- each sequence's last partition or two, where the causal limits
+ * fall -- to a per-sequence kernel with 8 to 32 (token, query head) rows of
+ * one kv head per CTA; f32 or other block sizes use CUDA cores.
+ * pa_set_decode_kernel, pa_set_shared_prefix_kernel and pa_set_verify_path
+ * apply.
+ * ---------------------------------------------------------------------- */
+typedef enum {
+  PA_VERIFY_AUTO = 0,          /* joint kernel for the visible partitions when T * G > 16 */
+  PA_VERIFY_PER_SEQUENCE = 1,  /* per-sequence partition kernels only */
+  PA_VERIFY_JOINT = 2          /* joint kernel whenever the call allows it; PA_ERR_UNSUPPORTED otherwise */
+} pa_verify_path;
+PA_API pa_status pa_set_verify_path(pa_verify_path path);
+PA_API size_t pa_decode_verify_workspace_size(int32_t num_seqs, int32_t num_query_tokens, int32_t num_q_heads,
+                                              int32_t head_dim, int64_t max_context_len);
+PA_API pa_status pa_decode_verify(const void* q, const void* key_cache, const void* value_cache,
+                                  const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                  const int32_t* context_lens, int32_t num_seqs, int32_t num_query_tokens,
+                                  int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                  int32_t num_blocks, float scale, void* out, pa_dtype dtype, void* workspace,
+                                  size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------
  * pa_decode_fixed_scratch -- pa_decode for callers that cannot allocate
  * device memory.  (The pages have no counterpart: this is a deployment
  * convenience of this library.)

@@ -14,7 +14,8 @@ from .allocator import PagedBlockManager
 
 
 def run(workload, with_data: bool = True, decode_seqs=None) -> dict:
-    """Execute ``workload.trace``; return allocator state, caches, slots, copy pairs and output.
+    """Execute ``workload.trace``; return allocator state (and the allocator), caches, slots, copy pairs
+    and output.
 
     ``with_data=False`` runs the allocator and slot bookkeeping only (no cache
     arrays, no attention), which is cheap even for the largest workloads.
@@ -66,7 +67,7 @@ def run(workload, with_data: bool = True, decode_seqs=None) -> dict:
                                                            w.dtype, seqs=decode_seqs)
         else:
             raise ValueError(f"unknown trace op {kind!r}")
-    result.update(state=mgr.state(), key_cache=kc, value_cache=vc, cow_pairs=all_pairs,
+    result.update(state=mgr.state(), manager=mgr, key_cache=kc, value_cache=vc, cow_pairs=all_pairs,
                   write_slots=np.concatenate(write_slots) if write_slots else np.zeros(0, np.int64),
                   append_slots=np.array(append_slots, dtype=np.int64))
     return result

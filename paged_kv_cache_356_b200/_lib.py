@@ -18,6 +18,7 @@ PA_DEV_TIMEOUT = 32
 PA_DECODE_AUTO, PA_DECODE_CUDA_CORES, PA_DECODE_TENSOR_CORES = 0, 1, 2
 PA_SHARED_PREFIX_AUTO, PA_SHARED_PREFIX_TCGEN05, PA_SHARED_PREFIX_MMA_SYNC, PA_SHARED_PREFIX_TCGEN05_SERIAL = 0, 1, 2, 3
 PA_SHARED_PREFIX_TCGEN05_2CTA = 4
+PA_VERIFY_AUTO, PA_VERIFY_PER_SEQUENCE, PA_VERIFY_JOINT = 0, 1, 2
 PA_FAULT_NONE, PA_FAULT_WITHHOLD_FIRST_ITEM = 0, 1
 PA_PARTITION_TOKENS = 512
 PA_FIXED_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -36,6 +37,10 @@ SIGNATURES = {
     "pa_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i64]),
     "pa_decode": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _i32,
                          _vp, _sz, _vp, _vp]),
+    "pa_decode_verify_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i64]),
+    "pa_set_verify_path": (_i32, [_i32]),
+    "pa_decode_verify": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
+                                _vp, _i32, _vp, _sz, _vp, _vp]),
     "pa_decode_partitions": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp,
                                     _i32, _vp, _sz, _vp, _vp]),
     "pa_decode_reduce": (_i32, [_vp, _i32, _i32, _i32, _i64, _vp, _i32, _vp, _sz, _vp]),

@@ -17,7 +17,7 @@ from . import _lib
 from ._lib import (PA_BF16, PA_DECODE_AUTO, PA_DECODE_CUDA_CORES, PA_DECODE_TENSOR_CORES,  # noqa: F401
                    PA_DEV_TIMEOUT, PA_SHARED_PREFIX_AUTO, PA_SHARED_PREFIX_MMA_SYNC, PA_SHARED_PREFIX_TCGEN05,
                    PA_SHARED_PREFIX_TCGEN05_SERIAL, PA_SHARED_PREFIX_TCGEN05_2CTA, PA_FAULT_NONE,
-                   PA_FAULT_WITHHOLD_FIRST_ITEM,
+                   PA_FAULT_WITHHOLD_FIRST_ITEM, PA_VERIFY_AUTO, PA_VERIFY_JOINT, PA_VERIFY_PER_SEQUENCE,
                    PA_DEV_BAD_CTX, PA_DEV_BAD_PAGE, PA_DEV_BAD_PAIR, PA_DEV_BAD_PLAN, PA_DEV_BAD_SLOT, PA_ERR_NOT_FOUND,
                    PA_ERR_OOM, PA_F16, PA_F32, PA_PARTITION_TOKENS)
 
@@ -186,6 +186,46 @@ def pa_decode_reduce(context_lens, max_context_len: int, out, workspace, stream=
     return out
 
 
+def pa_decode_verify_workspace_size(num_seqs: int, num_query_tokens: int, num_q_heads: int, head_dim: int,
+                                    max_context_len: int) -> int:
+    return int(_lib.load().pa_decode_verify_workspace_size(num_seqs, num_query_tokens, num_q_heads, head_dim,
+                                                           max_context_len))
+
+
+def pa_decode_verify(q, key_cache, value_cache, block_tables, context_lens, scale: float, out=None, workspace=None,
+                     dev_status=None, stream=None):
+    """Attention of T query tokens per sequence, each over the keys up to its own position.
+
+    ``q`` is [num_seqs, T, num_q_heads, head_dim]: the last T positions of each
+    context (their K/V already in the cache).  Returns ``out`` of q's shape.
+    """
+    torch = _torch()
+    nb, hkv, bs, d = _cache_shape(key_cache, value_cache)
+    if q.dim() != 4 or q.shape[3] != d or q.dtype != key_cache.dtype:
+        raise ValueError("q must be [num_seqs, num_query_tokens, num_q_heads, head_dim] of the cache dtype")
+    num_seqs, nq, hq = int(q.shape[0]), int(q.shape[1]), int(q.shape[2])
+    if block_tables.dim() != 2 or block_tables.shape[0] != num_seqs:
+        raise ValueError("block_tables must be [num_seqs, max_blocks_per_seq]")
+    if context_lens.dim() != 1 or context_lens.shape[0] != num_seqs:
+        raise ValueError("context_lens must be [num_seqs]")
+    mb = int(block_tables.shape[1])
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("out must match q")
+    need = pa_decode_verify_workspace_size(num_seqs, nq, hq, d, mb * bs)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _cuda(workspace, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.load().pa_decode_verify(
+        _cuda(q, "q"), _cuda(key_cache, "key_cache"), _cuda(value_cache, "value_cache"),
+        _cuda(block_tables, "block_tables", torch.int32), mb, _cuda(context_lens, "context_lens", torch.int32),
+        num_seqs, nq, hq, hkv, d, bs, nb, float(scale), _cuda(out, "out"), dtype_code(q.dtype), ws_ptr, ws_bytes,
+        _opt_status(dev_status), _stream_handle(stream, q.device)))
+    return out
+
+
 def pa_decode_fixed_scratch(q, key_cache, value_cache, block_tables, context_lens, scale: float, out,
                             dev_status=None, stream=None):
     """pa_decode without a workspace argument, for callers that may not allocate device memory.
@@ -238,6 +278,11 @@ def pa_set_decode_kernel(kernel: int) -> None:
 
 def pa_set_shared_prefix_kernel(kernel: int) -> None:
     _check(_lib.load().pa_set_shared_prefix_kernel(int(kernel)))
+
+
+def pa_set_verify_path(path: int) -> None:
+    """PA_VERIFY_AUTO, PA_VERIFY_PER_SEQUENCE or PA_VERIFY_JOINT (process-wide)."""
+    _check(_lib.load().pa_set_verify_path(int(path)))
 
 
 def pa_set_fault_injection(mode: int) -> None:

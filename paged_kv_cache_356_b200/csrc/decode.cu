@@ -39,6 +39,7 @@
 // per-sequence kernel covers the remaining partitions and the merge follows.
 #include <math.h>
 
+#include <algorithm>
 #include <atomic>
 #include <type_traits>
 #include <mutex>
@@ -2267,6 +2268,502 @@ __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel
 }
 
 // ---------------------------------------------------------------------------
+// Several query tokens per sequence (draft verification).  Query token t of T
+// sits at position ctx - T + t of its sequence and attends to the keys at or
+// before that position.  The rows of a kv head are its (token, query head)
+// pairs r = t * G + (h - kvh * G); q, out and the partials are indexed as if
+// the sequence had T * H_q query heads (DecodeArgs::num_q_heads holds T * H_q),
+// so the log-sum-exp merge kernel serves this path unchanged.
+// ---------------------------------------------------------------------------
+struct VerifyArgs {
+  int num_tokens;    // T
+  int q_heads;       // H_q
+  int row_groups;    // CTAs per kv head along grid y
+  int skip_visible;  // 1: the partitions every token sees in full come from the joint kernel
+};
+
+// Partitions [0, n) of a sequence that all T tokens see in full (none for a
+// one-partition sequence, whose row is written without a merge).
+__device__ __forceinline__ int verify_visible_partitions(int ctx, int num_tokens) {
+  return ctx > kPartition ? max(0, ctx - num_tokens + 1) / kPartition : 0;
+}
+
+// Work plan of the joint kernel for a verify call, from the context lengths:
+// sequence b's T tokens are T members (ids b * T + t, query rows of T * H_q
+// per sequence) reading b's table, in chunks of at most `per_chunk` tokens,
+// over its visible partitions.  chunks[b * cps + k] = (b, b * T + k * per_chunk,
+// count, visible partitions); members[i] = i.
+__global__ void verify_plan_kernel(const DecodeArgs a, int num_seqs, int num_tokens, int per_chunk, int cps,
+                                   int32_t* __restrict__ chunks, int32_t* __restrict__ members) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= num_seqs) return;
+  const int sp = verify_visible_partitions(context_of(a, b, false), num_tokens);
+  for (int k = 0; k < cps; ++k) {
+    const int first = k * per_chunk;
+    int4 c;
+    c.x = b;
+    c.y = b * num_tokens + first;
+    c.z = min(per_chunk, num_tokens - first);
+    c.w = sp;
+    reinterpret_cast<int4*>(chunks)[(int64_t)b * cps + k] = c;
+  }
+  for (int t = 0; t < num_tokens; ++t) members[(int64_t)b * num_tokens + t] = b * num_tokens + t;
+}
+
+// Row of q / out (in units of head_dim) for row r of kv head kvh of sequence b.
+__device__ __forceinline__ int64_t verify_row(const DecodeArgs& a, const VerifyArgs& v, int b, int kvh, int r) {
+  const int t = r / a.group;
+  return (int64_t)b * a.num_q_heads + (int64_t)t * v.q_heads + kvh * a.group + (r - t * a.group);
+}
+
+// Number of keys row r sees: positions 0 .. ctx - T + t.
+__device__ __forceinline__ int verify_limit(const DecodeArgs& a, const VerifyArgs& v, int ctx, int r) {
+  return max(0, ctx - v.num_tokens + 1 + r / a.group);
+}
+
+// Final rows, or the partition's partials, of rows [r0, r0 + nr) from the
+// per-warp (o, m, l) in shared memory: o_w[w * stride + j * D + d],
+// m at ml_w[w * stride + j], l at ml_w[w * stride + rows_cap + j].
+template <typename T, int D>
+__device__ __forceinline__ void verify_merge_store(const DecodeArgs& a, const VerifyArgs& v, int b, int kvh, int r0,
+                                                   int nr, int p, int np, int warps, int stride, int rows_cap,
+                                                   const float* o_w, const float* ml_w) {
+  for (int i = threadIdx.x; i < nr * D; i += blockDim.x) {
+    const int j = i / D;
+    const int d = i - j * D;
+    float mx = -INFINITY;
+    for (int w = 0; w < warps; ++w) mx = fmaxf(mx, ml_w[w * stride + j]);
+    float lsum = 0.f, osum = 0.f;
+    if (mx != -INFINITY) {
+      for (int w = 0; w < warps; ++w) {
+        const float c = exp2f(ml_w[w * stride + j] - mx);
+        lsum += ml_w[w * stride + rows_cap + j] * c;
+        osum += o_w[w * stride + j * D + d] * c;
+      }
+    }
+    const float res = lsum > 0.f ? osum / lsum : 0.f;
+    const int64_t row = verify_row(a, v, b, kvh, r0 + j);
+    if (np <= 1) {
+      reinterpret_cast<T*>(a.out)[row * D + d] = from_float<T>(res);
+    } else {
+      const int64_t part = row * a.max_partitions + p;
+      a.o_part[part * D + d] = res;
+      if (d == 0) {
+        a.m_part[part] = mx == -INFINITY ? -INFINITY : mx * kLn2;
+        a.l_part[part] = lsum;
+      }
+    }
+  }
+}
+
+template <typename T, int D>
+__device__ __forceinline__ void verify_zero_rows(const DecodeArgs& a, const VerifyArgs& v, int b, int kvh, int r0,
+                                                 int nr) {
+  for (int i = threadIdx.x; i < nr * D; i += blockDim.x) {
+    const int j = i / D;
+    reinterpret_cast<T*>(a.out)[verify_row(a, v, b, kvh, r0 + j) * D + (i - j * D)] = from_float<T>(0.f);
+  }
+}
+
+__device__ __forceinline__ void ldmatrix_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+
+// Tensor-core verify kernel.  Grid (num_seqs, num_kv_heads * row_groups, P);
+// NW warps stream their runs of 16-token tiles of the partition as in the
+// single-query kernel, with 8 * NT query rows (NT n8 MMA tiles) per CTA
+// instead of the G heads of one token.  The rows' Q sits in shared memory,
+// swizzled like the K/V tiles; a row's causal limit masks the scores of the
+// tiles it cuts (the last few tiles of the context), the others run unmasked.
+template <int D, int NW, int STAGES, int NT>
+struct VerifyShape {
+  static constexpr int kRows = 8 * NT;
+  static constexpr int kRowBytes = 2 * D;
+  static constexpr int kChunksPerRow = kRowBytes / 16;
+  static constexpr int kTile = 16;
+  static constexpr int kTileBytes = kTile * kRowBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kMergeBytes = kRows * D * 4 + 2 * kRows * 4;
+  static constexpr int kWarpBytes = STAGES * kStageBytes > kMergeBytes ? STAGES * kStageBytes : kMergeBytes;
+  static constexpr int kQBytes = kRows * kRowBytes;
+  static constexpr int kSmemBytes = kQBytes + NW * kWarpBytes;
+  static constexpr int kChunksPerLane = kTile * kChunksPerRow / 32;
+};
+
+template <typename T, int D, int NW, int STAGES, int NT>
+__global__ void __launch_bounds__(NW * 32) decode_verify_tc_kernel(const DecodeArgs a, const VerifyArgs v) {
+  const AfterPrerequisiteGrid after{threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0};
+  using S = VerifyShape<D, NW, STAGES, NT>;
+  constexpr int KSTEPS = D / 16;
+  constexpr int MTILES = D / 16;
+  extern __shared__ __align__(128) uint8_t smem[];
+
+  const int b = blockIdx.x;
+  const int kvh = blockIdx.y / v.row_groups;
+  const int r0 = (blockIdx.y - kvh * v.row_groups) * S::kRows;
+  const int nr = min(S::kRows, v.num_tokens * a.group - r0);
+  const int p = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2;
+  const int t = lane & 3;
+
+  const int ctx = context_of(a, b, threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0);
+  const int np = (ctx + kPartition - 1) / kPartition;
+  if (p >= max(np, 1)) return;
+  if (v.skip_visible && p < verify_visible_partitions(ctx, v.num_tokens)) return;
+  if (ctx == 0) {
+    verify_zero_rows<T, D>(a, v, b, kvh, r0, nr);
+    return;
+  }
+  const int bs = a.block_size;
+  const int tok_begin = p * kPartition;
+  const int tok_end = min(ctx, tok_begin + kPartition);
+  const int ntiles = (tok_end - tok_begin + S::kTile - 1) / S::kTile;
+  const int per_warp = (ntiles + NW - 1) / NW;
+  const int first_tile = warp * per_warp;
+  const int my_tiles = max(0, min(per_warp, ntiles - first_tile));
+
+  const int first_block = tok_begin / bs;
+  const int nblk = (tok_end - 1) / bs - first_block + 1;
+  int lane_page = 0;
+  if (lane < nblk) lane_page = __ldg(a.block_tables + (int64_t)b * a.max_blocks_per_seq + first_block + lane);
+
+  // Keys each of this lane's score rows (8 nt + 2 t + e) may see; padding rows see none.
+  int lim[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int row = 8 * nt + 2 * t + e;
+      lim[nt][e] = row < nr ? verify_limit(a, v, ctx, r0 + row) : 0;
+    }
+  const int lim_min = verify_limit(a, v, ctx, r0);  // smallest limit of a real row here
+
+  const uint32_t q_u32 = smem_u32(smem);
+  uint8_t* wsm = smem + S::kQBytes + warp * S::kWarpBytes;
+  const uint32_t wsm_u32 = smem_u32(wsm);
+  const T* kc = reinterpret_cast<const T*>(a.key_cache);
+  const T* vc = reinterpret_cast<const T*>(a.value_cache);
+
+  // The CTA's Q rows (zeros for padding rows): the oldest cp.async group.
+  for (int i = threadIdx.x; i < S::kRows * S::kChunksPerRow; i += NW * 32) {
+    const int r = i / S::kChunksPerRow;
+    const int c = i - r * S::kChunksPerRow;
+    const bool ok = r < nr;
+    const T* src = reinterpret_cast<const T*>(a.q) + (ok ? verify_row(a, v, b, kvh, r0 + r) : 0) * D + c * 8;
+    cp_async_16(q_u32 + r * S::kRowBytes + ((c ^ (r & 7)) << 4), src, ok ? 16u : 0u);
+  }
+  cp_async_commit();
+
+  auto load_tile = [&](int i, int stage) {
+    const int tok0 = tok_begin + (first_tile + i) * S::kTile;
+    int valid = min(S::kTile, tok_end - tok0);
+    int page = __shfl_sync(kFull, lane_page, tok0 / bs - first_block);
+    if ((unsigned)page >= (unsigned)a.num_blocks) {
+      if (lane == 0) flag_status(a.status, PA_DEV_BAD_PAGE);
+      valid = 0;
+      page = 0;
+    }
+    const int64_t row0 = ((int64_t)page * a.num_kv_heads + kvh) * bs + (tok0 % bs);
+    const T* ksrc = kc + row0 * D;
+    const T* vsrc = vc + row0 * D;
+    const uint32_t kdst = wsm_u32 + stage * S::kStageBytes;
+    const uint32_t vdst = kdst + S::kTileBytes;
+#pragma unroll
+    for (int j = 0; j < S::kChunksPerLane; ++j) {
+      const int idx = lane + 32 * j;
+      const int r = idx / S::kChunksPerRow;
+      const int c = idx - r * S::kChunksPerRow;
+      const bool ok = r < valid;
+      const int64_t src = (int64_t)(ok ? r : 0) * D + c * 8;
+      const uint32_t dst = r * S::kRowBytes + ((c ^ (r & 7)) << 4);
+      cp_async_16(kdst + dst, ksrc + src, ok ? 16u : 0u);
+      cp_async_16(vdst + dst, vsrc + src, ok ? 16u : 0u);
+    }
+  };
+
+  float o[NT][MTILES][4];
+  float m[NT][2], l[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int mt = 0; mt < MTILES; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+    m[nt][0] = m[nt][1] = -INFINITY;
+    l[nt][0] = l[nt][1] = 0.f;
+  }
+
+#pragma unroll
+  for (int i = 0; i < STAGES - 1; ++i) {
+    if (i < my_tiles) load_tile(i, i);
+    cp_async_commit();
+  }
+  cp_async_wait<STAGES - 1>();  // the Q group
+  __syncthreads();
+
+  for (int i = 0; i < my_tiles; ++i) {
+    {
+      const int nxt = i + STAGES - 1;
+      if (nxt < my_tiles) load_tile(nxt, nxt % STAGES);
+      cp_async_commit();
+    }
+    cp_async_wait<STAGES - 1>();
+    __syncwarp();
+
+    const int stage = i % STAGES;
+    const uint32_t kbase = wsm_u32 + stage * S::kStageBytes;
+    const uint32_t vbase = kbase + S::kTileBytes;
+    const int tok0 = tok_begin + (first_tile + i) * S::kTile;
+    int valid = min(S::kTile, tok_end - tok0);
+    {
+      const int page = __shfl_sync(kFull, lane_page, tok0 / bs - first_block);
+      if ((unsigned)page >= (unsigned)a.num_blocks) valid = 0;
+    }
+
+    // S^T = K_tile . Q^T, one n8 tile of rows at a time.
+    float s[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+    {
+      const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
+      const uint32_t rbase = kbase + r * S::kRowBytes;
+      const int qr = lane & 7;
+#pragma unroll
+      for (int ks = 0; ks < KSTEPS; ++ks) {
+        const int c = 2 * ks + (lane >> 4);
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(rbase + ((c ^ (r & 7)) << 4), a0, a1, a2, a3);
+        if constexpr (NT == 1) {
+          uint32_t b0, b1;
+          const int qc = 2 * ks + ((lane >> 3) & 1);
+          ldmatrix_x2(q_u32 + qr * S::kRowBytes + ((qc ^ qr) << 4), b0, b1);
+          mma_16816<T>(s[0], a0, a1, a2, a3, b0, b1);
+        } else {
+#pragma unroll
+          for (int nt = 0; nt < NT; nt += 2) {
+            // Matrices: rows of tile nt (chunks 2ks, 2ks+1), then of tile nt + 1.
+            const int qrow = 8 * (nt + (lane >> 4)) + qr;
+            const int qc = 2 * ks + ((lane >> 3) & 1);
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4(q_u32 + qrow * S::kRowBytes + ((qc ^ qr) << 4), b0, b1, b2, b3);
+            mma_16816<T>(s[nt], a0, a1, a2, a3, b0, b1);
+            mma_16816<T>(s[nt + 1], a0, a1, a2, a3, b2, b3);
+          }
+        }
+      }
+    }
+    // s[nt][0..1]: token g, rows 8 nt + 2t, 2t + 1; s[nt][2..3]: token g + 8.
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[nt][e] *= a.qk_scale_log2;
+    if (tok0 + S::kTile > lim_min || valid < S::kTile) {
+      const int cut = tok0 + valid;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int lm = min(lim[nt][e], cut);
+          if (tok0 + g >= lm) s[nt][e] = -INFINITY;
+          if (tok0 + g + 8 >= lm) s[nt][2 + e] = -INFINITY;
+        }
+    }
+
+    uint32_t pb[NT][2], pl[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float pr[4], alpha[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float mx = fmaxf(s[nt][j], s[nt][2 + j]);
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+        const float mn = fmaxf(m[nt][j], mx);
+        const float base = mn == -INFINITY ? 0.f : mn;
+        alpha[j] = exp2f(m[nt][j] - base);
+        pr[j] = exp2f(s[nt][j] - base);
+        pr[2 + j] = exp2f(s[nt][2 + j] - base);
+        l[nt][j] = l[nt][j] * alpha[j] + pr[j] + pr[2 + j];
+        m[nt][j] = mn;
+      }
+#pragma unroll
+      for (int mt = 0; mt < MTILES; ++mt) {
+        o[nt][mt][0] *= alpha[0];
+        o[nt][mt][1] *= alpha[1];
+        o[nt][mt][2] *= alpha[0];
+        o[nt][mt][3] *= alpha[1];
+      }
+      // P^T as the B operand, a 16-bit high part plus the rounding residual.
+      const uint32_t hi0 = pack2<T>(pr[0], pr[1]);
+      const uint32_t hi1 = pack2<T>(pr[2], pr[3]);
+      const float2 q0 = unpack2<T>(hi0), q1 = unpack2<T>(hi1);
+      pb[nt][0] = movmatrix_trans(hi0);
+      pb[nt][1] = movmatrix_trans(hi1);
+      pl[nt][0] = movmatrix_trans(pack2<T>(pr[0] - q0.x, pr[1] - q0.y));
+      pl[nt][1] = movmatrix_trans(pack2<T>(pr[2] - q1.x, pr[3] - q1.y));
+    }
+
+    // O^T += V_tile^T . P^T for every row tile, one m16 tile of head_dim at a time.
+    {
+      const int mat = lane >> 3;
+      const int r = (lane & 7) + ((mat >> 1) << 3);
+      const uint32_t rbase = vbase + r * S::kRowBytes;
+#pragma unroll
+      for (int mt = 0; mt < MTILES; ++mt) {
+        const int c = 2 * mt + (mat & 1);
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4_trans(rbase + ((c ^ (r & 7)) << 4), a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          mma_16816<T>(o[nt][mt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+          mma_16816<T>(o[nt][mt], a0, a1, a2, a3, pl[nt][0], pl[nt][1]);
+        }
+      }
+    }
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+  __syncwarp();
+
+  // Warp partials into this warp's region: o[kRows][D], then m[kRows], l[kRows].
+  float* o_w = reinterpret_cast<float*>(wsm);
+  float* ml_w = o_w + S::kRows * D;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      l[nt][j] += __shfl_xor_sync(kFull, l[nt][j], 4);
+      l[nt][j] += __shfl_xor_sync(kFull, l[nt][j], 8);
+      l[nt][j] += __shfl_xor_sync(kFull, l[nt][j], 16);
+    }
+    const int rr = 8 * nt + 2 * t;
+#pragma unroll
+    for (int mt = 0; mt < MTILES; ++mt) {
+      const int d = 16 * mt + g;
+      o_w[rr * D + d] = o[nt][mt][0];
+      o_w[(rr + 1) * D + d] = o[nt][mt][1];
+      o_w[rr * D + d + 8] = o[nt][mt][2];
+      o_w[(rr + 1) * D + d + 8] = o[nt][mt][3];
+    }
+    if (g == 0) {
+      ml_w[rr] = m[nt][0];
+      ml_w[rr + 1] = m[nt][1];
+      ml_w[S::kRows + rr] = l[nt][0];
+      ml_w[S::kRows + rr + 1] = l[nt][1];
+    }
+  }
+  __syncthreads();
+  const float* base_f = reinterpret_cast<const float*>(smem + S::kQBytes);
+  verify_merge_store<T, D>(a, v, b, kvh, r0, nr, p, np, NW, S::kWarpBytes / 4, S::kRows, base_f,
+                           base_f + S::kRows * D);
+}
+
+// CUDA-core verify kernel (fp32, or block sizes off the 16-token tile).
+// Grid (num_seqs, num_kv_heads * row_groups, P); a CTA serves GC rows.
+template <typename T, int D, int GC, int NW>
+__global__ void __launch_bounds__(NW * 32) decode_verify_cc_kernel(const DecodeArgs a, const VerifyArgs v) {
+  constexpr int VPL = D / 32;
+  constexpr int kStride = GC * D + 2 * GC;
+  __shared__ float w_s[NW * kStride];
+
+  const int b = blockIdx.x;
+  const int kvh = blockIdx.y / v.row_groups;
+  const int r0 = (blockIdx.y - kvh * v.row_groups) * GC;
+  const int nr = min(GC, v.num_tokens * a.group - r0);
+  const int p = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int ctx = context_of(a, b, threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0);
+  const int np = (ctx + kPartition - 1) / kPartition;
+  if (p >= max(np, 1)) return;
+  if (ctx == 0) {
+    verify_zero_rows<T, D>(a, v, b, kvh, r0, nr);
+    return;
+  }
+  const int tok_begin = p * kPartition;
+  const int tok_end = min(ctx, tok_begin + kPartition);
+
+  float qv[GC][VPL];
+  int lim[GC];
+#pragma unroll
+  for (int j = 0; j < GC; ++j) {
+    lim[j] = j < nr ? verify_limit(a, v, ctx, r0 + j) : 0;
+    if (j < nr) {
+      load_floats<T, VPL>(reinterpret_cast<const T*>(a.q) + verify_row(a, v, b, kvh, r0 + j) * D + lane * VPL,
+                          qv[j]);
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) qv[j][i] *= a.qk_scale_log2;
+    } else {
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) qv[j][i] = 0.f;
+    }
+  }
+  float m[GC], l[GC], o[GC][VPL];
+#pragma unroll
+  for (int j = 0; j < GC; ++j) {
+    m[j] = -INFINITY;
+    l[j] = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) o[j][i] = 0.f;
+  }
+
+  const T* kc = reinterpret_cast<const T*>(a.key_cache);
+  const T* vc = reinterpret_cast<const T*>(a.value_cache);
+  const int32_t* table = a.block_tables + (int64_t)b * a.max_blocks_per_seq;
+  for (int tok = tok_begin + warp; tok < tok_end; tok += NW) {
+    const int page = __ldg(table + tok / a.block_size);
+    if ((unsigned)page >= (unsigned)a.num_blocks) {
+      if (lane == 0) flag_status(a.status, PA_DEV_BAD_PAGE);
+      continue;
+    }
+    const int64_t row =
+        (((int64_t)page * a.num_kv_heads + kvh) * a.block_size + tok % a.block_size) * D + lane * VPL;
+    float kf[VPL], vf[VPL];
+    load_floats<T, VPL>(kc + row, kf);
+    load_floats<T, VPL>(vc + row, vf);
+    float s[GC];
+#pragma unroll
+    for (int j = 0; j < GC; ++j) {
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) acc = fmaf(qv[j][i], kf[i], acc);
+      s[j] = acc;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+      for (int j = 0; j < GC; ++j) s[j] += __shfl_xor_sync(kFull, s[j], off);
+    }
+#pragma unroll
+    for (int j = 0; j < GC; ++j) {
+      if (tok >= lim[j]) continue;  // after this row's position (uniform across the warp)
+      const float mn = fmaxf(m[j], s[j]);
+      const float alpha = exp2f(m[j] - mn);
+      const float pr = exp2f(s[j] - mn);
+      l[j] = l[j] * alpha + pr;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) o[j][i] = fmaf(pr, vf[i], o[j][i] * alpha);
+      m[j] = mn;
+    }
+  }
+
+  float* mine = w_s + warp * kStride;
+#pragma unroll
+  for (int j = 0; j < GC; ++j) {
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) mine[j * D + lane * VPL + i] = o[j][i];
+    if (lane == 0) {
+      mine[GC * D + j] = m[j];
+      mine[GC * D + GC + j] = l[j];
+    }
+  }
+  __syncthreads();
+  verify_merge_store<T, D>(a, v, b, kvh, r0, nr, p, np, NW, kStride, GC, w_s, w_s + GC * D);
+}
+
+// ---------------------------------------------------------------------------
 // Host side.
 // ---------------------------------------------------------------------------
 std::atomic<int> g_kernel_choice{PA_DECODE_AUTO};
@@ -2548,6 +3045,79 @@ cudaError_t launch_reduce(const DecodeArgs& a, int head_dim, int num_seqs, cudaS
   return cudaErrorInvalidValue;
 }
 
+// `v.skip_visible`: launched as a programmatic dependent of the joint kernel,
+// which covers the partitions every token sees in full.
+template <typename T, int D, int NW, int STAGES, int NT>
+cudaError_t launch_verify_tc(const DecodeArgs& a, VerifyArgs v, int num_seqs, int partitions, cudaStream_t stream) {
+  using S = VerifyShape<D, NW, STAGES, NT>;
+  static std::atomic<uint64_t> done{0};
+  auto kernel = decode_verify_tc_kernel<T, D, NW, STAGES, NT>;
+  cudaError_t err = ensure_smem(kernel, S::kSmemBytes, done);
+  if (err != cudaSuccess) return err;
+  v.row_groups = (v.num_tokens * a.group + S::kRows - 1) / S::kRows;
+  if ((int64_t)a.num_kv_heads * v.row_groups > 65535) return cudaErrorInvalidValue;
+  const dim3 grid(num_seqs, a.num_kv_heads * v.row_groups, partitions);
+  if (!v.skip_visible) {
+    kernel<<<grid, NW * 32, S::kSmemBytes, stream>>>(a, v);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(NW * 32);
+  cfg.dynamicSmemBytes = S::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a, v);
+}
+
+// Rows per CTA: the fewest n8 tiles that hold a kv head's T * G rows, at most
+// 4 (2 at head_dim 256, where the accumulators of more would spill); larger
+// row counts take several CTAs per kv head, which read the same pages, mostly
+// from L2.
+template <typename T, int D>
+cudaError_t launch_verify_tc_dim(const DecodeArgs& a, const VerifyArgs& v, int num_seqs, int partitions,
+                                 cudaStream_t stream) {
+  const int rows = v.num_tokens * a.group;
+  if constexpr (D == 256) {
+    if (rows <= 8) return launch_verify_tc<T, D, 4, 2, 1>(a, v, num_seqs, partitions, stream);
+    return launch_verify_tc<T, D, 4, 2, 2>(a, v, num_seqs, partitions, stream);
+  } else {
+    if (rows <= 8) return launch_verify_tc<T, D, 4, 3, 1>(a, v, num_seqs, partitions, stream);
+    if (rows <= 16) return launch_verify_tc<T, D, 4, 3, 2>(a, v, num_seqs, partitions, stream);
+    return launch_verify_tc<T, D, 4, 3, 4>(a, v, num_seqs, partitions, stream);
+  }
+}
+
+template <typename T>
+cudaError_t launch_verify_cc(const DecodeArgs& a, VerifyArgs v, int head_dim, int num_seqs, int partitions,
+                             cudaStream_t stream) {
+  v.row_groups = (v.num_tokens * a.group + kCcHeads - 1) / kCcHeads;
+  if ((int64_t)a.num_kv_heads * v.row_groups > 65535) return cudaErrorInvalidValue;
+  const dim3 grid(num_seqs, a.num_kv_heads * v.row_groups, partitions);
+  switch (head_dim) {
+    case 64: decode_verify_cc_kernel<T, 64, kCcHeads, kCcWarps><<<grid, kCcWarps * 32, 0, stream>>>(a, v); break;
+    case 128: decode_verify_cc_kernel<T, 128, kCcHeads, kCcWarps><<<grid, kCcWarps * 32, 0, stream>>>(a, v); break;
+    case 256: decode_verify_cc_kernel<T, 256, kCcHeads, kCcWarps><<<grid, kCcWarps * 32, 0, stream>>>(a, v); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_verify_tc_any(const DecodeArgs& a, const VerifyArgs& v, int head_dim, int num_seqs,
+                                 int partitions, cudaStream_t stream) {
+  switch (head_dim) {
+    case 64: return launch_verify_tc_dim<T, 64>(a, v, num_seqs, partitions, stream);
+    case 128: return launch_verify_tc_dim<T, 128>(a, v, num_seqs, partitions, stream);
+    case 256: return launch_verify_tc_dim<T, 256>(a, v, num_seqs, partitions, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
 bool tc_supported(pa_dtype dt, int head_dim, int group, int block_size) {
   return (dt == PA_BF16 || dt == PA_F16) && (head_dim == 64 || head_dim == 128 || head_dim == 256) &&
          group >= 1 && group <= 8 && block_size % 16 == 0 && block_size <= 256;
@@ -2750,6 +3320,128 @@ extern "C" pa_status pa_decode_reduce(const int32_t* context_lens, int32_t num_s
   a.m_part = reinterpret_cast<float*>(ws + w.m_off);
   a.l_part = reinterpret_cast<float*>(ws + w.l_off);
   return launch_reduce_any(a, dtype, head_dim, num_seqs, static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------------------
+// pa_decode_verify: T query tokens per sequence, each attending causally.
+// ---------------------------------------------------------------------------
+namespace {
+std::atomic<int> g_verify_path{PA_VERIFY_AUTO};
+
+// Above this many rows (T * G) per kv head the joint kernel takes the visible partitions (at 16
+// rows the per-sequence kernel alone is still faster).
+constexpr int kVerifyJointRows = 16;
+
+// The partials (the pa_decode layout with T * H_q heads), then the joint kernel's plan:
+// chunks int32 [num_seqs * T][4] at most, members int32 [num_seqs * T].
+struct VerifyLayout {
+  WorkspaceLayout parts;
+  size_t chunks_off, members_off, total;
+};
+
+VerifyLayout verify_layout(int64_t num_seqs, int64_t num_tokens, int64_t num_q_heads, int64_t head_dim,
+                           int64_t partitions) {
+  VerifyLayout v;
+  v.parts = workspace_layout(num_seqs, num_tokens * num_q_heads, head_dim, partitions);
+  v.chunks_off = v.parts.total;
+  v.members_off = v.chunks_off + align256((size_t)num_seqs * num_tokens * 16);
+  v.total = v.members_off + align256((size_t)num_seqs * num_tokens * 4);
+  return v;
+}
+}  // namespace
+
+extern "C" pa_status pa_set_verify_path(pa_verify_path path) {
+  if (path < PA_VERIFY_AUTO || path > PA_VERIFY_JOINT) return fail(PA_ERR_INVALID, "unknown verify path %d", (int)path);
+  g_verify_path.store(path);
+  return PA_OK;
+}
+
+extern "C" size_t pa_decode_verify_workspace_size(int32_t num_seqs, int32_t num_query_tokens, int32_t num_q_heads,
+                                                  int32_t head_dim, int64_t max_context_len) {
+  if (num_seqs <= 0 || num_query_tokens <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0 ||
+      (int64_t)num_query_tokens * num_q_heads > (1 << 24))
+    return 0;
+  const int64_t partitions = (max_context_len + kPartition - 1) / kPartition;
+  if (partitions <= 1) return 0;
+  return verify_layout(num_seqs, num_query_tokens, num_q_heads, head_dim, partitions).total;
+}
+
+extern "C" pa_status pa_decode_verify(const void* q, const void* key_cache, const void* value_cache,
+                                      const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                      const int32_t* context_lens, int32_t num_seqs, int32_t num_query_tokens,
+                                      int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                      int32_t block_size, int32_t num_blocks, float scale, void* out,
+                                      pa_dtype dtype, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                      void* stream) {
+  if (num_query_tokens < 1) return fail(PA_ERR_INVALID, "decode_verify: num_query_tokens %d", num_query_tokens);
+  if (num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0)
+    return fail(PA_ERR_INVALID, "decode_verify: num_q_heads must be a positive multiple of num_kv_heads");
+  if ((int64_t)num_query_tokens * num_q_heads > (1 << 24))
+    return fail(PA_ERR_UNSUPPORTED, "decode_verify: num_query_tokens * num_q_heads above 2^24");
+  // q, out and the partials are laid out as T * H_q query heads per sequence.
+  DecodeArgs a;
+  int partitions = 0;
+  pa_status st = prepare_decode(q, key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                                num_query_tokens * num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                                scale, out, dtype, workspace, workspace_bytes, dev_status, a, partitions);
+  if (st != PA_OK || num_seqs == 0) return st;
+  const int G = num_q_heads / num_kv_heads;
+  a.group = G;
+  VerifyArgs v{num_query_tokens, num_q_heads, 0, 0};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int choice = g_kernel_choice.load();
+  const bool tc_ok = (dtype == PA_BF16 || dtype == PA_F16) && block_size % 16 == 0 && block_size <= 256;
+  if (choice == PA_DECODE_TENSOR_CORES && !tc_ok)
+    return fail(PA_ERR_UNSUPPORTED, "decode_verify: tensor-core kernel needs bf16/f16 and block_size %% 16 == 0");
+  cudaError_t err;
+
+  // The partitions all T tokens see in full are a shared prefix of T members:
+  // the joint kernel reads each of their pages once for all T * G rows.
+  const int path = g_verify_path.load();
+  const int per_chunk = G <= PA_PREFIX_QUERIES_PER_CTA ? std::min(num_query_tokens, PA_PREFIX_QUERIES_PER_CTA / G) : 0;
+  const int max_visible = (int)std::min<int64_t>((int64_t)max_blocks_per_seq * block_size / kPartition, partitions);
+  const bool joint_ok = tc_ok && choice != PA_DECODE_CUDA_CORES && (head_dim == 64 || head_dim == 128) &&
+                        partitions > 1 && per_chunk > 0 && max_visible > 0 &&
+                        (int64_t)num_seqs * num_query_tokens <= (1 << 26);
+  if (path == PA_VERIFY_JOINT && !joint_ok)
+    return fail(PA_ERR_UNSUPPORTED, "decode_verify: the joint path needs bf16/f16, head_dim 64 or 128, block_size "
+                                    "%% 16 == 0, G <= %d and contexts beyond one partition", PA_PREFIX_QUERIES_PER_CTA);
+  const bool joint = joint_ok && (path == PA_VERIFY_JOINT ||
+                                  (path == PA_VERIFY_AUTO && (int64_t)num_query_tokens * G > kVerifyJointRows));
+  if (joint) {
+    const VerifyLayout lay = verify_layout(num_seqs, num_query_tokens, num_q_heads, head_dim, partitions);
+    if (workspace_bytes < lay.total)
+      return fail(PA_ERR_INVALID, "decode_verify: workspace of %zu bytes needed, %zu given", lay.total,
+                  workspace_bytes);
+    int32_t* chunks = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.chunks_off);
+    int32_t* members = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.members_off);
+    const int cps = (num_query_tokens + per_chunk - 1) / per_chunk;
+    const int num_members = num_seqs * num_query_tokens;
+    verify_plan_kernel<<<(num_seqs + 127) / 128, 128, 0, s>>>(a, num_seqs, num_query_tokens, per_chunk, cps, chunks,
+                                                                members);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode_verify plan kernel: %s", cudaGetErrorString(err));
+    // The joint kernel indexes q, the partials and its members with H_q heads per member.
+    DecodeArgs aj = a;
+    aj.num_q_heads = num_q_heads;
+    const dim3 grid(num_seqs * cps, num_kv_heads, max_visible);
+    err = dtype == PA_BF16 ? launch_shared_dim<__nv_bfloat16>(aj, head_dim, grid, chunks, members, num_members,
+                                                              num_members, dtype, s)
+                           : launch_shared_dim<__half>(aj, head_dim, grid, chunks, members, num_members, num_members,
+                                                       dtype, s);
+    if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode_verify joint kernel: %s", cudaGetErrorString(err));
+    v.skip_visible = 1;
+  }
+  if (tc_ok && choice != PA_DECODE_CUDA_CORES)
+    err = dtype == PA_BF16 ? launch_verify_tc_any<__nv_bfloat16>(a, v, head_dim, num_seqs, partitions, s)
+                           : launch_verify_tc_any<__half>(a, v, head_dim, num_seqs, partitions, s);
+  else
+    err = dtype == PA_F32    ? launch_verify_cc<float>(a, v, head_dim, num_seqs, partitions, s)
+          : dtype == PA_BF16 ? launch_verify_cc<__nv_bfloat16>(a, v, head_dim, num_seqs, partitions, s)
+                             : launch_verify_cc<__half>(a, v, head_dim, num_seqs, partitions, s);
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode_verify partition kernel: %s", cudaGetErrorString(err));
+  if (partitions <= 1) return PA_OK;
+  return launch_reduce_any(a, dtype, head_dim, num_seqs, s);
 }
 
 // ---------------------------------------------------------------------------

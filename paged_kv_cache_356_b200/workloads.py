@@ -46,6 +46,7 @@ _TAG_LENGTHS = 1
 _TAG_POOL = 2
 _TAG_QUERY = 3
 _TAG_KV = 4
+_TAG_DRAFT = 5
 
 _BF16_NORMAL_TABLE = None
 
@@ -148,6 +149,20 @@ class Workload:
         k = normal_values(rng, n, self.dtype).reshape(count, self.num_kv_heads, self.head_dim)
         v = normal_values(rng, n, self.dtype).reshape(count, self.num_kv_heads, self.head_dim)
         return k, v
+
+    def draft_query(self, num_tokens: int) -> np.ndarray:
+        """q of a draft-verification step, [num_seqs, num_tokens, num_q_heads, head_dim]."""
+        n = self.num_seqs * num_tokens * self.num_q_heads * self.head_dim
+        vals = normal_values(_rng(self.seed, _TAG_DRAFT, num_tokens, 0), n, self.dtype)
+        return vals.reshape(self.num_seqs, num_tokens, self.num_q_heads, self.head_dim)
+
+    def draft_kv(self, num_tokens: int) -> Tuple[np.ndarray, np.ndarray]:
+        """K and V of the draft tokens, stored at the last ``num_tokens`` positions of each
+        sequence before the verification step: [num_seqs * num_tokens, Hkv, D] each, sequence-major."""
+        n = self.num_seqs * num_tokens * self.num_kv_heads * self.head_dim
+        rng = _rng(self.seed, _TAG_DRAFT, num_tokens, 1)
+        shape = (self.num_seqs * num_tokens, self.num_kv_heads, self.head_dim)
+        return normal_values(rng, n, self.dtype).reshape(shape), normal_values(rng, n, self.dtype).reshape(shape)
 
     def writes(self) -> List[tuple]:
         return [op for op in self.trace if op[0] == "write"]
