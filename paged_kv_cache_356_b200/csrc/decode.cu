@@ -2402,7 +2402,6 @@ __global__ void __launch_bounds__(NW * 32) decode_verify_tc_kernel(const DecodeA
   const int kvh = blockIdx.y / v.row_groups;
   const int r0 = (blockIdx.y - kvh * v.row_groups) * S::kRows;
   const int nr = min(S::kRows, v.num_tokens * a.group - r0);
-  const int p = blockIdx.z;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2;
@@ -2410,8 +2409,9 @@ __global__ void __launch_bounds__(NW * 32) decode_verify_tc_kernel(const DecodeA
 
   const int ctx = context_of(a, b, threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0);
   const int np = (ctx + kPartition - 1) / kPartition;
+  // With the joint kernel on the partitions every token sees, grid z counts the ones after them.
+  const int p = blockIdx.z + (v.skip_visible ? verify_visible_partitions(ctx, v.num_tokens) : 0);
   if (p >= max(np, 1)) return;
-  if (v.skip_visible && p < verify_visible_partitions(ctx, v.num_tokens)) return;
   if (ctx == 0) {
     verify_zero_rows<T, D>(a, v, b, kvh, r0, nr);
     return;
@@ -2569,30 +2569,52 @@ __global__ void __launch_bounds__(NW * 32) decode_verify_tc_kernel(const DecodeA
         }
     }
 
-    uint32_t pb[NT][2], pl[NT][2];
+    // Each row's reference m (base 2) is raised only when a score passes it by more than 8, so
+    // the weights stay below 2^8 and O is rescaled rarely; the partials store that reference.
+    float tmax[NT][2];
+    bool raise = false;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      float pr[4], alpha[2];
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         float mx = fmaxf(s[nt][j], s[nt][2 + j]);
         mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
         mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
         mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-        const float mn = fmaxf(m[nt][j], mx);
-        const float base = mn == -INFINITY ? 0.f : mn;
-        alpha[j] = exp2f(m[nt][j] - base);
-        pr[j] = exp2f(s[nt][j] - base);
-        pr[2 + j] = exp2f(s[nt][2 + j] - base);
-        l[nt][j] = l[nt][j] * alpha[j] + pr[j] + pr[2 + j];
-        m[nt][j] = mn;
+        tmax[nt][j] = mx;
+        raise |= mx > m[nt][j] + 8.f;
       }
+    if (__any_sync(kFull, raise)) {
 #pragma unroll
-      for (int mt = 0; mt < MTILES; ++mt) {
-        o[nt][mt][0] *= alpha[0];
-        o[nt][mt][1] *= alpha[1];
-        o[nt][mt][2] *= alpha[0];
-        o[nt][mt][3] *= alpha[1];
+      for (int nt = 0; nt < NT; ++nt) {
+        float alpha[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float mn = fmaxf(m[nt][j], tmax[nt][j]);
+          alpha[j] = ex2_approx(m[nt][j] - (mn == -INFINITY ? 0.f : mn));
+          l[nt][j] *= alpha[j];
+          m[nt][j] = mn;
+        }
+#pragma unroll
+        for (int mt = 0; mt < MTILES; ++mt) {
+          o[nt][mt][0] *= alpha[0];
+          o[nt][mt][1] *= alpha[1];
+          o[nt][mt][2] *= alpha[0];
+          o[nt][mt][3] *= alpha[1];
+        }
+      }
+    }
+
+    uint32_t pb[NT][2], pl[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float pr[4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const float base = m[nt][j] == -INFINITY ? 0.f : m[nt][j];
+        pr[j] = ex2_approx(s[nt][j] - base);
+        pr[2 + j] = ex2_approx(s[nt][2 + j] - base);
+        l[nt][j] += pr[j] + pr[2 + j];
       }
       // P^T as the B operand, a 16-bit high part plus the rounding residual.
       const uint32_t hi0 = pack2<T>(pr[0], pr[1]);
@@ -3056,7 +3078,10 @@ cudaError_t launch_verify_tc(const DecodeArgs& a, VerifyArgs v, int num_seqs, in
   if (err != cudaSuccess) return err;
   v.row_groups = (v.num_tokens * a.group + S::kRows - 1) / S::kRows;
   if ((int64_t)a.num_kv_heads * v.row_groups > 65535) return cudaErrorInvalidValue;
-  const dim3 grid(num_seqs, a.num_kv_heads * v.row_groups, partitions);
+  // After the visible partitions a sequence has at most 1 + ceil((T - 1) / 512) left.
+  const int tail = 1 + (v.num_tokens - 1 + kPartition - 1) / kPartition;
+  const dim3 grid(num_seqs, a.num_kv_heads * v.row_groups,
+                  v.skip_visible ? std::min(partitions, tail) : partitions);
   if (!v.skip_visible) {
     kernel<<<grid, NW * 32, S::kSmemBytes, stream>>>(a, v);
     return cudaGetLastError();
