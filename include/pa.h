@@ -455,6 +455,34 @@ PA_API pa_status pa_block_alloc_prefix_plan(const pa_block_alloc* a, const int64
 PA_API pa_status pa_block_alloc_free_pool(const pa_block_alloc* a, int32_t* out, int32_t cap,
                                    int32_t* n_out);
 
+/* Occupancy and internal fragmentation of the pool.
+ * [Internals] "The Mathematical Cause of KV Cache Fragmentation": internal
+ * fragmentation is reserved memory that holds no token; under paging only
+ * the unwritten slots of held pages are wasted.  A page shared by several
+ * sequences is one physical page; its filled slots are the most any holder
+ * has stored in it.  [Internals] "Architectural Recommendations for
+ * Infrastructure Engineers", item 3: alert when free pages fall below 10
+ * percent of the pool (PA_LOW_FREE_FRACTION; any threshold may be passed). */
+#define PA_LOW_FREE_FRACTION 0.10
+typedef struct {
+  int32_t num_blocks;
+  int32_t block_size;
+  int32_t free_pages;       /* pages in the free pool */
+  int32_t used_pages;       /* pages with a reference count >= 1 */
+  int32_t shared_pages;     /* pages with a reference count >= 2 */
+  int32_t num_sequences;
+  int64_t logical_tokens;   /* sum of the sequences' token counts (a shared token once per holder) */
+  int64_t physical_tokens;  /* slots of used pages that hold a token (a shared page once) */
+  int64_t waste_slots;      /* used_pages * block_size - physical_tokens */
+  double waste_fraction;    /* waste_slots / (used_pages * block_size); 0 with no used page */
+  double free_fraction;     /* free_pages / num_blocks; 0 for an empty pool */
+  int32_t low_free_alarm;   /* 1 if num_blocks > 0 and free_fraction < alarm_free_fraction */
+  int32_t reserved0;        /* 0 */
+} pa_pool_stats;
+
+/* Fills *out (host).  O(pages held); PA_ERR_INVALID on a NULL argument. */
+PA_API pa_status pa_block_alloc_stats(const pa_block_alloc* a, double alarm_free_fraction, pa_pool_stats* out);
+
 #ifdef __cplusplus
 }
 #endif

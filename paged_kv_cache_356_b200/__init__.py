@@ -12,9 +12,9 @@ from .binding import (BlockAllocator, PagedAttentionError, PagedAttentionOOM, Se
                       pa_block_alloc_block_tables, pa_block_alloc_create, pa_block_alloc_destroy,
                       pa_block_alloc_fork, pa_block_alloc_free_pool, pa_block_alloc_free_sequence,
                       pa_block_alloc_num_free, pa_block_alloc_num_sequences, pa_block_alloc_num_tokens,
-                      pa_block_alloc_ref_count, pa_block_alloc_slot_mapping, pa_copy_blocks, pa_decode,
-                      pa_decode_fixed_scratch, pa_decode_partitions, pa_decode_reduce, pa_decode_verify,
-                      pa_decode_verify_workspace_size,
-                      pa_decode_shared_prefix, pa_block_alloc_prefix_plan, prefix_plan_to_device,
-                      pa_decode_workspace_size, pa_reshape_and_cache, pa_set_decode_kernel,
-                      pa_set_decode_tiling, pa_set_shared_prefix_kernel, pa_set_verify_path, pa_version)
+                      pa_block_alloc_prefix_plan, pa_block_alloc_ref_count, pa_block_alloc_slot_mapping,
+                      pa_block_alloc_stats, pa_copy_blocks, pa_decode, pa_decode_fixed_scratch,
+                      pa_decode_partitions, pa_decode_reduce, pa_decode_shared_prefix, pa_decode_verify,
+                      pa_decode_verify_workspace_size, pa_decode_workspace_size, pa_reshape_and_cache,
+                      pa_set_decode_kernel, pa_set_decode_tiling, pa_set_shared_prefix_kernel,
+                      pa_set_verify_path, pa_version, prefix_plan_to_device)

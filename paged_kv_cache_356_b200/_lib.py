@@ -18,6 +18,18 @@ PA_DEV_TIMEOUT = 32
 PA_DECODE_AUTO, PA_DECODE_CUDA_CORES, PA_DECODE_TENSOR_CORES = 0, 1, 2
 PA_SHARED_PREFIX_AUTO, PA_SHARED_PREFIX_TCGEN05, PA_SHARED_PREFIX_MMA_SYNC, PA_SHARED_PREFIX_TCGEN05_SERIAL = 0, 1, 2, 3
 PA_SHARED_PREFIX_TCGEN05_2CTA = 4
+PA_LOW_FREE_FRACTION = 0.10
+
+
+class PoolStats(ctypes.Structure):
+    """pa_pool_stats of include/pa.h."""
+    _fields_ = [("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32), ("free_pages", ctypes.c_int32),
+                ("used_pages", ctypes.c_int32), ("shared_pages", ctypes.c_int32),
+                ("num_sequences", ctypes.c_int32), ("logical_tokens", ctypes.c_int64),
+                ("physical_tokens", ctypes.c_int64), ("waste_slots", ctypes.c_int64),
+                ("waste_fraction", ctypes.c_double), ("free_fraction", ctypes.c_double),
+                ("low_free_alarm", ctypes.c_int32), ("reserved0", ctypes.c_int32)]
+
 PA_VERIFY_AUTO, PA_VERIFY_PER_SEQUENCE, PA_VERIFY_JOINT = 0, 1, 2
 PA_FAULT_NONE, PA_FAULT_WITHHOLD_FIRST_ITEM = 0, 1
 PA_PARTITION_TOKENS = 512
@@ -66,6 +78,7 @@ SIGNATURES = {
     "pa_block_alloc_num_sequences": (_i32, [_vp]),
     "pa_block_alloc_ref_count": (_i32, [_vp, _i32]),
     "pa_block_alloc_free_pool": (_i32, [_vp, _pi32, _i32, _pi32]),
+    "pa_block_alloc_stats": (_i32, [_vp, ctypes.c_double, ctypes.c_void_p]),
     "pa_block_alloc_prefix_plan": (_i32, [_vp, _pi64, _i32, _i32, _pi32, _pi32, _pi32, _pi32, _pi32, _pi32,
                                           _pi32]),
 }

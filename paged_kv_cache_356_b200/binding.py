@@ -402,6 +402,15 @@ def pa_block_alloc_free_pool(handle) -> np.ndarray:
     return out
 
 
+def pa_block_alloc_stats(handle, alarm_free_fraction: float = _lib.PA_LOW_FREE_FRACTION) -> dict:
+    """Pool occupancy and internal fragmentation (pa_pool_stats) as a dict."""
+    st = _lib.PoolStats()
+    _check(_lib.load().pa_block_alloc_stats(handle, float(alarm_free_fraction), ctypes.byref(st)))
+    out = {name: getattr(st, name) for name, _ in _lib.PoolStats._fields_ if name != "reserved0"}
+    out["low_free_alarm"] = bool(out["low_free_alarm"])
+    return out
+
+
 def pa_block_alloc_prefix_plan(handle, seqs: Sequence[int], group_size: int) -> dict:
     """Host prefix plan of a batch (see include/pa.h): numpy arrays and counts."""
     ids = np.ascontiguousarray(seqs, dtype=np.int64)
@@ -484,3 +493,6 @@ class BlockAllocator:
 
     def prefix_plan(self, seqs, group_size):
         return pa_block_alloc_prefix_plan(self.handle, seqs, group_size)
+
+    def stats(self, alarm_free_fraction=_lib.PA_LOW_FREE_FRACTION):
+        return pa_block_alloc_stats(self.handle, alarm_free_fraction)

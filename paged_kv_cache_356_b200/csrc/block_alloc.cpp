@@ -225,6 +225,38 @@ pa_status pa_block_alloc_free_pool(const pa_block_alloc* a, int32_t* out, int32_
   return PA_OK;
 }
 
+pa_status pa_block_alloc_stats(const pa_block_alloc* a, double alarm_free_fraction, pa_pool_stats* out) {
+  if (!a || !out) return fail(PA_ERR_INVALID, "stats: NULL argument");
+  const int64_t bs = a->block_size;
+  // Filled slots per page: the most any holder has stored in it.
+  std::vector<int32_t> filled(a->num_blocks, 0);
+  pa_pool_stats st{};
+  st.num_blocks = a->num_blocks;
+  st.block_size = a->block_size;
+  st.free_pages = (int32_t)a->count;
+  st.num_sequences = (int32_t)a->seqs.size();
+  for (const auto& kv : a->seqs) {
+    const auto& sq = kv.second;
+    st.logical_tokens += sq.tokens;
+    for (size_t i = 0; i < sq.pages.size(); ++i) {
+      const int64_t n = std::min<int64_t>(bs, sq.tokens - (int64_t)i * bs);
+      int32_t& f = filled[sq.pages[i]];
+      if (n > f) f = (int32_t)n;
+    }
+  }
+  for (int32_t p = 0; p < a->num_blocks; ++p) {
+    if (a->refs[p] > 0) ++st.used_pages;
+    if (a->refs[p] > 1) ++st.shared_pages;
+    st.physical_tokens += filled[p];
+  }
+  st.waste_slots = (int64_t)st.used_pages * bs - st.physical_tokens;
+  st.waste_fraction = st.used_pages > 0 ? (double)st.waste_slots / (double)((int64_t)st.used_pages * bs) : 0.0;
+  st.free_fraction = a->num_blocks > 0 ? (double)st.free_pages / (double)a->num_blocks : 0.0;
+  st.low_free_alarm = a->num_blocks > 0 && st.free_fraction < alarm_free_fraction;
+  *out = st;
+  return PA_OK;
+}
+
 pa_status pa_block_alloc_prefix_plan(const pa_block_alloc* a, const int64_t* seqs, int32_t n, int32_t group_size,
                                      int32_t* first_partition, int32_t* chunks, int32_t* members, int32_t* num_chunks,
                                      int32_t* num_members, int32_t* max_shared_partitions,

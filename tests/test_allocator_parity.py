@@ -154,3 +154,74 @@ def test_workload_traces_match_oracle(name):
     tables, lens = dut.block_tables(list(range(w.num_seqs)), w.max_blocks_per_seq, pad=-1)
     np.testing.assert_array_equal(tables, ref["block_tables"])
     np.testing.assert_array_equal(lens, ref["context_lens"])
+
+
+# -- pool statistics ------------------------------------------------------------------------
+
+def _random_ops(seed, total=300):
+    """The same random op stream applied to the oracle and to the C allocator; yields after each op."""
+    rng = random.Random(seed)
+    bs = rng.choice([1, 3, 16, 32])
+    order = list(range(total))
+    rng.shuffle(order)
+    ref = PagedBlockManager(total, bs, order)
+    dut = pa.BlockAllocator(total, bs, np.array(order, dtype=np.int32))
+    live, next_id = [], 0
+    for _ in range(250):
+        op = rng.randrange(4)
+        try:
+            if op == 0 or not live:
+                n = rng.randrange(0, 70)
+                ref.allocate_sequence(next_id, n)
+                dut.allocate_sequence(next_id, n)
+                live.append(next_id)
+                next_id += 1
+            elif op == 1:
+                parent = rng.choice(live)
+                ref.fork(parent, next_id)
+                dut.fork(parent, next_id)
+                live.append(next_id)
+                next_id += 1
+            elif op == 2:
+                s = rng.choice(live)
+                for _ in range(rng.randrange(1, 9)):
+                    ref.append_token(s)
+                    dut.append_token(s)
+            else:
+                s = rng.choice(live)
+                ref.free_sequence(s)
+                dut.free_sequence(s)
+                live.remove(s)
+        except MemoryError:
+            pass
+        yield ref, dut
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_pool_stats_match_the_oracle_after_every_op(seed):
+    from oracle import fragmentation
+    for ref, dut in _random_ops(seed):
+        for alarm in (0.10, 0.5):
+            want = fragmentation.pool_stats(ref.state(), ref.total_pages, ref.block_size, alarm)
+            assert dut.stats(alarm) == want
+
+
+@pytest.mark.parametrize("name", ["llama8b", "prefix", "beam32k"])
+def test_pool_stats_of_workload_traces(name):
+    from oracle import fragmentation
+    w = workloads.by_name(name)
+    ref = scenario.run(w, with_data=False)
+    dut = pa.BlockAllocator(w.num_blocks, w.block_size, w.initial_free_order())
+    for op in w.trace:
+        if op[0] == "allocate":
+            dut.allocate_sequence(op[1], op[2])
+        elif op[0] == "fork":
+            dut.fork(op[1], op[2])
+        elif op[0] == "append":
+            for _ in range(op[2]):
+                dut.append_token(op[1])
+    assert dut.stats() == fragmentation.pool_stats(ref["state"], w.num_blocks, w.block_size)
+
+
+def test_pool_stats_rejects_null():
+    assert pa._lib.load().pa_block_alloc_stats(None, 0.1, None) == pa._lib.PA_ERR_INVALID
