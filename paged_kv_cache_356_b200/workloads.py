@@ -278,15 +278,15 @@ def _independent(name, seed, num_seqs, hq, hkv, d, bs, ctx) -> Workload:
                     _pool_size(pages), trace=_independent_trace(ctx))
 
 
-def llama8b(seed: int = 1, num_seqs: int = 64, lo: int = 128, hi: int = 4096) -> Workload:
+def llama8b(seed: int = 1, num_seqs: int = 64, lo: int = 128, hi: int = 4096, block_size: int = 16) -> Workload:
     ctx = _rng(seed, _TAG_LENGTHS).integers(lo, hi + 1, size=num_seqs)
-    return _independent("llama8b", seed, num_seqs, 32, 8, 128, 16, ctx)
+    return _independent("llama8b", seed, num_seqs, 32, 8, 128, block_size, ctx)
 
 
-def llama70b(seed: int = 2, num_seqs: int = 256, lo: int = 512, hi: int = 8192) -> Workload:
+def llama70b(seed: int = 2, num_seqs: int = 256, lo: int = 512, hi: int = 8192, block_size: int = 16) -> Workload:
     u = _rng(seed, _TAG_LENGTHS).uniform(math.log(lo), math.log(hi), size=num_seqs)
     ctx = np.clip(np.floor(np.exp(u)), lo, hi).astype(np.int64)
-    return _independent("llama70b", seed, num_seqs, 64, 8, 128, 16, ctx)
+    return _independent("llama70b", seed, num_seqs, 64, 8, 128, block_size, ctx)
 
 
 def prefix(seed: int = 3, num_seqs: int = 100, prefix_len: int = 10_000, max_tail: int = 512,
@@ -299,10 +299,11 @@ def prefix(seed: int = 3, num_seqs: int = 100, prefix_len: int = 10_000, max_tai
                     trace=_shared_trace(prefix_len, [int(t) for t in tails]))
 
 
-def beam32k(seed: int = 4, num_beams: int = 8, prompt_len: int = 32_768, own: int = 64) -> Workload:
+def beam32k(seed: int = 4, num_beams: int = 8, prompt_len: int = 32_768, own: int = 64,
+            block_size: int = 16) -> Workload:
     ctx = tuple([prompt_len + own] * num_beams)
-    bound = -(-prompt_len // 16) + num_beams * (1 + -(-own // 16))
-    return Workload("beam32k", seed, num_beams, 64, 8, 128, 16, "bf16", "beam", ctx,
+    bound = -(-prompt_len // block_size) + num_beams * (1 + -(-own // block_size))
+    return Workload("beam32k", seed, num_beams, 64, 8, 128, block_size, "bf16", "beam", ctx,
                     _pool_size(bound), prefix_len=prompt_len,
                     trace=_shared_trace(prompt_len, [own] * num_beams))
 

@@ -28,3 +28,23 @@ def test_unique_and_logical_kv_bytes():
     per_token = 2 * w.num_kv_heads * w.head_dim * w.elem_bytes
     assert unique == (4 * bs + 3 * 16) * per_token
     assert logical == 3 * 80 * per_token
+
+
+def test_fragmentation_rows_match_the_oracle_and_the_pages_bound():
+    """bench --fragmentation: the C allocator's statistics equal the oracle's for the same trace; for
+    independent sequences the paged waste is far under the pages' "under 4 percent", the contiguous
+    reservation's far above it."""
+    from oracle import fragmentation, scenario
+    from paged_kv_cache_356_b200 import workloads
+    rows = bench.fragmentation_rows(names=("llama8b", "beam32k"), block_sizes=(16, 32))
+    assert len(rows) == 4
+    for r in rows:
+        w = workloads.by_name(r["workload"], block_size=r["block_size"])
+        ref = fragmentation.pool_stats(scenario.run(w, with_data=False)["state"], w.num_blocks, w.block_size)
+        assert r["paged_waste_fraction"] == ref["waste_fraction"]
+        assert r["physical_tokens"] == ref["physical_tokens"] and r["used_pages"] == ref["used_pages"]
+        assert not r["low_free_alarm"]
+    ind = [r for r in rows if r["workload"] == "llama8b"]
+    assert all(r["paged_waste_fraction"] < 0.04 < r["contiguous_waste_fraction"] for r in ind)
+    beam = [r for r in rows if r["workload"] == "beam32k"]
+    assert all(r["shared_pages"] > 0 and r["contiguous_over_paged_slots"] > 5 for r in beam)
