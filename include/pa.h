@@ -189,9 +189,9 @@ PA_API pa_status pa_decode_reduce(const int32_t* context_lens, int32_t num_seqs,
  * pa_decode_verify -- several query tokens per sequence (checking draft
  * tokens of speculative decoding against the paged cache in one pass).
  *
- * [Internals] "The Mathematical Cause of KV Cache Fragmentation" points to
- * speculative-decoding kernels that verify parallel draft tokens across
- * paged memory; it gives no formula.  Reading: the T = num_query_tokens
+ * [Internals] "The Mathematical Cause of KV Cache Fragmentation" mentions
+ * speculative-decoding kernels that check a sequence's draft tokens together
+ * against the paged cache; it gives no formula.  Reading: the T = num_query_tokens
  * query tokens of sequence b are the last T positions of its context, their
  * K/V already written (pa_reshape_and_cache); token t sits at position
  * pos_t = context_lens[b] - T + t and attends causally:
