@@ -69,6 +69,8 @@ def parse_args(argv=None):
     ap.add_argument("--verify-tokens", type=int, default=0,
                     help="T > 0: each step writes T draft tokens per sequence and runs pa_decode_verify "
                          "(T causal query tokens per sequence) instead of a one-token decode step")
+    ap.add_argument("--verify-rows", type=int, default=0, choices=[0, 8, 16, 32],
+                    help="with --verify-tokens: rows per CTA of the per-sequence verify kernel (0: default)")
     ap.add_argument("--verify-path", choices=["auto", "per_sequence", "joint"], default="auto",
                     help="with --verify-tokens: joint kernel for the partitions all tokens see (auto: when T*G > 16)")
     return ap.parse_args(argv)
@@ -451,6 +453,7 @@ def run_ours(args):
                              "cc": pa.PA_DECODE_CUDA_CORES}[args.kernel])
     warps, stages = (int(x) for x in args.tiling.split("x"))
     pa.pa_set_decode_tiling(warps, stages)
+    pa.pa_set_verify_tiling(args.verify_rows)
     pa.pa_set_verify_path({"auto": pa.PA_VERIFY_AUTO, "per_sequence": pa.PA_VERIFY_PER_SEQUENCE,
                            "joint": pa.PA_VERIFY_JOINT}[args.verify_path])
     pa.pa_set_shared_prefix_kernel({"auto": pa.PA_SHARED_PREFIX_AUTO, "tcgen05": pa.PA_SHARED_PREFIX_TCGEN05,
@@ -648,6 +651,7 @@ def run_ours(args):
         if T > 0:
             cfg["query_tokens"] = T
             cfg["verify_path"] = f"{args.verify_path} ({'joint + per-sequence' if verify_joint else 'per-sequence'})"
+            cfg["verify_rows_per_cta"] = args.verify_rows or "default"
             cfg["workload"] += f"; {T} draft tokens per sequence verified per step (causal)"
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

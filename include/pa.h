@@ -231,6 +231,12 @@ typedef enum {
   PA_VERIFY_JOINT = 2          /* joint kernel whenever the call allows it; PA_ERR_UNSUPPORTED otherwise */
 } pa_verify_path;
 PA_API pa_status pa_set_verify_path(pa_verify_path path);
+/* Rows of (token, query head) pairs per CTA of the per-sequence verify
+ * kernel: 8, 16 or 32 (at most 16 at head_dim 256), or 0 for the default
+ * (the fewest that hold a kv head's T * G rows, up to 32).  Fewer rows per
+ * CTA mean more CTAs per kv head (each reading the partition's pages, mostly
+ * from L2) and fewer registers per thread.  Process-wide. */
+PA_API pa_status pa_set_verify_tiling(int32_t rows_per_cta);
 PA_API size_t pa_decode_verify_workspace_size(int32_t num_seqs, int32_t num_query_tokens, int32_t num_q_heads,
                                               int32_t head_dim, int64_t max_context_len);
 PA_API pa_status pa_decode_verify(const void* q, const void* key_cache, const void* value_cache,

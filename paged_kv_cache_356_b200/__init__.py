@@ -17,4 +17,4 @@ from .binding import (BlockAllocator, PagedAttentionError, PagedAttentionOOM, Se
                       pa_decode_partitions, pa_decode_reduce, pa_decode_shared_prefix, pa_decode_verify,
                       pa_decode_verify_workspace_size, pa_decode_workspace_size, pa_reshape_and_cache,
                       pa_set_decode_kernel, pa_set_decode_tiling, pa_set_shared_prefix_kernel,
-                      pa_set_verify_path, pa_version, prefix_plan_to_device)
+                      pa_set_verify_path, pa_set_verify_tiling, pa_version, prefix_plan_to_device)

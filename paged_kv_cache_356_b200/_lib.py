@@ -51,6 +51,7 @@ SIGNATURES = {
                          _vp, _sz, _vp, _vp]),
     "pa_decode_verify_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i64]),
     "pa_set_verify_path": (_i32, [_i32]),
+    "pa_set_verify_tiling": (_i32, [_i32]),
     "pa_decode_verify": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
                                 _vp, _i32, _vp, _sz, _vp, _vp]),
     "pa_decode_partitions": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp,

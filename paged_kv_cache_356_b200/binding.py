@@ -285,6 +285,11 @@ def pa_set_verify_path(path: int) -> None:
     _check(_lib.load().pa_set_verify_path(int(path)))
 
 
+def pa_set_verify_tiling(rows_per_cta: int) -> None:
+    """Rows per CTA of the per-sequence verify kernel: 8, 16, 32, or 0 for the default."""
+    _check(_lib.load().pa_set_verify_tiling(int(rows_per_cta)))
+
+
 def pa_set_fault_injection(mode: int) -> None:
     """Test hook for the device-side timeout path (see include/pa.h)."""
     _check(_lib.load().pa_set_fault_injection(int(mode)))

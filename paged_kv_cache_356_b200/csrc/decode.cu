@@ -2792,6 +2792,7 @@ std::atomic<int> g_kernel_choice{PA_DECODE_AUTO};
 std::atomic<int> g_fault{PA_FAULT_NONE};
 std::atomic<int> g_tc_warps{4};
 std::atomic<int> g_tc_stages{2};
+std::atomic<int> g_verify_rows{0};
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -3107,12 +3108,15 @@ template <typename T, int D>
 cudaError_t launch_verify_tc_dim(const DecodeArgs& a, const VerifyArgs& v, int num_seqs, int partitions,
                                  cudaStream_t stream) {
   const int rows = v.num_tokens * a.group;
+  // pa_set_verify_tiling may cap the rows per CTA (more row groups, fewer registers per thread).
+  const int cap = g_verify_rows.load();
+  const int per_cta = std::min(rows <= 8 ? 8 : rows <= 16 ? 16 : 32, cap > 0 ? cap : 32);
   if constexpr (D == 256) {
-    if (rows <= 8) return launch_verify_tc<T, D, 4, 2, 1>(a, v, num_seqs, partitions, stream);
+    if (per_cta <= 8) return launch_verify_tc<T, D, 4, 2, 1>(a, v, num_seqs, partitions, stream);
     return launch_verify_tc<T, D, 4, 2, 2>(a, v, num_seqs, partitions, stream);
   } else {
-    if (rows <= 8) return launch_verify_tc<T, D, 4, 3, 1>(a, v, num_seqs, partitions, stream);
-    if (rows <= 16) return launch_verify_tc<T, D, 4, 3, 2>(a, v, num_seqs, partitions, stream);
+    if (per_cta <= 8) return launch_verify_tc<T, D, 4, 3, 1>(a, v, num_seqs, partitions, stream);
+    if (per_cta <= 16) return launch_verify_tc<T, D, 4, 3, 2>(a, v, num_seqs, partitions, stream);
     return launch_verify_tc<T, D, 4, 3, 4>(a, v, num_seqs, partitions, stream);
   }
 }
@@ -3172,6 +3176,14 @@ extern "C" pa_status pa_set_shared_prefix_kernel(pa_shared_prefix_kernel k) {
       k != PA_SHARED_PREFIX_TCGEN05_SERIAL && k != PA_SHARED_PREFIX_TCGEN05_2CTA)
     return fail(PA_ERR_INVALID, "pa_set_shared_prefix_kernel: unknown kernel %d", (int)k);
   g_shared_kernel.store((int)k);
+  return PA_OK;
+}
+
+extern "C" pa_status pa_set_verify_tiling(int32_t rows_per_cta) {
+  if (rows_per_cta != 0 && rows_per_cta != 8 && rows_per_cta != 16 && rows_per_cta != 32)
+    return fail(PA_ERR_UNSUPPORTED, "pa_set_verify_tiling: %d rows per CTA (built: 8, 16, 32; 0 = default)",
+                rows_per_cta);
+  g_verify_rows.store(rows_per_cta);
   return PA_OK;
 }
 

@@ -80,3 +80,60 @@ def test_step_replay_is_idempotent(full_run):
     run.step()
     torch.cuda.synchronize()
     assert torch.equal(run.out.view(torch.int16), first.view(torch.int16))
+
+
+# -- draft verification at full size (the bench's --verify-tokens step) ------------------------------
+
+@pytest.fixture(scope="module", params=["llama8b", "llama70b"])
+def verify_run(request):
+    import torch
+    pa.pa_set_decode_kernel(pa.PA_DECODE_AUTO)
+    w = workloads.by_name(request.param)
+    run = TraceRunner(w)
+    run.run(decode=False)
+    torch.cuda.synchronize()
+    yield w, run
+    del run
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("num_tokens", [4, 8])
+def test_verify_step_on_sampled_sequences(verify_run, num_tokens):
+    """Draft tokens written at each sequence's last T positions, then pa_decode_verify (auto path) as
+    the bench times it; sampled rows against textbook causal attention over the sequence's tokens,
+    regenerated from the seeds with the draft tokens' K/V in place."""
+    import torch
+    w, run = verify_run
+    T = num_tokens
+    ctx = np.array(w.context_lens)
+    slots = np.concatenate([run.alloc.slot_mapping(b, int(ctx[b]) - T, T) for b in range(w.num_seqs)])
+    dk, dv = w.draft_kv(T)
+    q = w.draft_query(T)
+    pages = torch.from_numpy(slots // w.block_size).cuda()
+    offs = torch.from_numpy(slots % w.block_size).cuda()
+    saved = run.key_cache[pages, :, offs, :].clone(), run.value_cache[pages, :, offs, :].clone()
+    pa.pa_reshape_and_cache(run._to_device(dk), run._to_device(dv), torch.from_numpy(slots.astype(np.int64)).cuda(),
+                            run.key_cache, run.value_cache)
+    out = pa.pa_decode_verify(run._to_device(q), run.key_cache, run.value_cache, run.block_tables,
+                              run.context_lens, w.scale)
+    torch.cuda.synchronize()
+    # the trace's own K/V back in place for the next case
+    run.key_cache[pages, :, offs, :] = saved[0]
+    run.value_cache[pages, :, offs, :] = saved[1]
+    assert run.status() == 0
+    rng = np.random.default_rng(T)
+    pick = sorted({int(np.argmax(ctx)), int(np.argmin(ctx)), *rng.choice(w.num_seqs, 4, False)})
+    heads = sorted(rng.choice(w.num_q_heads, 8, False))
+    q64 = attention.to_float64(q, w.dtype)
+    g = w.group_size
+    ref = np.zeros((len(pick), T, len(heads), w.head_dim))
+    for i, b in enumerate(pick):
+        k, v = w.sequence_kv(b)
+        k, v = k.copy(), v.copy()
+        k[-T:], v[-T:] = dk[b * T:(b + 1) * T], dv[b * T:(b + 1) * T]
+        k64, v64 = attention.to_float64(k, w.dtype), attention.to_float64(v, w.dtype)
+        for t in range(T):
+            n = attention.visible_keys(int(ctx[b]), T, t)
+            for j, h in enumerate(heads):
+                ref[i, t, j] = attention.softmax_attention(q64[b, t, h], k64[:n, h // g], v64[:n, h // g], w.scale)
+    assert_decode_close(out[pick][:, :, heads], ref, w.dtype, f"{w.name} T={T}")

@@ -31,6 +31,7 @@ def _reset_kernel():
     pa.pa_set_decode_kernel(pa.PA_DECODE_AUTO)
     pa.pa_set_verify_path(pa.PA_VERIFY_AUTO)
     pa.pa_set_shared_prefix_kernel(pa.PA_SHARED_PREFIX_AUTO)
+    pa.pa_set_verify_tiling(0)
 
 
 def _values(rng, n, dtype):
@@ -133,6 +134,20 @@ def test_joint_path_partition_edges(num_tokens, hq, hkv, d, joint_kernel):
                                     "mma_sync": pa.PA_SHARED_PREFIX_MMA_SYNC}[joint_kernel])
     case = _case(300 + num_tokens, _edge_contexts(num_tokens), num_tokens, hq, hkv, d, 16, "bf16")
     assert_decode_close(_run(case, "tc", path="joint"), _oracle(case), "bf16", joint_kernel)
+
+
+@pytest.mark.parametrize("path", ["per_sequence", "joint"])
+@pytest.mark.parametrize("rows_per_cta", [8, 16, 32])
+def test_every_built_row_tiling_matches(rows_per_cta, path):
+    """32 rows per kv head served by 4, 2 or 1 CTAs of 8, 16 or 32 rows."""
+    pa.pa_set_verify_tiling(rows_per_cta)
+    case = _case(400 + rows_per_cta, CONTEXTS, 4, 64, 8, 128, 16, "bf16")
+    assert_decode_close(_run(case, "tc", path=path), _oracle(case), "bf16", f"{rows_per_cta} {path}")
+
+
+def test_unbuilt_row_tiling_is_rejected():
+    with pytest.raises(pa.PagedAttentionError):
+        pa.pa_set_verify_tiling(24)
 
 
 def test_joint_path_that_cannot_run_is_rejected():
