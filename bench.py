@@ -52,10 +52,6 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle time budget for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-chunks", type=int, default=4,
-                    help="end-to-end leg: split the batch into this many sub-batches whose copies overlap the "
-                         "previous sub-batch's kernels (1 = copy everything, then compute; shared-prefix "
-                         "steps always use 1, their plan spans the batch)")
     ap.add_argument("--no-clocks", action="store_true", help="skip the nvidia-smi clock record (profiler runs)")
     ap.add_argument("--micro", action="store_true",
                     help="instead of the decode step, time the cache write (65,536 tokens) and the page copy "
@@ -728,36 +724,15 @@ def end_to_end(args, torch, pa, run, w, unique, world, dist, inputs, decode):
     d_out = torch.empty_like(out_dev)
     seqs = list(range(w.num_seqs))
     tab_np, ctx_np = h_tab.numpy(), h_ctx.numpy()
-    # Sub-batches: sequences [lo, hi) with their rows of the step's cache write (the write holds the
-    # same number of tokens for every sequence, in sequence order).
-    chunks = 1 if run.plan is not None else max(1, min(args.e2e_chunks, w.num_seqs))
-    per_seq = h_k.shape[0] // w.num_seqs
-    assert per_seq * w.num_seqs == h_k.shape[0]
-    bounds = [(w.num_seqs * c // chunks, w.num_seqs * (c + 1) // chunks) for c in range(chunks)]
-    compute = torch.cuda.current_stream()
-    copy_in, copy_out = torch.cuda.Stream(), torch.cuda.Stream()
-    ev_in = [torch.cuda.Event() for _ in bounds]
-    ev_done = [torch.cuda.Event() for _ in bounds]
 
     def e2e_step():
-        for c, (lo, hi) in enumerate(bounds):
-            run.alloc.block_tables(seqs[lo:hi], w.max_blocks_per_seq, pad=-1, out=tab_np[lo:hi],
-                                   lens_out=ctx_np[lo:hi])
-            t0, t1 = lo * per_seq, hi * per_seq
-            with torch.cuda.stream(copy_in):
-                for dst, src in ((d_q[lo:hi], h_q[lo:hi]), (d_k[t0:t1], h_k[t0:t1]), (d_v[t0:t1], h_v[t0:t1]),
-                                 (d_s[t0:t1], h_s[t0:t1]), (d_tab[lo:hi], h_tab[lo:hi]),
-                                 (d_ctx[lo:hi], h_ctx[lo:hi])):
-                    dst.copy_(src, non_blocking=True)
-                ev_in[c].record(copy_in)
-            compute.wait_event(ev_in[c])
-            pa.pa_reshape_and_cache(d_k[t0:t1], d_v[t0:t1], d_s[t0:t1], run.key_cache, run.value_cache)
-            decode(d_q[lo:hi], d_tab[lo:hi], d_ctx[lo:hi], d_out[lo:hi])
-            ev_done[c].record(compute)
-            with torch.cuda.stream(copy_out):
-                copy_out.wait_event(ev_done[c])
-                h_out[lo:hi].copy_(d_out[lo:hi], non_blocking=True)
-        copy_out.synchronize()
+        run.alloc.block_tables(seqs, w.max_blocks_per_seq, pad=-1, out=tab_np, lens_out=ctx_np)
+        for dst, src in ((d_q, h_q), (d_k, h_k), (d_v, h_v), (d_s, h_s), (d_tab, h_tab), (d_ctx, h_ctx)):
+            dst.copy_(src, non_blocking=True)
+        pa.pa_reshape_and_cache(d_k, d_v, d_s, run.key_cache, run.value_cache)
+        decode(d_q, d_tab, d_ctx, d_out)
+        h_out.copy_(d_out, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
 
     for _ in range(3):
         e2e_step()
@@ -773,10 +748,9 @@ def end_to_end(args, torch, pa, run, w, unique, world, dist, inputs, decode):
     h2d = sum(x.numel() * x.element_size() for x in (h_q, h_k, h_v, h_s, h_tab, h_ctx))
     d2h = h_out.numel() * h_out.element_size()
     return {"value": unique * args.steps / elapsed / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": 1000 * elapsed / args.steps, "sub_batches": chunks,
+            "d2h_bytes_per_step": d2h, "ms_per_step": 1000 * elapsed / args.steps,
             "includes": "host table export (C ABI), pinned H2D of q/new K,V/slots/tables/lengths, "
-                        "reshape_and_cache + decode, D2H of out, stream sync; with sub-batches, copy "
-                        "streams move sub-batch c+1 in and c-1 out while c computes"}
+                        "reshape_and_cache + decode, D2H of out, stream sync"}
 
 
 # ---------------------------------------------------------------------------------------------
