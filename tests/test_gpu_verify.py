@@ -150,6 +150,14 @@ def test_unbuilt_row_tiling_is_rejected():
         pa.pa_set_verify_tiling(24)
 
 
+@pytest.mark.parametrize("route", ROUTES, ids=["-".join(r) for r in ROUTES])
+def test_prefill_chunk_of_many_tokens(route):
+    """A chunk of 100 new tokens at the end of each context (chunked prefill is the same computation):
+    400 rows per kv head, many row groups and joint-kernel chunks per sequence."""
+    case = _case(500, [100, 101, 700, 1537, 2100], 100, 16, 4, 64, 16, "bf16")
+    assert_decode_close(_run(case, route[0], path=route[1]), _oracle(case), "bf16", str(route))
+
+
 def test_joint_path_that_cannot_run_is_rejected():
     case = _case(17, [10, 20], 2, 8, 2, 64, 16, "bf16")      # one partition: nothing for the joint kernel
     with pytest.raises(pa.PagedAttentionError):
