@@ -72,3 +72,35 @@ def test_device_calls_reject_cpu_tensors():
                                      kc, kc.clone())
     with pytest.raises(TypeError):
         binding.pa_copy_blocks(kc, kc.clone(), torch.zeros(1, 2, dtype=torch.int64))
+
+
+def test_verify_workspace_size_matches_documented_layout():
+    """The pa_decode partials with T * H_q heads per sequence, then the joint kernel's plan arrays."""
+    align = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert binding.pa_decode_verify_workspace_size(4, 3, 8, 128, 512) == 0          # one partition
+    assert binding.pa_decode_verify_workspace_size(4, 0, 8, 128, 4096) == 0         # no query token
+    b, t, hq, d, ctx = 256, 4, 64, 128, 8192
+    parts = binding.pa_decode_workspace_size(b, t * hq, d, ctx)
+    assert binding.pa_decode_verify_workspace_size(b, t, hq, d, ctx) == parts + align(16 * b * t) + align(4 * b * t)
+    assert binding.pa_decode_verify_workspace_size(3, 7, 5, 64, 1025) == (
+        binding.pa_decode_workspace_size(3, 35, 64, 1025) + align(16 * 21) + align(4 * 21))
+
+
+def test_verify_and_pool_setters_validate_on_the_host():
+    with pytest.raises(binding.PagedAttentionError):
+        binding.pa_set_verify_path(7)
+    with pytest.raises(binding.PagedAttentionError):
+        binding.pa_set_verify_tiling(12)
+    binding.pa_set_verify_path(binding.PA_VERIFY_AUTO)
+    binding.pa_set_verify_tiling(0)
+
+
+def test_verify_rejects_cpu_tensors_and_bad_shapes():
+    import torch
+    kc = torch.zeros(2, 1, 16, 64, dtype=torch.bfloat16)
+    tables = torch.zeros(1, 2, dtype=torch.int32)
+    ctx = torch.ones(1, dtype=torch.int32)
+    with pytest.raises(ValueError):   # 3-D q
+        binding.pa_decode_verify(torch.zeros(1, 4, 64, dtype=torch.bfloat16), kc, kc.clone(), tables, ctx, 0.1)
+    with pytest.raises(TypeError):    # host tensors
+        binding.pa_decode_verify(torch.zeros(1, 2, 4, 64, dtype=torch.bfloat16), kc, kc.clone(), tables, ctx, 0.1)
