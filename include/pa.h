@@ -56,7 +56,7 @@ typedef enum pa_status {
   PA_ERR_OOM = -2,         /* the free-page pool cannot satisfy the request; state unchanged */
   PA_ERR_CUDA = -3,        /* a CUDA runtime call failed; see pa_last_error() */
   PA_ERR_NOT_FOUND = -4,   /* unknown sequence id */
-  PA_ERR_UNSUPPORTED = -5  /* a shape / dtype combination this build has no kernel for */
+  PA_ERR_UNSUPPORTED = -5  /* a shape / dtype combination the library has no kernel for */
 } pa_status;
 
 typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1, PA_F16 = 2 } pa_dtype;
