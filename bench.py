@@ -722,7 +722,7 @@ def end_to_end(args, torch, pa, run, w, unique, world, dist, inputs, decode):
     d_tab = torch.empty_like(run.block_tables)
     d_ctx = torch.empty_like(run.context_lens)
     d_out = torch.empty_like(out_dev)
-    seqs = list(range(w.num_seqs))
+    seqs = np.arange(w.num_seqs, dtype=np.int64)   # passed through to the C export without conversion
     tab_np, ctx_np = h_tab.numpy(), h_ctx.numpy()
 
     def e2e_step():
