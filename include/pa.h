@@ -410,6 +410,15 @@ PA_API pa_status pa_block_alloc_allocate_sequence(pa_block_alloc* a, int64_t seq
 PA_API pa_status pa_block_alloc_append_token(pa_block_alloc* a, int64_t seq, int64_t* slot_out,
                                       int32_t* cow_src, int32_t* cow_dst);
 
+/* pa_block_alloc_append_token for n sequences in order (one position each,
+ * as a decode step grows every sequence of a batch): slots_out[i] (may be
+ * NULL), cow_src[i], cow_dst[i] as above.  Stops at the first failure and
+ * returns its status; *n_done (may be NULL) receives the number of appends
+ * made, each complete, and the failed one changed nothing. */
+PA_API pa_status pa_block_alloc_append_tokens(pa_block_alloc* a, const int64_t* seqs, int32_t n,
+                                              int64_t* slots_out, int32_t* cow_src, int32_t* cow_dst,
+                                              int32_t* n_done);
+
 /* New sequence `child` sharing every page of `parent` (each gains one
  * reference); it starts with the parent's token count. */
 PA_API pa_status pa_block_alloc_fork(pa_block_alloc* a, int64_t parent, int64_t child);

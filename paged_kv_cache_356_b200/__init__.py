@@ -8,7 +8,8 @@ package is its thin Python binding (``binding``), the in-tree build
 (``runner``) and the seeded synthetic workloads (``workloads``).
 """
 from .binding import (BlockAllocator, PagedAttentionError, PagedAttentionOOM, SequenceNotFound,  # noqa: F401
-                      pa_block_alloc_allocate_sequence, pa_block_alloc_append_token, pa_block_alloc_block_table,
+                      pa_block_alloc_allocate_sequence, pa_block_alloc_append_token, pa_block_alloc_append_tokens,
+                      pa_block_alloc_block_table,
                       pa_block_alloc_block_tables, pa_block_alloc_create, pa_block_alloc_destroy,
                       pa_block_alloc_fork, pa_block_alloc_free_pool, pa_block_alloc_free_sequence,
                       pa_block_alloc_num_free, pa_block_alloc_num_sequences, pa_block_alloc_num_tokens,

@@ -79,6 +79,7 @@ SIGNATURES = {
     "pa_block_alloc_num_sequences": (_i32, [_vp]),
     "pa_block_alloc_ref_count": (_i32, [_vp, _i32]),
     "pa_block_alloc_free_pool": (_i32, [_vp, _pi32, _i32, _pi32]),
+    "pa_block_alloc_append_tokens": (_i32, [_vp, _pi64, _i32, _pi64, _pi32, _pi32, _pi32]),
     "pa_block_alloc_stats": (_i32, [_vp, ctypes.c_double, ctypes.c_void_p]),
     "pa_block_alloc_prefix_plan": (_i32, [_vp, _pi64, _i32, _i32, _pi32, _pi32, _pi32, _pi32, _pi32, _pi32,
                                           _pi32]),

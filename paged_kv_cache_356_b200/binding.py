@@ -342,6 +342,20 @@ def pa_block_alloc_append_token(handle, seq: int) -> Tuple[int, int, int]:
     return slot.value, src.value, dst.value
 
 
+def pa_block_alloc_append_tokens(handle, seqs: Sequence[int]) -> Tuple[np.ndarray, np.ndarray]:
+    """One position for each of ``seqs`` in order, in one call: (slots int64 [n], cow pairs int32 [n, 2],
+    -1 where no page was forked).  On failure raises; the appends before the failing one stand."""
+    ids = np.ascontiguousarray(seqs, dtype=np.int64)
+    n = len(ids)
+    slots = np.empty(n, dtype=np.int64)
+    src = np.empty(n, dtype=np.int32)
+    dst = np.empty(n, dtype=np.int32)
+    done = ctypes.c_int32()
+    _check(_lib.load().pa_block_alloc_append_tokens(handle, _i64p(ids), n, _i64p(slots), _i32p(src), _i32p(dst),
+                                                    ctypes.byref(done)))
+    return slots, np.stack([src, dst], axis=1)
+
+
 def pa_block_alloc_fork(handle, parent: int, child: int) -> None:
     _check(_lib.load().pa_block_alloc_fork(handle, parent, child))
 
@@ -465,6 +479,9 @@ class BlockAllocator:
 
     def append_token(self, seq):
         return pa_block_alloc_append_token(self.handle, seq)
+
+    def append_tokens(self, seqs):
+        return pa_block_alloc_append_tokens(self.handle, seqs)
 
     def fork(self, parent, child):
         pa_block_alloc_fork(self.handle, parent, child)

@@ -130,6 +130,20 @@ pa_status pa_block_alloc_append_token(pa_block_alloc* a, int64_t seq, int64_t* s
   return PA_OK;
 }
 
+pa_status pa_block_alloc_append_tokens(pa_block_alloc* a, const int64_t* seqs, int32_t n, int64_t* slots_out,
+                                       int32_t* cow_src, int32_t* cow_dst, int32_t* n_done) {
+  if (n_done) *n_done = 0;
+  if (!a || n < 0 || (n > 0 && (!seqs || !cow_src || !cow_dst)))
+    return fail(PA_ERR_INVALID, "append_tokens: bad argument");
+  for (int32_t i = 0; i < n; ++i) {
+    const pa_status st =
+        pa_block_alloc_append_token(a, seqs[i], slots_out ? slots_out + i : nullptr, cow_src + i, cow_dst + i);
+    if (st != PA_OK) return st;  // that append changed nothing; the earlier ones stand
+    if (n_done) *n_done = i + 1;
+  }
+  return PA_OK;
+}
+
 pa_status pa_block_alloc_fork(pa_block_alloc* a, int64_t parent, int64_t child) {
   if (!a) return fail(PA_ERR_INVALID, "fork: NULL handle");
   auto it = a->seqs.find(parent);

@@ -225,3 +225,58 @@ def test_pool_stats_of_workload_traces(name):
 
 def test_pool_stats_rejects_null():
     assert pa._lib.load().pa_block_alloc_stats(None, 0.1, None) == pa._lib.PA_ERR_INVALID
+
+
+# -- batched appends ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("seed", range(4))
+def test_batched_appends_equal_sequential_ones_in_the_oracle(seed):
+    """pa_block_alloc_append_tokens over a batch = the oracle's append_token for each sequence in order:
+    the same slots, copy-on-write pairs and state, through forks and shared partial pages."""
+    rng = random.Random(seed)
+    bs = rng.choice([1, 4, 16])
+    total = 500
+    order = list(range(total))
+    rng.shuffle(order)
+    ref = PagedBlockManager(total, bs, order)
+    dut = pa.BlockAllocator(total, bs, np.array(order, dtype=np.int32))
+    live = []
+    for s in range(6):
+        n = rng.randrange(0, 40)
+        ref.allocate_sequence(s, n)
+        dut.allocate_sequence(s, n)
+        live.append(s)
+    for child in range(6, 12):
+        parent = rng.choice(live)
+        ref.fork(parent, child)
+        dut.fork(parent, child)
+        live.append(child)
+    for _ in range(30):
+        batch = [rng.choice(live) for _ in range(rng.randrange(1, 12))]
+        want = [ref.append_token(s) for s in batch]
+        slots, pairs = dut.append_tokens(batch)
+        assert [int(x) for x in slots] == [w[0] for w in want]
+        assert [tuple(int(v) for v in p) for p in pairs] == [w[1] if w[1] else (-1, -1) for w in want]
+    assert _state(dut, live, total) == ref.state()
+
+
+def test_batched_appends_stop_at_the_first_failure():
+    import ctypes
+    a = pa.BlockAllocator(3, 4)
+    a.allocate_sequence(0, 4)        # one full page
+    a.allocate_sequence(1, 3)        # one page, room for one more
+    # 0 needs a page (1 left), 1 fits, 0 fits, 0 fits, 0 fits, then 0 needs a page: none left
+    seqs = np.array([0, 1, 0, 0, 0, 0], dtype=np.int64)
+    slots = np.empty(6, dtype=np.int64)
+    src = np.empty(6, dtype=np.int32)
+    dst = np.empty(6, dtype=np.int32)
+    done = ctypes.c_int32()
+    lib = pa._lib.load()
+    st = lib.pa_block_alloc_append_tokens(a.handle, pa._i64p(seqs), 6, pa._i64p(slots), pa._i32p(src),
+                                          pa._i32p(dst), ctypes.byref(done))
+    assert st == pa._lib.PA_ERR_OOM and done.value == 5
+    assert a.num_tokens(0) == 8 and a.num_tokens(1) == 4 and a.num_free() == 0
+    with pytest.raises(MemoryError):
+        a.append_tokens([1, 0])      # 1 needs a page: fails first, nothing changes
+    assert a.num_tokens(1) == 4 and a.num_tokens(0) == 8
+    assert lib.pa_block_alloc_append_tokens(a.handle, None, 1, None, None, None, None) == pa._lib.PA_ERR_INVALID
