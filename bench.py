@@ -765,26 +765,36 @@ def fragmentation_rows(names=("llama8b", "llama70b", "prefix", "beam32k"), block
     """Run each workload's allocator trace through pa_block_alloc; pool statistics per (workload, bs)."""
     from paged_kv_cache_356_b200 import binding as pa
     from paged_kv_cache_356_b200 import workloads
+    def replay(w, alloc):
+        ops = 0
+        for op in w.trace:
+            if op[0] == "allocate":
+                alloc.allocate_sequence(op[1], op[2])
+                ops += 1
+            elif op[0] == "fork":
+                alloc.fork(op[1], op[2])
+                ops += 1
+            elif op[0] == "append":
+                for _ in range(op[2]):
+                    alloc.append_token(op[1])
+                ops += op[2]
+        return ops
+
     rows = []
     for name in names:
         for bs in block_sizes:
             w = workloads.by_name(name, block_size=bs)
             alloc = pa.BlockAllocator(w.num_blocks, w.block_size, w.initial_free_order())
-            ops = 0
             t0 = time.perf_counter()
-            for op in w.trace:
-                if op[0] == "allocate":
-                    alloc.allocate_sequence(op[1], op[2])
-                    ops += 1
-                elif op[0] == "fork":
-                    alloc.fork(op[1], op[2])
-                    ops += 1
-                elif op[0] == "append":
-                    for _ in range(op[2]):
-                        alloc.append_token(op[1])
-                    ops += op[2]
+            ops = replay(w, alloc)
             host_s = time.perf_counter() - t0
             st = alloc.stats()
+            # The same trace in a pool that ends 5% free (the traces only grow, so their peak is
+            # their end): the low-free-pages alarm has to fire there.
+            tight = pa.BlockAllocator(int(math.ceil(st["used_pages"] / 0.95)), bs)
+            replay(w, tight)
+            st_tight = tight.stats()
+            tight.close()
             reserved = w.num_seqs * MAX_LEN[name]
             rows.append({
                 "workload": name, "block_size": bs, "num_seqs": w.num_seqs, "pool_pages": w.num_blocks,
@@ -797,6 +807,8 @@ def fragmentation_rows(names=("llama8b", "llama70b", "prefix", "beam32k"), block
                 "contiguous_over_paged_slots": reserved / max(1, st["used_pages"] * bs),
                 "free_fraction": st["free_fraction"], "low_free_alarm": st["low_free_alarm"],
                 "allocator_ops": ops, "allocator_us_per_op": 1e6 * host_s / max(1, ops),
+                "tight_pool_pages": st_tight["num_blocks"], "tight_free_fraction": st_tight["free_fraction"],
+                "tight_low_free_alarm": st_tight["low_free_alarm"],
             })
             alloc.close()
     return rows
@@ -812,7 +824,8 @@ def run_fragmentation(args):
                            "contiguous_reservation": f"{MAX_LEN[row['workload']]} tokens per sequence"},
                 "detail": row,
                 "note": "host control plane only (pa_block_alloc through the C ABI); the pool is the workload's "
-                        "1.25x-sized shuffled pool, so the free-page alarm (under 10 percent free) stays off"}
+                        "1.25x-sized shuffled pool, where the free-page alarm (under 10 percent free) stays off; "
+                        "tight_* repeat the trace in a pool that ends 5 percent free, where it fires"}
         print(json.dumps(line), flush=True)
     return 0
 

@@ -44,6 +44,7 @@ def test_fragmentation_rows_match_the_oracle_and_the_pages_bound():
         assert r["paged_waste_fraction"] == ref["waste_fraction"]
         assert r["physical_tokens"] == ref["physical_tokens"] and r["used_pages"] == ref["used_pages"]
         assert not r["low_free_alarm"]
+        assert r["tight_low_free_alarm"] and 0.04 < r["tight_free_fraction"] < 0.06
     ind = [r for r in rows if r["workload"] == "llama8b"]
     assert all(r["paged_waste_fraction"] < 0.04 < r["contiguous_waste_fraction"] for r in ind)
     beam = [r for r in rows if r["workload"] == "beam32k"]
