@@ -264,9 +264,13 @@ PA_API pa_status pa_decode_verify(const void* q, const void* key_cache, const vo
  * pa_decode_workspace_size(num_seqs, num_q_heads, head_dim,
  * max_blocks_per_seq * block_size) > PA_FIXED_SCRATCH_BYTES) returns
  * PA_ERR_INVALID without launching anything; use pa_decode for it.
- * The first call on each device does a one-time set-up (it looks up the
- * array's device address with that device current); make that first call
- * before any stream capture.  The call allocates nothing and frees nothing.
+ * The first accepted call in each device's context does a one-time set-up:
+ * it looks up the array's device address with that device current and
+ * caches it for that context (a context created again, e.g. after
+ * cudaDeviceReset, gets a fresh lookup on its first call).  Make that first
+ * call before any stream capture.  Calls with num_seqs == 0 and calls
+ * rejected for their sizes return before the set-up.  The call allocates
+ * nothing and frees nothing.
  * Every call shares the one array and leaves its contents behind; nothing in
  * it needs to start at zero (each call writes every partial it later reads),
  * but calls that overlap on the GPU (on different streams, or from several
@@ -324,19 +328,27 @@ PA_API pa_status pa_decode_shared_prefix(const void* q, const void* key_cache, c
                                          int32_t* dev_status, void* stream);
 
 /* Which joint kernel pa_decode_shared_prefix runs (process-wide; default
- * AUTO = TCGEN05): TCGEN05 is the pipelined persistent kernel on the 5th-
- * generation tensor cores (TMA loads, tcgen05.mma with Tensor Memory
- * accumulators, one CTA per SM); TCGEN05_2CTA the same pipeline in a leaner
- * form that runs two CTAs per SM; TCGEN05_SERIAL the one-partition-per-CTA
- * tcgen05 kernel without the software pipeline; MMA_SYNC the mma.sync
- * kernel.  All compute the same partials; the switch exists for testing and
- * measurement. */
+ * AUTO = TCGEN05).  TCGEN05 is the balanced persistent kernel on the 5th-
+ * generation tensor cores (one CTA per SM, cp.async loads into swizzled
+ * shared memory, tcgen05.mma with Tensor Memory accumulators): it covers the
+ * groups' shared partitions and also every member's own tokens, split evenly
+ * over the SMs in runs of 64-token steps, so a per-sequence kernel runs only
+ * for sequences outside every group; a run writes one partial per query row
+ * into the slot of the partition where it starts and marks the slots of the
+ * later partitions it covers empty (l = 0).  The other kernels compute the
+ * partials of each shared partition and leave the members' other partitions
+ * to the per-sequence kernel: TCGEN05_ITEMS the persistent per-partition
+ * tcgen05 kernel (TMA loads); TCGEN05_2CTA the same pipeline in a leaner form
+ * that runs two CTAs per SM; TCGEN05_SERIAL the one-partition-per-CTA tcgen05
+ * kernel without the software pipeline; MMA_SYNC the mma.sync kernel.  All
+ * give the same output; the switch exists for testing and measurement. */
 typedef enum pa_shared_prefix_kernel {
   PA_SHARED_PREFIX_AUTO = 0,
   PA_SHARED_PREFIX_TCGEN05 = 1,
   PA_SHARED_PREFIX_MMA_SYNC = 2,
   PA_SHARED_PREFIX_TCGEN05_SERIAL = 3,
-  PA_SHARED_PREFIX_TCGEN05_2CTA = 4
+  PA_SHARED_PREFIX_TCGEN05_2CTA = 4,
+  PA_SHARED_PREFIX_TCGEN05_ITEMS = 5
 } pa_shared_prefix_kernel;
 PA_API pa_status pa_set_shared_prefix_kernel(pa_shared_prefix_kernel kernel);
 

@@ -18,6 +18,7 @@ PA_DEV_TIMEOUT = 32
 PA_DECODE_AUTO, PA_DECODE_CUDA_CORES, PA_DECODE_TENSOR_CORES = 0, 1, 2
 PA_SHARED_PREFIX_AUTO, PA_SHARED_PREFIX_TCGEN05, PA_SHARED_PREFIX_MMA_SYNC, PA_SHARED_PREFIX_TCGEN05_SERIAL = 0, 1, 2, 3
 PA_SHARED_PREFIX_TCGEN05_2CTA = 4
+PA_SHARED_PREFIX_TCGEN05_ITEMS = 5
 PA_LOW_FREE_FRACTION = 0.10
 
 

@@ -16,7 +16,8 @@ import numpy as np
 from . import _lib
 from ._lib import (PA_BF16, PA_DECODE_AUTO, PA_DECODE_CUDA_CORES, PA_DECODE_TENSOR_CORES,  # noqa: F401
                    PA_DEV_TIMEOUT, PA_SHARED_PREFIX_AUTO, PA_SHARED_PREFIX_MMA_SYNC, PA_SHARED_PREFIX_TCGEN05,
-                   PA_SHARED_PREFIX_TCGEN05_SERIAL, PA_SHARED_PREFIX_TCGEN05_2CTA, PA_FAULT_NONE,
+                   PA_SHARED_PREFIX_TCGEN05_SERIAL, PA_SHARED_PREFIX_TCGEN05_2CTA,
+                   PA_SHARED_PREFIX_TCGEN05_ITEMS, PA_FAULT_NONE,
                    PA_FAULT_WITHHOLD_FIRST_ITEM, PA_VERIFY_AUTO, PA_VERIFY_JOINT, PA_VERIFY_PER_SEQUENCE,
                    PA_DEV_BAD_CTX, PA_DEV_BAD_PAGE, PA_DEV_BAD_PAIR, PA_DEV_BAD_PLAN, PA_DEV_BAD_SLOT, PA_ERR_NOT_FOUND,
                    PA_ERR_OOM, PA_F16, PA_F32, PA_PARTITION_TOKENS)

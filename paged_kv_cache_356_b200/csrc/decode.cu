@@ -40,6 +40,8 @@
 #include <math.h>
 
 #include <algorithm>
+#include <climits>
+#include <cstring>
 #include <atomic>
 #include <type_traits>
 #include <mutex>
@@ -71,6 +73,7 @@ struct DecodeArgs {
   float* l_part;
   int32_t* status;
   const int32_t* first_partition;  // optional: partitions [0, first) of b come from the shared-prefix kernel
+  int skip_members;                // with first_partition: sequences with first > 0 are left out entirely
   int partition_base;              // grid z of the partition kernels starts at this partition
   int max_blocks_per_seq;
   int num_q_heads;
@@ -154,6 +157,8 @@ struct AfterPrerequisiteGrid {
 template <typename T, int D, int GC, int NW>
 __global__ void __launch_bounds__(NW * 32) decode_cc_kernel(const DecodeArgs a) {
   const AfterPrerequisiteGrid after{threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0};
+  // A joint kernel launched after this one as a programmatic dependent may start now.
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   constexpr int VPL = D / 32;
   __shared__ float o_w[NW * GC * D];
   __shared__ float m_w[NW * GC];
@@ -172,7 +177,8 @@ __global__ void __launch_bounds__(NW * 32) decode_cc_kernel(const DecodeArgs a) 
   const int ctx = context_of(a, b, threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0);
   const int np = (ctx + kPartition - 1) / kPartition;
   if (p >= max(np, 1)) return;
-  if (a.first_partition && p < __ldg(a.first_partition + b)) return;
+  if (a.first_partition && (a.skip_members ? __ldg(a.first_partition + b) > 0 : p < __ldg(a.first_partition + b)))
+    return;
   if (ctx == 0) {
     store_zero_rows<T, D>(a, b, h0, nh);
     return;
@@ -279,6 +285,8 @@ struct TcShape {
 template <typename T, int D, int NW, int STAGES>
 __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(const DecodeArgs a) {
   const AfterPrerequisiteGrid after{threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0};
+  // A joint kernel launched after this one as a programmatic dependent may start now.
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   using S = TcShape<D, NW, STAGES>;
   constexpr int KSTEPS = D / 16;
   constexpr int MTILES = D / 16;
@@ -297,7 +305,8 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(const DecodeArgs a) 
   const int ctx = context_of(a, b, threadIdx.x == 0 && kvh == 0 && blockIdx.z == 0);
   const int np = (ctx + kPartition - 1) / kPartition;
   if (p >= max(np, 1)) return;
-  if (a.first_partition && p < __ldg(a.first_partition + b)) return;
+  if (a.first_partition && (a.skip_members ? __ldg(a.first_partition + b) > 0 : p < __ldg(a.first_partition + b)))
+    return;
   if (ctx == 0) {
     store_zero_rows<T, D>(a, b, h0, G);
     return;
@@ -1680,6 +1689,868 @@ __global__ void __launch_bounds__(Tc05pShape<D, STAGES>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Balanced shared-prefix kernel on tcgen05 (the default joint kernel).  One
+// persistent CTA per SM covers a share of the whole call:
+//   shared steps   the 64-token steps of every (kv head, chunk) lane that all of
+//                  the chunk's members share (its whole shared partitions), and
+//   tail steps     every (kv head, member) lane from the end of the member's
+//                  shared partitions to its context length.
+// Shared steps are split evenly over the CTAs in contiguous ranges (a range
+// may end in one lane and go on in the next); a tail lane goes whole to the
+// CTA whose range holds its start, weighed as its steps plus kEpilogueSteps
+// for its epilogue, so that the CTAs finish together and no per-sequence
+// kernel has to follow for the members.  A CTA's run of consecutive steps in
+// one lane is a segment: for each of its query rows it writes one partial
+// (o / l, m, l) into a workspace slot of the lane's partitions -- the k-th
+// segment of a lane takes the lane's k-th slot -- and the segment that ends
+// the lane writes l = 0 into the lane's slots left over, which the merge skips.
+// A lane has no more segments than partitions: CTA ranges are at least 16
+// steps long, and no range ends inside a lane of one partition.
+//
+// Roles (9 warps):
+//   warps 0-3       softmax: thread r owns query row r (TMEM lane r), as in the
+//                   per-partition kernel; a tail segment masks the tokens past
+//                   its member's context, and every step masks the 16-token
+//                   groups whose page is out of range (bits the producers
+//                   publish with the stage).
+//   warps 4-6, 8    producers: producer k loads 16-token group k of every step
+//                   -- its page's K and V slabs, 16-byte cp.async copies into
+//                   the 128-byte-swizzled stage, their completion tracked by the
+//                   stage's mbarrier -- with the page numbers of 32 steps held
+//                   one per lane (the next 32 already requested); three steps
+//                   before a segment ends they load the next segment's query
+//                   rows (one per lane), descriptor and workspace rows.
+//   warp 7          MMA issuer (one lane): S(g) = Q.K^T, then O += P(g-1).V(g-1).
+// Hand-offs, bounded waits, the abort path and the fault hook are those of
+// the per-partition kernel.
+// ---------------------------------------------------------------------------
+template <int D, int STAGES>
+struct SegShape {
+  // Four producer warps, one 16-token group of every step each (measured: seven,
+  // sharing every step's copies, were slower -- the softmax warps then share
+  // their schedulers with two producers each).
+  static constexpr int kProducerWarps = 4;
+  static constexpr int kMmaWarp = 7;
+  static constexpr int kThreads = 32 * 9;
+  static constexpr int kRows = 128;
+  static constexpr int kStep = 64;
+  static constexpr int kBlocks = D / 64;
+  static constexpr int kQBlockBytes = kRows * 128;
+  static constexpr int kQBytes = kBlocks * kQBlockBytes;
+  static constexpr int kKVBlockBytes = kStep * 128;
+  static constexpr int kTileBytes = kBlocks * kKVBlockBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kChunksPerRow = D / 8;         // 16-byte chunks of one K or V row
+  static constexpr int kRowsPerCopy = 32 / kChunksPerRow;  // rows one warp-wide copy covers
+  static constexpr int kCopiesPerGroup = 16 / kRowsPerCopy;
+
+  static constexpr int kQOff = 0;
+  static constexpr int kStageOff = 2 * kQBytes;
+  static constexpr int kDescOff = kStageOff + STAGES * kStageBytes;            // int32 [2][16]
+  static constexpr int kRowOff = kDescOff + 128;                               // int32 [2][kRows]
+  static constexpr int kBarOff = kRowOff + 2 * kRows * 4;
+  // s_full, p_full, o_done, q_full, item_free x2; kv_full, kv_empty x STAGES; mma_drain
+  static constexpr int kNumBars = 2 * 5 + 2 * STAGES + 1;
+  static constexpr int kTaddrOff = kBarOff + 8 * kNumBars;
+  static constexpr int kSmemBytes = kTaddrOff + 16 + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kSCol = 0, kPCol = 128, kOCol = 256;  // S[b] at 64b, P[b] at 128 + 32b, O[b] at 256 + 128b
+  static constexpr int kEpilogueSteps = 2;  // weight of a tail lane's epilogue, in steps
+  static_assert(D <= 128, "O double buffer needs D <= 128");
+  static_assert(kRows == 32 * 4, "one query row per lane of the first four producer warps");
+  static_assert(kStep == 16 * 4, "four 16-token groups per step");
+  static_assert(kQBytes >= 4 * 32 * 20 * 4, "the epilogue's four 32-row float tiles fit in a query buffer");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+  // Producer warp index of warp w (warps 4-6 and 8).
+  __host__ __device__ static constexpr int producer_of(int w) { return w < kMmaWarp ? w - 4 : w - 5; }
+};
+
+// Chunk c of a shared-prefix plan; an entry that would index outside an array
+// is reported (when `report`) and read as an empty chunk.
+struct SegChunk {
+  int leader, moff, mcount, sp;
+};
+__device__ __forceinline__ SegChunk seg_chunk(const DecodeArgs& a, const int32_t* __restrict__ chunks, int c,
+                                             int num_members, int num_seqs, bool report) {
+  SegChunk k{__ldg(chunks + 4 * c), __ldg(chunks + 4 * c + 1), __ldg(chunks + 4 * c + 2), __ldg(chunks + 4 * c + 3)};
+  const bool ok = (unsigned)k.leader < (unsigned)num_seqs && k.moff >= 0 && k.mcount >= 0 &&
+                  (int64_t)k.moff + k.mcount <= num_members && (int64_t)k.mcount * a.group <= 128 && k.sp >= 0 &&
+                  (int64_t)k.sp * kPartition <= (int64_t)a.max_blocks_per_seq * a.block_size &&
+                  k.sp <= a.max_partitions;
+  if (!ok) {
+    if (report) flag_status(a.status, PA_DEV_BAD_PLAN);
+    k.mcount = 0;
+  }
+  if (k.mcount == 0) k.sp = 0;
+  return k;
+}
+
+// A segment: steps [s0, s1) of one lane.  kind 0 = shared (rows: the chunk's
+// members), 1 = tail (rows: member `b`); `leader` is the sequence whose block
+// table gives the pages; tokens at or past `ctx` are masked.  Its partial goes
+// to workspace slot `slot`; slots [slot + 1, mark_end) are marked empty.
+struct Seg {
+  int kind, kvh, leader, moff, mcount, b, s0, s1, ctx, slot, mark_end;
+};
+
+// The segments of one CTA, in order.  Every lane of a producer warp runs the
+// same walk (warp-uniform results); every producer warp runs its own copy.
+// All unit counts stay below kSegMaxUnits (the launcher checks an upper bound),
+// so the walk runs in 32-bit arithmetic: total * k for k <= 148 CTAs fits.
+constexpr int kSegMaxUnits = 1 << 23;
+struct SegWalk {
+  int u0, u1;          // this CTA's range of weighted units
+  int total;           // units of the whole call
+  int ctas;            // CTAs with a range
+  int base;            // units of all shared lanes: H_kv * S_sh
+  int s_sh, tw;        // shared steps per kv head; tail weight per kv head
+  // shared lanes
+  int su, su_end;      // next shared unit, end of this CTA's shared units
+  int skvh, sc, soff;  // lane (kv head, chunk) of unit su and its offset in the lane
+  SegChunk sci;
+  SegChunk cl;         // plans of at most 32 chunks: chunk `lane` of this lane
+  int cl_incl;         // and the lanes' units of chunks 0 .. lane
+  // tail lanes: sequences [tm0, tm0 + 32) of kv head tkvh, weighted start tw_at
+  int tkvh, tm0;
+  int tw_at;
+  uint32_t tmask;      // members of the loaded batch still to hand out
+  bool tloaded, tdone;
+  int tT, tfp, tctx;      // per lane: tail steps, first tail partition and context of sequence tm0 + lane
+};
+
+// Tail of batch sequence b: its steps from the end of its shared partitions
+// to its context (0 for a sequence outside every group), first tail partition
+// and context.
+__device__ __forceinline__ void seg_tail_of(const DecodeArgs& a, const int32_t* __restrict__ first_partition, int b,
+                                            int num_seqs, int& T, int& fp, int& ctx) {
+  T = 0;
+  fp = 0;
+  ctx = 0;
+  if (b < num_seqs) {
+    fp = __ldg(first_partition + b);
+    ctx = context_of(a, b, false);
+    if (fp <= 0 || fp > a.max_partitions) fp = 0;
+    else T = max(0, (ctx + 63) / 64 - 8 * fp);
+  }
+}
+
+// Warp-wide inclusive sum.
+__device__ __forceinline__ int warp_incl_sum(int v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(kFull, v, off);
+    if (lane >= off) v += o;
+  }
+  return v;
+}
+
+// Units of shared lane (kv head, c): kSegLeadIn units that carry no step (the
+// cost of starting a segment: the previous one's epilogue and the switch of
+// query rows), then one unit per 64-token step of the chunk's shared partitions.
+constexpr int kSegLeadIn = 3;
+__device__ __forceinline__ int seg_lane_units(int sp) { return sp > 0 ? 8 * sp + kSegLeadIn : 0; }
+
+// Chunk c of the plan from the lane registers of the walk (plans of at most 32
+// chunks: lane c holds chunk c) or from global memory.
+__device__ __forceinline__ SegChunk seg_chunk_of(const SegWalk& w, int c, const DecodeArgs& a,
+                                                 const int32_t* __restrict__ chunks, int num_chunks,
+                                                 int num_members, int num_seqs) {
+  if (num_chunks <= 32) {
+    return SegChunk{__shfl_sync(kFull, w.cl.leader, c), __shfl_sync(kFull, w.cl.moff, c),
+                    __shfl_sync(kFull, w.cl.mcount, c), __shfl_sync(kFull, w.cl.sp, c)};
+  }
+  return seg_chunk(a, chunks, c, num_members, num_seqs, false);
+}
+
+// Lane (kv head, chunk), unit offset within the lane and the chunk's shared
+// partitions of shared unit u (warp-collective; u < H_kv * s_sh).
+__device__ __forceinline__ void seg_locate(const SegWalk& w, int u, const DecodeArgs& a,
+                                           const int32_t* __restrict__ chunks, int num_chunks, int num_members,
+                                           int num_seqs, int& kvh, int& c, int& off, int& sp) {
+  const int lane = threadIdx.x & 31;
+  kvh = u / w.s_sh;
+  int r = u - kvh * w.s_sh;
+  c = 0;
+  off = 0;
+  sp = 0;
+  for (int c0 = 0; c0 < num_chunks; c0 += 32) {
+    int n, incl;
+    if (num_chunks <= 32) {
+      n = seg_lane_units(w.cl.sp);
+      incl = w.cl_incl;
+    } else {
+      const int cc = c0 + lane;
+      n = cc < num_chunks ? seg_lane_units(seg_chunk(a, chunks, cc, num_members, num_seqs, false).sp) : 0;
+      incl = warp_incl_sum(n);
+    }
+    const uint32_t hit = __ballot_sync(kFull, incl > r);
+    if (hit) {
+      const int l = __ffs(hit) - 1;
+      const int nl = __shfl_sync(kFull, n, l);
+      c = c0 + l;
+      off = r - (__shfl_sync(kFull, incl, l) - nl);
+      sp = (nl - kSegLeadIn) / 8;
+      return;
+    }
+    r -= __shfl_sync(kFull, incl, 31);
+  }
+}
+
+// Start of CTA k's range: total * k / ctas, except that a range never ends
+// inside the steps of a lane of one partition (such a cut moves to the nearer
+// end of them).
+__device__ __forceinline__ int seg_cut(const SegWalk& w, int k, const DecodeArgs& a,
+                                       const int32_t* __restrict__ chunks, int num_chunks, int num_members,
+                                       int num_seqs) {
+  int u = (int)((unsigned)w.total * (unsigned)k / (unsigned)w.ctas);
+  if (u < w.base && w.s_sh > 0) {
+    int kvh, c, off, sp;
+    seg_locate(w, u, a, chunks, num_chunks, num_members, num_seqs, kvh, c, off, sp);
+    const int step = off - kSegLeadIn;
+    if (sp == 1 && step > 0) u += step < 4 ? -step : 8 - step;
+  }
+  return u;
+}
+
+template <int E>
+__device__ __forceinline__ void seg_walk_init(SegWalk& w, const DecodeArgs& a, const int32_t* __restrict__ chunks,
+                                              int num_chunks, const int32_t* __restrict__ members, int num_members,
+                                              const int32_t* __restrict__ first_partition, int num_seqs, bool report) {
+  const int lane = threadIdx.x & 31;
+  // Shared units per kv head and the tail weight per kv head.  The chunk, member
+  // and sequence loads of one pass are independent (one round trip); plans of up
+  // to 32 chunks keep their chunks in lane registers.
+  if (lane < num_members) asm volatile("prefetch.global.L1 [%0];\n" ::"l"(members + lane));
+  int s_sh = 0, tw = 0;
+  w.cl = SegChunk{0, 0, 0, 0};
+  w.cl_incl = 0;
+  for (int i0 = 0; i0 < num_chunks || i0 < num_seqs; i0 += 32) {
+    const int i = i0 + lane;
+    const SegChunk ci = i < num_chunks ? seg_chunk(a, chunks, i, num_members, num_seqs, report) : SegChunk{0, 0, 0, 0};
+    const int n = seg_lane_units(ci.sp);
+    int T, fp, ctx;
+    seg_tail_of(a, first_partition, i, num_seqs, T, fp, ctx);
+    const int incl = warp_incl_sum(n);
+    if (i0 == 0) {
+      w.cl = ci;
+      w.cl_incl = incl;
+    }
+    s_sh += __shfl_sync(kFull, incl, 31);
+    tw += __shfl_sync(kFull, warp_incl_sum(T > 0 ? T + E : 0), 31);
+  }
+  w.s_sh = s_sh;
+  w.tw = tw;
+  w.base = a.num_kv_heads * s_sh;
+  w.total = w.base + a.num_kv_heads * tw;
+  // Every range spans at least 16 units; CTAs past the last range get none.
+  w.ctas = w.total / 16;
+  if (w.ctas < 1) w.ctas = 1;
+  if (w.ctas > gridDim.x) w.ctas = gridDim.x;
+  if ((int)blockIdx.x < w.ctas) {
+    w.u0 = seg_cut(w, blockIdx.x, a, chunks, num_chunks, num_members, num_seqs);
+    w.u1 = blockIdx.x + 1 == w.ctas ? w.total : seg_cut(w, blockIdx.x + 1, a, chunks, num_chunks, num_members, num_seqs);
+  } else {
+    w.u0 = w.u1 = w.total;
+  }
+  // Shared cursor: lane (kv head, chunk) and unit offset of unit u0.
+  w.su = w.su_end = 0;
+  w.skvh = w.sc = w.soff = 0;
+  w.sci = SegChunk{0, 0, 0, 0};
+  if (w.u0 < w.base && s_sh > 0) {
+    w.su = w.u0;
+    w.su_end = w.u1 < w.base ? w.u1 : w.base;
+    int sp;
+    seg_locate(w, w.u0, a, chunks, num_chunks, num_members, num_seqs, w.skvh, w.sc, w.soff, sp);
+    w.sci = seg_chunk_of(w, w.sc, a, chunks, num_chunks, num_members, num_seqs);
+  }
+  // Tail cursor: the first kv head whose tail lanes can start in [u0, u1).
+  w.tdone = !(tw > 0 && w.u1 > w.base && w.u1 > w.u0);
+  w.tkvh = (!w.tdone && w.u0 > w.base) ? (w.u0 - w.base) / tw : 0;
+  w.tm0 = 0;
+  w.tw_at = w.base + w.tkvh * tw;
+  w.tmask = 0;
+  w.tloaded = false;
+  w.tT = w.tfp = w.tctx = 0;
+}
+
+template <int E>
+__device__ __forceinline__ bool seg_walk_next(SegWalk& w, Seg& s, const DecodeArgs& a,
+                                              const int32_t* __restrict__ chunks, int num_chunks,
+                                              const int32_t* __restrict__ members, int num_members,
+                                              const int32_t* __restrict__ first_partition, int num_seqs) {
+  const int lane = threadIdx.x & 31;
+  while (w.su < w.su_end) {
+    const int units = seg_lane_units(w.sci.sp);
+    const int len = 8 * w.sci.sp;
+    const int lane0 = w.su - w.soff;
+    const int off1 = units - w.soff < w.su_end - w.su ? units : w.soff + (w.su_end - w.su);
+    const int s0 = max(0, w.soff - kSegLeadIn), s1 = max(0, off1 - kSegLeadIn);
+    w.su += off1 - w.soff;
+    w.soff = off1;
+    const int kvh = w.skvh;
+    const SegChunk ci = w.sci;
+    if (w.soff == units && w.su < w.su_end) {  // on to the next non-empty lane
+      do {
+        if (++w.sc == num_chunks) {
+          w.sc = 0;
+          ++w.skvh;
+        }
+        w.sci = seg_chunk_of(w, w.sc, a, chunks, num_chunks, num_members, num_seqs);
+      } while (w.sci.sp == 0 && w.skvh < a.num_kv_heads);
+      w.soff = 0;
+    }
+    if (s1 <= s0) continue;  // the range held only lead-in units of this lane
+    // Slot: 0 for the segment with the lane's first step; a segment that starts
+    // after it starts this CTA's range, and the CTAs from the one holding the
+    // lane's first step up to this one each began one segment of the lane before.
+    int slot = 0;
+    if (s0 > 0) {
+      const int first = lane0 + kSegLeadIn;
+      slot = (int)blockIdx.x - (int)(((unsigned)w.ctas * (unsigned)(first + 1) - 1u) / (unsigned)w.total);
+    }
+    const int mark_end = s1 == len ? ci.sp : slot + 1;
+    s = Seg{0, kvh, ci.leader, ci.moff, ci.mcount, -1, s0, s1, INT_MAX, slot, mark_end};
+    return true;
+  }
+  while (true) {
+    if (w.tmask) {
+      const int l = __ffs(w.tmask) - 1;
+      w.tmask &= w.tmask - 1;
+      const int T = __shfl_sync(kFull, w.tT, l), b = w.tm0 + l;
+      const int fp = __shfl_sync(kFull, w.tfp, l), ctx = __shfl_sync(kFull, w.tctx, l);
+      s = Seg{1, w.tkvh, b, 0, 1, b, 8 * fp, 8 * fp + T, ctx, fp, (ctx + kPartition - 1) / kPartition};
+      return true;
+    }
+    if (w.tdone) return false;
+    if (w.tloaded) {  // the loaded batch is handed out: the next one
+      w.tloaded = false;
+      w.tm0 += 32;
+      if (w.tm0 >= num_seqs) {
+        w.tm0 = 0;
+        if (++w.tkvh >= a.num_kv_heads) {
+          w.tdone = true;
+          return false;
+        }
+      }
+    }
+    if (w.tw_at >= w.u1) {
+      w.tdone = true;
+      return false;
+    }
+    seg_tail_of(a, first_partition, w.tm0 + lane, num_seqs, w.tT, w.tfp, w.tctx);
+    const int wt = w.tT > 0 ? w.tT + E : 0;
+    const int incl = warp_incl_sum(wt);
+    const int start = w.tw_at + incl - wt;
+    w.tmask = __ballot_sync(kFull, wt > 0 && start >= w.u0 && start < w.u1);
+    w.tw_at += __shfl_sync(kFull, incl, 31);
+    w.tloaded = true;
+  }
+}
+
+template <typename T, int D, int STAGES>
+__global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
+    decode_shared_seg_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k, int tma_k,
+                             const int32_t* __restrict__ chunks, int num_chunks,
+                             const int32_t* __restrict__ members, int num_members,
+                             const int32_t* __restrict__ first_partition, int num_seqs, int fault) {
+  using S = SegShape<D, STAGES>;
+  constexpr int E = S::kEpilogueSteps;
+  extern __shared__ uint8_t smem_raw[];
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int bs = a.block_size;
+  const int G = a.group;
+
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  // Written by the producers, published with q_full: the segment in buffer b
+  // -- [0] valid (0 ends the walk), [1] kv head, [2] s0, [3] s1, [4] rows,
+  // [5] context limit, [6] slot, [7] end of the slots marked empty, [8] the
+  // sequence whose table gives the pages, [9 + k] bit i: 16-token group k of
+  // step s0 + i is on an out-of-range page (i < 32) -- and the workspace row
+  // base of each of its query rows (-1: none).
+  volatile int32_t* desc = reinterpret_cast<volatile int32_t*>(base_ptr + S::kDescOff);  // [2][16]
+  int32_t* prow_s = reinterpret_cast<int32_t*>(base_ptr + S::kRowOff);                   // [2][kRows]
+  const uint32_t bar0 = base + S::kBarOff;
+  auto s_full = [&](int b) { return bar0 + 8u * b; };
+  auto p_full = [&](int b) { return bar0 + 16u + 8u * b; };
+  auto o_done = [&](int b) { return bar0 + 32u + 8u * b; };
+  auto q_full = [&](int b) { return bar0 + 48u + 8u * b; };
+  auto item_free = [&](int b) { return bar0 + 64u + 8u * b; };
+  auto kv_full = [&](int st) { return bar0 + 80u + 8u * st; };
+  auto kv_empty = [&](int st) { return bar0 + 80u + 8u * STAGES + 8u * st; };
+  const uint32_t mma_drain = bar0 + 80u + 16u * STAGES;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + S::kTaddrOff + 8);
+  const uint32_t taddr_slot = base + S::kTaddrOff;
+
+  auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    const long long t0 = clock64();
+    while (!tc05::mbar_try_wait_sleep(bar, parity, 20000u)) {
+      if (*abort_flag) return false;
+      if (clock64() - t0 > kWaitCycles) {
+        *abort_flag = 1;
+        return false;
+      }
+    }
+    return true;
+  };
+  auto wwait = [&](uint32_t bar, uint32_t parity) -> bool { return __all_sync(kFull, wait(bar, parity)); };
+
+  // The producers' walk of the plan and their first page windows do not touch
+  // shared memory: their global loads start before the set-up below.
+  const bool producer = warp >= 4 && warp != S::kMmaWarp;
+  const int pw = producer ? S::producer_of(warp) : 0;  // group pw of every step; query rows 32 pw + lane
+  SegWalk walk;
+  Seg seg, nxt;
+  bool have = false, have_nxt = false;
+  // Page of group pw of step w0 + lane of segment s, -1 outside the segment or the table.
+  auto window = [&](const Seg& s, int w0) -> int {
+    const int64_t tok = 64 * (int64_t)(w0 + lane) + 16 * pw;
+    const int64_t blk = tok / bs;
+    return (w0 + lane < s.s1 && tok < s.ctx && blk < a.max_blocks_per_seq)
+               ? __ldg(a.block_tables + (int64_t)s.leader * a.max_blocks_per_seq + blk)
+               : -1;
+  };
+  auto next_seg = [&](Seg& s) {
+    return seg_walk_next<E>(walk, s, a, chunks, num_chunks, members, num_members, first_partition, num_seqs);
+  };
+  // The segment after the current one is known, and its first page windows are
+  // requested, as soon as the current one starts: its query rows are loaded
+  // three steps before the current one ends without waiting for the table.
+  int win_cur = -1, win_nxt = -1, nxt_cur = -1, nxt_nxt = -1;
+  if (producer) {
+    seg_walk_init<E>(walk, a, chunks, num_chunks, members, num_members, first_partition, num_seqs,
+                     pw == 0 && lane == 0 && blockIdx.x == 0);
+    have = next_seg(seg);
+    if (have) {
+      win_cur = window(seg, seg.s0);
+      win_nxt = window(seg, seg.s0 + 32);
+    }
+    have_nxt = have && next_seg(nxt);
+    nxt_cur = have_nxt ? window(nxt, nxt.s0) : -1;
+    nxt_nxt = have_nxt ? window(nxt, nxt.s0 + 32) : -1;
+  }
+
+  // -- set-up -----------------------------------------------------------------------------------
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b) {
+      tc05::mbar_init(s_full(b), 1);
+      tc05::mbar_init(p_full(b), 4);
+      tc05::mbar_init(o_done(b), 1);
+      tc05::mbar_init(q_full(b), S::kProducerWarps);  // lane 0 of each producer warp (+ their copies)
+      tc05::mbar_init(item_free(b), 4);
+    }
+    for (int st = 0; st < STAGES; ++st) {
+      tc05::mbar_init(kv_full(st), S::kProducerWarps);
+      tc05::mbar_init(kv_empty(st), 1);
+    }
+    tc05::mbar_init(mma_drain, 1);
+    *abort_flag = 0;
+    tc05::fence_mbar_init();
+    if (tma_k) tc05::prefetch_tensormap(&tmap_k);
+  }
+  if (warp == 0) {
+    tc05::alloc(taddr_slot, S::kTmemCols);
+    tc05::relinquish();
+  }
+  tc05::fence_before();
+  __syncthreads();
+  tc05::fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base_ptr + S::kTaddrOff);
+
+  // The merge that follows may be launched now (it waits for this grid).
+  if (tid == 0) asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  if (producer) {
+    // ---------------------------------------------------------------- producers
+    const T* qbase = reinterpret_cast<const T*>(a.q);
+    const T* kcache = reinterpret_cast<const T*>(a.key_cache);
+    const T* vcache = reinterpret_cast<const T*>(a.value_cache);
+    // Query rows of segment s into buffer qb, its workspace row bases, and its
+    // descriptor (producer pw: the out-of-range pages of group pw in the first 32
+    // steps, from `win`); q_full(qb) completes once every producer has arrived and
+    // the copies have landed.
+    auto load_q = [&](const Seg& s, int qb, int win) {
+      {
+        const uint32_t qs = base + S::kQOff + qb * S::kQBytes;
+        const int r = pw * 32 + lane;
+        const int nrows = s.mcount * G;
+        int64_t row = -1;
+        if (r < nrows) {
+          const int mi = r / G;
+          const int b = s.kind == 0 ? __ldg(members + s.moff + mi) : s.b;
+          if ((unsigned)b < (unsigned)num_seqs) row = (int64_t)b * a.num_q_heads + s.kvh * G + (r - mi * G);
+          else flag_status(a.status, PA_DEV_BAD_PLAN);
+        }
+        const T* src = qbase + (row < 0 ? 0 : row) * D;
+#pragma unroll
+        for (int ck = 0; ck < D / 8; ++ck)
+          cp_async_16(qs + (ck >> 3) * S::kQBlockBytes + r * 128 + (((ck & 7) ^ (r & 7)) << 4), src + ck * 8,
+                      row < 0 ? 0u : 16u);
+        prow_s[qb * S::kRows + r] = row < 0 ? -1 : (int32_t)(row * a.max_partitions);
+        tc05::cp_async_arrive(q_full(qb));
+        const int64_t tok = 64 * (int64_t)(s.s0 + lane) + 16 * pw;
+        const uint32_t bad = __ballot_sync(kFull, s.s0 + lane < s.s1 && tok < s.ctx &&
+                                                      (unsigned)win >= (unsigned)a.num_blocks);
+        if (lane == 0) desc[qb * 16 + 9 + pw] = (int32_t)bad;
+        if (pw == 0 && lane == 0) {
+          desc[qb * 16 + 1] = s.kvh;
+          desc[qb * 16 + 2] = s.s0;
+          desc[qb * 16 + 3] = s.s1;
+          desc[qb * 16 + 4] = nrows;
+          desc[qb * 16 + 5] = s.ctx;
+          desc[qb * 16 + 6] = s.slot;
+          desc[qb * 16 + 7] = s.mark_end;
+          desc[qb * 16 + 8] = s.leader;
+          desc[qb * 16 + 0] = 1;
+        }
+      }
+    };
+    auto end_walk = [&](int qb) {  // buffer qb holds no segment: the other roles stop there
+      if (pw == 0 && lane == 0) desc[qb * 16 + 0] = 0;
+    };
+    auto publish_q = [&](int qb) {
+      __syncwarp();
+      if (lane == 0) tc05::mbar_arrive(q_full(qb));
+    };
+    if (have) load_q(seg, 0, win_cur);
+    else end_walk(0);
+    if (fault != PA_FAULT_WITHHOLD_FIRST_ITEM) publish_q(0);  // test hook: the other roles' waits run out
+    int64_t g = 0;
+    bool stop = false;
+    for (int j = 0; have && !stop; ++j) {
+      const int qb = j & 1;
+      const int len = seg.s1 - seg.s0;
+      const int qload_at = len > 3 ? len - 3 : 0;
+      int w0 = seg.s0;
+      for (int i = 0; i < len; ++i, ++g) {
+        const int step = seg.s0 + i;
+        if (step - w0 == 32) {
+          w0 += 32;
+          win_cur = win_nxt;
+          win_nxt = window(seg, w0 + 32);
+        }
+        const int st = (int)(g % STAGES);
+        if (g >= STAGES && !wwait(kv_empty(st), (uint32_t)(((g - STAGES) / STAGES) & 1))) { stop = true; break; }
+        const int page = __shfl_sync(kFull, win_cur, step - w0);
+        const int tok = 64 * step + 16 * pw;
+        const bool page_ok = (unsigned)page < (unsigned)a.num_blocks;
+        if (lane == 0 && tok < seg.ctx && !page_ok) flag_status(a.status, PA_DEV_BAD_PAGE);
+        const int64_t slab = ((int64_t)(page_ok ? page : 0) * a.num_kv_heads + seg.kvh) * bs + tok % bs;
+        const uint32_t stage = base + S::kStageOff + st * S::kStageBytes;
+        // V (and K without the tensor map): 16-byte cp.async copies, zero past the
+        // context and on an out-of-range page; their completion joins the stage's
+        // phase before this warp's arrival below.
+#pragma unroll
+        for (int kv = 0; kv < 2; ++kv) {
+          if (kv == 0 && tma_k) continue;
+          const T* cache = kv ? vcache : kcache;
+#pragma unroll
+          for (int i2 = 0; i2 < S::kCopiesPerGroup; ++i2) {
+            const int rl = i2 * S::kRowsPerCopy + lane / S::kChunksPerRow;  // row within the group
+            const int ck = lane % S::kChunksPerRow;
+            const int row = 16 * pw + rl;                                    // row within the step
+            const bool valid = page_ok && tok + rl < seg.ctx;
+            const T* src = cache + (valid ? (slab + rl) * D + ck * 8 : 0);
+            const uint32_t dst = stage + kv * S::kTileBytes + (ck >> 3) * S::kKVBlockBytes + row * 128 +
+                                 (((ck & 7) ^ (row & 7)) << 4);
+            cp_async_16(dst, src, valid ? 16u : 0u);
+          }
+        }
+        tc05::cp_async_arrive(kv_full(st));
+        __syncwarp();
+        if (lane == 0) {
+          if (tma_k) {
+            // K by the tensor-memory-access unit: one 16-row box per 64-column block
+            // (an out-of-range page loads as zeros; rows past the context are masked
+            // by the softmax).  The arrival announces the bytes before the copies start.
+            tc05::mbar_arrive_expect_tx(kv_full(st), S::kBlocks * 16 * 128);
+            const int32_t y = page_ok ? (int32_t)slab : (int32_t)((int64_t)a.num_blocks * a.num_kv_heads * bs);
+#pragma unroll
+            for (int blk = 0; blk < S::kBlocks; ++blk)
+              tc05::tma_load_2d(stage + blk * S::kKVBlockBytes + 16 * pw * 128, &tmap_k, kv_full(st), 64 * blk, y);
+          } else {
+            tc05::mbar_arrive(kv_full(st));
+          }
+        }
+        // Three steps before the end: the next segment's queries go into the other
+        // buffer once the segment that last used it (j - 1) has been read out.
+        if (i == qload_at) {
+          if (j >= 1 && !wwait(item_free(qb ^ 1), (uint32_t)(((j - 1) >> 1) & 1))) { stop = true; break; }
+          if (have_nxt) load_q(nxt, qb ^ 1, nxt_cur);
+          else end_walk(qb ^ 1);
+          publish_q(qb ^ 1);
+        }
+      }
+      if (stop || __any_sync(kFull, *abort_flag != 0)) break;
+      seg = nxt;
+      have = have_nxt;
+      win_cur = nxt_cur;
+      win_nxt = nxt_nxt;
+      have_nxt = have && next_seg(nxt);
+      nxt_cur = have_nxt ? window(nxt, nxt.s0) : -1;
+      nxt_nxt = have_nxt ? window(nxt, nxt.s0 + 32) : -1;
+    }
+    tc05::cp_async_wait_all();  // nothing may land in shared memory after the CTA leaves
+  } else if (warp == S::kMmaWarp) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+      constexpr uint32_t idesc_s = tc05::instr_desc_f16(fmt, S::kRows, S::kStep, 0, 0);
+      constexpr uint32_t idesc_o = tc05::instr_desc_f16(fmt, S::kRows, D, 0, 1);
+      auto mma2 = [&](int64_t gp, int j, bool first) -> bool {  // O[segment j] (+)= P(gp) . V(gp)
+        if (!wait(p_full((int)(gp & 1)), (uint32_t)((gp >> 1) & 1))) return false;
+        tc05::fence_after();
+        const int st = (int)(gp % STAGES);
+        const uint32_t vs = base + S::kStageOff + st * S::kStageBytes + S::kTileBytes;
+        const uint32_t ocol = S::kOCol + 128u * (uint32_t)(j & 1);
+#pragma unroll
+        for (int kt = 0; kt < S::kStep / 16; ++kt)
+          tc05::mma_ts(tmem + ocol, tmem + S::kPCol + 32 * (uint32_t)(gp & 1) + 8 * kt,
+                       tc05::smem_desc_sw128(vs + kt * 16 * 128, S::kKVBlockBytes, 1024), idesc_o,
+                       (!first || kt > 0) ? 1u : 0u);
+        tc05::commit(o_done((int)(gp & 1)));
+        tc05::commit(kv_empty(st));
+        return true;
+      };
+      int64_t g = 0;
+      bool ok = true;
+      for (int j = 0; ok; ++j) {
+        const int qb = j & 1;
+        if (!wait(q_full(qb), (uint32_t)((j >> 1) & 1))) break;
+        if (desc[qb * 16 + 0] == 0) break;  // the walk has ended
+        const int len = desc[qb * 16 + 3] - desc[qb * 16 + 2];
+        tc05::fence_after();
+        tc05::fence_proxy_async_smem();
+        const uint32_t qs = base + S::kQOff + qb * S::kQBytes;
+        for (int i = 0; i < len; ++i, ++g) {
+          const int st = (int)(g % STAGES);
+          // S buffer g & 1 is free: this thread has seen p_full(g - 2), which the softmax
+          // raises after reading S(g - 2).
+          if (!wait(kv_full(st), (uint32_t)((g / STAGES) & 1))) { ok = false; break; }
+          tc05::fence_after();
+          tc05::fence_proxy_async_smem();  // the stage's cp.async writes, for the tensor cores
+          const uint32_t ks = base + S::kStageOff + st * S::kStageBytes;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t blk = k >> 2, koff = (k & 3) * 32;
+            tc05::mma_ss(tmem + S::kSCol + 64 * (uint32_t)(g & 1),
+                         tc05::smem_desc_sw128(qs + blk * S::kQBlockBytes + koff, 16, 1024),
+                         tc05::smem_desc_sw128(ks + blk * S::kKVBlockBytes + koff, 16, 1024), idesc_s,
+                         k > 0 ? 1u : 0u);
+          }
+          tc05::commit(s_full((int)(g & 1)));
+          if (i >= 1 && !mma2(g - 1, j, i == 1)) { ok = false; break; }
+        }
+        // Close the segment (its epilogue must not wait for the next segment's queries).
+        if (ok && !mma2(g - 1, j, len == 1)) ok = false;
+      }
+      tc05::commit(mma_drain);
+      {
+        const long long t0 = clock64();
+        while (!tc05::mbar_try_wait(mma_drain, 0) && clock64() - t0 < kWaitCycles) {
+        }
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax warps 0-3
+    const uint32_t row_t = tmem + ((uint32_t)(32 * warp) << 16);
+    int64_t g = 0;
+    for (int j = 0;; ++j) {
+      const int qb = j & 1;
+      if (!wwait(q_full(qb), (uint32_t)((j >> 1) & 1))) break;  // segment, rows and descriptor
+      if (desc[qb * 16 + 0] == 0) break;                          // the walk has ended
+      const int s0 = desc[qb * 16 + 2], s1 = desc[qb * 16 + 3];
+      const int nrows = desc[qb * 16 + 4], ctx = desc[qb * 16 + 5];
+      const int slot = desc[qb * 16 + 6], mark_end = desc[qb * 16 + 7], leader = desc[qb * 16 + 8];
+      const bool busy = 32 * warp < nrows;
+      // Out-of-range pages: bit i of bad_w[k] is group k of step mw0 + i.  The
+      // producers publish the first 32 steps; later windows of 32 steps are
+      // requested one window ahead (page of group k of step mw0 + 32 + lane).
+      uint32_t bad_w[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) bad_w[q] = (uint32_t)desc[qb * 16 + 9 + q];
+      int mw0 = s0;
+      int pre[4];
+      auto request = [&](int w0) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int st_ = w0 + lane;
+          const int64_t tok = 64 * (int64_t)st_ + 16 * q;
+          const int64_t blk = tok / bs;
+          pre[q] = (st_ < s1 && tok < ctx && blk < a.max_blocks_per_seq)
+                       ? __ldg(a.block_tables + (int64_t)leader * a.max_blocks_per_seq + blk)
+                       : 0;
+        }
+      };
+      if (s1 > s0 + 32) request(s0 + 32);
+      float m_use = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int step = s0; step < s1; ++step, ++g) {
+        if (step == mw0 + 32) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) bad_w[q] = __ballot_sync(kFull, (unsigned)pre[q] >= (unsigned)a.num_blocks);
+          mw0 += 32;
+          if (s1 > mw0 + 32) request(mw0 + 32);
+        }
+        if (!wwait(s_full((int)(g & 1)), (uint32_t)((g >> 1) & 1))) { ok = false; break; }
+        tc05::fence_after();
+        uint32_t sreg[2][32];
+        if (busy) {
+          tc05::ld32(row_t + S::kSCol + 64 * (uint32_t)(g & 1), sreg[0]);
+          tc05::ld32(row_t + S::kSCol + 64 * (uint32_t)(g & 1) + 32, sreg[1]);
+          tc05::wait_ld();
+        }
+        const int sh = step - mw0;
+        const int bad = (int)(((bad_w[0] >> sh) & 1u) | (((bad_w[1] >> sh) & 1u) << 1) |
+                              (((bad_w[2] >> sh) & 1u) << 2) | (((bad_w[3] >> sh) & 1u) << 3));
+        const int lim = ctx - 64 * step;  // tokens of this step inside the context
+        uint32_t pk[32];
+        float alpha = 1.f;
+        if (busy) {
+          float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          float nref;
+          if (bad == 0 && lim >= 64 && a.qk_scale_log2 > 0.f) {
+#pragma unroll
+            for (int e = 0; e < 64; ++e) mx4[e & 3] = fmaxf(mx4[e & 3], __uint_as_float(sreg[e >> 5][e & 31]));
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * a.qk_scale_log2;
+            if (mx > m_use + 8.f) {
+              alpha = m_use == -INFINITY ? 0.f : ex2_approx(m_use - mx);
+              m_use = mx;
+            }
+            nref = -m_use;
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            // Every score is finite here: half the weights on the special-function
+            // unit, half on the FMA pipe, which the softmax otherwise leaves idle.
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+              const int e0 = 2 * jj, e1 = 2 * jj + 1;
+              const float p0 = ex2_approx(fmaf(__uint_as_float(sreg[e0 >> 5][e0 & 31]), a.qk_scale_log2, nref));
+              const float p1 = exp2_poly(fmaf(__uint_as_float(sreg[e1 >> 5][e1 & 31]), a.qk_scale_log2, nref));
+              ls[jj & 3] += p0 + p1;
+              pk[jj] = pack2<T>(p0, p1);
+            }
+            l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+          } else {
+            // Tokens past the context or on an out-of-range page have score -inf (weight 0).
+#pragma unroll
+            for (int e = 0; e < 64; ++e) {
+              const bool masked = e >= lim || ((bad >> (e >> 4)) & 1);
+              const float v = masked ? -INFINITY : __uint_as_float(sreg[e >> 5][e & 31]) * a.qk_scale_log2;
+              sreg[e >> 5][e & 31] = __float_as_uint(v);
+              mx4[e & 3] = fmaxf(mx4[e & 3], v);
+            }
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            if (mx > m_use + 8.f) {
+              alpha = m_use == -INFINITY ? 0.f : ex2_approx(m_use - mx);
+              m_use = mx;
+            }
+            nref = m_use == -INFINITY ? 0.f : -m_use;
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+              const int e0 = 2 * jj, e1 = 2 * jj + 1;
+              const float p0 = ex2_approx(__uint_as_float(sreg[e0 >> 5][e0 & 31]) + nref);
+              const float p1 = ex2_approx(__uint_as_float(sreg[e1 >> 5][e1 & 31]) + nref);
+              ls[jj & 3] += p0 + p1;
+              pk[jj] = pack2<T>(p0, p1);
+            }
+            l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+          }
+        }
+        if (busy && step > s0 && __any_sync(kFull, alpha != 1.f)) {
+          // O is current once O += P.V of step g - 1 has completed.
+          if (!wwait(o_done((int)((g - 1) & 1)), (uint32_t)(((g - 1) >> 1) & 1))) { ok = false; break; }
+          tc05::fence_after();
+          const uint32_t ocol = S::kOCol + 128u * (uint32_t)qb;
+#pragma unroll 1
+          for (int cb = 0; cb < D / 16; ++cb) {
+            uint32_t ov[16];
+            tc05::ld16(row_t + ocol + 16 * cb, ov);
+            tc05::wait_ld();
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) ov[jj] = __float_as_uint(__uint_as_float(ov[jj]) * alpha);
+            tc05::st16(row_t + ocol + 16 * cb, ov);
+          }
+        }
+        // P buffer g & 1 was last read by O += P.V of step g - 2, which the MMA
+        // thread issued before S(g): S(g) has completed, so that MMA has too.
+        if (busy) {
+          tc05::st32(row_t + S::kPCol + 32 * (uint32_t)(g & 1), pk);
+          tc05::wait_st();
+        }
+        tc05::fence_before();
+        __syncwarp();
+        if (lane == 0) tc05::mbar_arrive(p_full((int)(g & 1)));
+      }
+      if (!ok) break;
+      // Epilogue: the segment's last O += P.V (step g - 1) has to complete.
+      const int64_t gl = g - 1;
+      if (!wwait(o_done((int)(gl & 1)), (uint32_t)((gl >> 1) & 1))) break;
+      tc05::fence_after();
+      if (busy) {
+        const int32_t rbase = prow_s[qb * S::kRows + tid];  // workspace row base of this thread's query row
+        const int32_t prow = rbase < 0 ? -1 : rbase + slot;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const uint32_t ocol = S::kOCol + 128u * (uint32_t)qb;
+        constexpr int kTileStride = 20;  // floats
+        float* tile = reinterpret_cast<float*>(base_ptr + S::kQOff + qb * S::kQBytes) + warp * 32 * kTileStride;
+        float4* wr = reinterpret_cast<float4*>(tile + lane * kTileStride);
+        const int rsub = lane >> 2, csub = lane & 3;
+#pragma unroll 1
+        for (int cb = 0; cb < D / 16; ++cb) {
+          uint32_t ov[16];
+          tc05::ld16(row_t + ocol + 16 * cb, ov);
+          tc05::wait_ld();
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            wr[q4] = make_float4(__uint_as_float(ov[4 * q4]) * inv, __uint_as_float(ov[4 * q4 + 1]) * inv,
+                                 __uint_as_float(ov[4 * q4 + 2]) * inv, __uint_as_float(ov[4 * q4 + 3]) * inv);
+          __syncwarp();
+          float4 v[4];
+          int32_t pr[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            pr[i] = __shfl_sync(kFull, prow, 8 * i + rsub);
+            v[i] = *reinterpret_cast<const float4*>(tile + (8 * i + rsub) * kTileStride + 4 * csub);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (pr[i] >= 0) *reinterpret_cast<float4*>(a.o_part + (int64_t)pr[i] * D + 16 * cb + 4 * csub) = v[i];
+        }
+        if (prow >= 0) {
+          a.m_part[prow] = m_use == -INFINITY ? -INFINITY : m_use * kLn2;
+          a.l_part[prow] = l;
+          for (int p = slot + 1; p < mark_end; ++p) {  // the lane's slots no segment takes: empty
+            a.m_part[rbase + p] = -INFINITY;
+            a.l_part[rbase + p] = 0.f;
+          }
+        }
+      }
+      tc05::fence_before();
+      __syncwarp();
+      if (lane == 0) tc05::mbar_arrive(item_free(qb));
+    }
+  }
+
+  // -- teardown ---------------------------------------------------------------------------------
+  __syncthreads();
+  if (*abort_flag && tid == 0) flag_status(a.status, PA_DEV_TIMEOUT);
+  tc05::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc05::fence_after();
+    tc05::dealloc(tmem, S::kTmemCols);
+  }
+  // A per-sequence kernel launched before this one (for sequences outside every
+  // group) has to finish before this grid does, for the merge that follows.
+  if (tid == 0) asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Two-CTAs-per-SM variant of the persistent tcgen05 shared-prefix kernel.  The
 // one-CTA kernel is bound by its own per-step chain (S MMA, softmax pass, O
 // MMA) while the SM's tensor pipe and its share of DRAM stay mostly idle; two
@@ -2127,10 +2998,14 @@ __global__ void __launch_bounds__(Tc05dShape<D, STAGES>::kThreads, 2)
 // grows with the partition count).  Warp w of an item merges partitions w,
 // w + WPI, ... with its own running maximum (the lanes compute 32 weights per
 // round; partial rows are loaded in prefetched groups), then the item's warps
-// merge through shared memory the same way.
+// merge through shared memory the same way.  A partition whose l is 0 (no
+// token, or a slot a shared-prefix segment marked empty) adds nothing and its
+// row is not read.  Launched as a programmatic dependent of the kernel that
+// writes the partials, it waits for that grid before reading them.
 // ---------------------------------------------------------------------------
 template <typename T, int D, int WPI>
 __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel(const DecodeArgs a, int num_seqs) {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   constexpr int VPL = D / 32;
   constexpr int NW = WPI > 4 ? WPI : 4;
   constexpr int IPC = NW / WPI;  // items per CTA
@@ -2154,11 +3029,13 @@ __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel
   // This warp's partitions are p = sub + WPI * (lane + 32 c), c = 0, 1, ...
   // Lane `lane` holds m and l of its first one; the first UNROLL partial rows
   // are requested before the max is known, and each group of rows is
-  // accumulated while the next group is in flight.
-  auto load_rows = [&](float (&x)[UNROLL][VPL], int p0, int k, int cnt) {
+  // accumulated while the next group is in flight.  `lw` is the lane's l of
+  // the current group: rows with l = 0 are not read.
+  auto load_rows = [&](float (&x)[UNROLL][VPL], int p0, int k, int cnt, float lw) {
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {
-      if (k + u < cnt) {
+      const float lu = __shfl_sync(kFull, lw, min(k + u, 31));
+      if (k + u < cnt && lu > 0.f) {
         const float* src = a.o_part + (base + p0 + WPI * (k + u)) * D + lane * VPL;
         if constexpr (VPL % 4 == 0) {
 #pragma unroll
@@ -2186,7 +3063,7 @@ __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel
     l_first = a.l_part[base + pf];
   }
   float x[UNROLL][VPL];
-  load_rows(x, sub, 0, merge ? min(32, (np - sub + WPI - 1) / WPI) : 0);
+  load_rows(x, sub, 0, merge ? min(32, (np - sub + WPI - 1) / WPI) : 0, l_first);
   float mx = m_first;
   if (merge)
     for (int p = pf + WPI * 32; p < np; p += WPI * 32) mx = fmaxf(mx, a.m_part[base + p]);
@@ -2200,19 +3077,19 @@ __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel
   if (merge && mx != -INFINITY) {
     for (int p0 = sub, c = 0; p0 < np; p0 += WPI * 32, ++c) {
       const int p = p0 + WPI * lane;
-      float wt = 0.f;
+      float wt = 0.f, lcur = 0.f;
       if (p < np) {
         const float mp = c == 0 ? m_first : a.m_part[base + p];
-        const float lp = c == 0 ? l_first : a.l_part[base + p];
-        wt = lp * expf(mp - mx);
+        lcur = c == 0 ? l_first : a.l_part[base + p];
+        wt = lcur > 0.f ? lcur * expf(mp - mx) : 0.f;
       }
       lsum += wt;
       const int cnt = min(32, (np - p0 + WPI - 1) / WPI);
-      if (c > 0) load_rows(x, p0, 0, cnt);
+      if (c > 0) load_rows(x, p0, 0, cnt, lcur);
       for (int k = 0; k < cnt; k += UNROLL) {
         float xn[UNROLL][VPL];
         const bool more = k + UNROLL < cnt;
-        if (more) load_rows(xn, p0, k + UNROLL, cnt);
+        if (more) load_rows(xn, p0, k + UNROLL, cnt, lcur);
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
           const float wk = __shfl_sync(kFull, wt, min(k + u, 31));
@@ -2988,6 +3865,28 @@ cudaError_t launch_shared_tc05d(const DecodeArgs& a, const CUtensorMap& mk, cons
   return cudaGetLastError();
 }
 
+// The balanced tcgen05 kernel: one CTA per SM (CTAs past the work's last range
+// exit at once).  `dependent`: a per-sequence kernel runs before it on the stream.
+template <typename T, int D>
+cudaError_t launch_shared_seg(const DecodeArgs& a, pa_dtype dtype, int num_chunks, const int32_t* chunks,
+                              const int32_t* members, int num_members, const int32_t* first_partition, int num_seqs,
+                              bool dependent, cudaStream_t stream) {
+  constexpr int kStages = D == 128 ? 5 : 8;
+  using S = SegShape<D, kStages>;
+  static std::atomic<uint64_t> done{0};
+  auto kernel = decode_shared_seg_kernel<T, D, kStages>;
+  cudaError_t err = ensure_smem(kernel, S::kSmemBytes, done);
+  if (err != cudaSuccess) return err;
+  // K goes through the tensor-memory-access unit when the cache fits a tensor map
+  // (V, and K otherwise, through cp.async).
+  CUtensorMap mk;
+  std::memset(&mk, 0, sizeof(mk));
+  const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * a.block_size;
+  const int tma_k = rows < (1ll << 31) && encode_cache_map(&mk, a.key_cache, dtype, rows, D) ? 1 : 0;
+  return launch_pdl(kernel, dim3(sm_count()), dim3(S::kThreads), S::kSmemBytes, stream, dependent, a, mk, tma_k,
+                    chunks, num_chunks, members, num_members, first_partition, num_seqs, (int)g_fault.load());
+}
+
 std::atomic<int> g_shared_kernel{PA_SHARED_PREFIX_AUTO};
 
 template <typename T>
@@ -2996,7 +3895,7 @@ cudaError_t launch_shared_dim(const DecodeArgs& a, int head_dim, dim3 grid, cons
                               cudaStream_t stream) {
   const int choice = g_shared_kernel.load();
   if (choice == PA_SHARED_PREFIX_AUTO || choice == PA_SHARED_PREFIX_TCGEN05 ||
-      choice == PA_SHARED_PREFIX_TCGEN05_2CTA) {
+      choice == PA_SHARED_PREFIX_TCGEN05_2CTA || choice == PA_SHARED_PREFIX_TCGEN05_ITEMS) {
     const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * a.block_size;
     CUtensorMap mk, mv;
     if (rows < (1ll << 31) && encode_cache_map(&mk, a.key_cache, dtype, rows, head_dim) &&
@@ -3042,28 +3941,46 @@ cudaError_t launch_cc(const DecodeArgs& a, int head_dim, int num_seqs, int parti
   return cudaGetLastError();
 }
 
+// Launch with programmatic stream serialisation when `dependent` (the kernel
+// may start before the one before it on the stream finishes, and waits for it
+// with griddepcontrol.wait), as an ordinary launch otherwise.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       bool dependent, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <typename T, int D>
-cudaError_t launch_reduce_dim(const DecodeArgs& a, int num_seqs, cudaStream_t stream) {
+cudaError_t launch_reduce_dim(const DecodeArgs& a, int num_seqs, cudaStream_t stream, bool dependent) {
   const int64_t items = (int64_t)num_seqs * a.num_q_heads;
-  auto grid = [&](int ipc) { return (unsigned)((items + ipc - 1) / ipc); };
+  auto grid = [&](int ipc) { return dim3((unsigned)((items + ipc - 1) / ipc)); };
   // Warps per (sequence, query head), by partition count (an 8-warp form,
   // tried for more than 32 partitions, measured no faster).
   if (a.max_partitions <= 16)
-    decode_reduce_kernel<T, D, 1><<<grid(4), 128, 0, stream>>>(a, num_seqs);
-  else if (a.max_partitions <= 48)
-    decode_reduce_kernel<T, D, 2><<<grid(2), 128, 0, stream>>>(a, num_seqs);
-  else
-    decode_reduce_kernel<T, D, 4><<<grid(1), 128, 0, stream>>>(a, num_seqs);
-  return cudaGetLastError();
+    return launch_pdl(decode_reduce_kernel<T, D, 1>, grid(4), dim3(128), 0, stream, dependent, a, num_seqs);
+  if (a.max_partitions <= 48)
+    return launch_pdl(decode_reduce_kernel<T, D, 2>, grid(2), dim3(128), 0, stream, dependent, a, num_seqs);
+  return launch_pdl(decode_reduce_kernel<T, D, 4>, grid(1), dim3(128), 0, stream, dependent, a, num_seqs);
 }
 
 template <typename T>
-cudaError_t launch_reduce(const DecodeArgs& a, int head_dim, int num_seqs, cudaStream_t stream) {
+cudaError_t launch_reduce(const DecodeArgs& a, int head_dim, int num_seqs, cudaStream_t stream,
+                          bool dependent = false) {
   if ((int64_t)num_seqs * a.num_q_heads > 0x7fffffffLL) return cudaErrorInvalidValue;
   switch (head_dim) {
-    case 64: return launch_reduce_dim<T, 64>(a, num_seqs, stream);
-    case 128: return launch_reduce_dim<T, 128>(a, num_seqs, stream);
-    case 256: return launch_reduce_dim<T, 256>(a, num_seqs, stream);
+    case 64: return launch_reduce_dim<T, 64>(a, num_seqs, stream, dependent);
+    case 128: return launch_reduce_dim<T, 128>(a, num_seqs, stream, dependent);
+    case 256: return launch_reduce_dim<T, 256>(a, num_seqs, stream, dependent);
   }
   return cudaErrorInvalidValue;
 }
@@ -3173,7 +4090,8 @@ extern "C" pa_status pa_set_fault_injection(int32_t mode) {
 
 extern "C" pa_status pa_set_shared_prefix_kernel(pa_shared_prefix_kernel k) {
   if (k != PA_SHARED_PREFIX_AUTO && k != PA_SHARED_PREFIX_TCGEN05 && k != PA_SHARED_PREFIX_MMA_SYNC &&
-      k != PA_SHARED_PREFIX_TCGEN05_SERIAL && k != PA_SHARED_PREFIX_TCGEN05_2CTA)
+      k != PA_SHARED_PREFIX_TCGEN05_SERIAL && k != PA_SHARED_PREFIX_TCGEN05_2CTA &&
+      k != PA_SHARED_PREFIX_TCGEN05_ITEMS)
     return fail(PA_ERR_INVALID, "pa_set_shared_prefix_kernel: unknown kernel %d", (int)k);
   g_shared_kernel.store((int)k);
   return PA_OK;
@@ -3284,10 +4202,11 @@ pa_status launch_partitions(const DecodeArgs& a, pa_dtype dtype, int head_dim, i
   return PA_OK;
 }
 
-pa_status launch_reduce_any(const DecodeArgs& a, pa_dtype dtype, int head_dim, int num_seqs, cudaStream_t s) {
-  const cudaError_t err = dtype == PA_F32    ? launch_reduce<float>(a, head_dim, num_seqs, s)
-                          : dtype == PA_BF16 ? launch_reduce<__nv_bfloat16>(a, head_dim, num_seqs, s)
-                                             : launch_reduce<__half>(a, head_dim, num_seqs, s);
+pa_status launch_reduce_any(const DecodeArgs& a, pa_dtype dtype, int head_dim, int num_seqs, cudaStream_t s,
+                            bool dependent = false) {
+  const cudaError_t err = dtype == PA_F32    ? launch_reduce<float>(a, head_dim, num_seqs, s, dependent)
+                          : dtype == PA_BF16 ? launch_reduce<__nv_bfloat16>(a, head_dim, num_seqs, s, dependent)
+                                             : launch_reduce<__half>(a, head_dim, num_seqs, s, dependent);
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode reduce kernel: %s", cudaGetErrorString(err));
   return PA_OK;
 }
@@ -3496,24 +4415,72 @@ static __device__ __align__(256) unsigned char g_fixed_scratch[PA_FIXED_SCRATCH_
 
 constexpr int kMaxDevices = 64;
 std::mutex g_fixed_scratch_mutex;
-void* g_fixed_scratch_addr[kMaxDevices] = {};
+// One cached address per device, valid for the context it was looked up in:
+// a context that is torn down (cudaDeviceReset, or the primary context
+// released) and created again loads the module again, and the array may then
+// sit at another address.  Context ids are never reused within a process.
+struct FixedScratchEntry {
+  unsigned long long ctx_id;
+  void* addr;
+};
+FixedScratchEntry g_fixed_scratch_cache[kMaxDevices] = {};
 
-// Device address of g_fixed_scratch on the current device, looked up once per
-// device (with that device current) and cached.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// The unique id of the calling thread's current context, or 0 when it has
+// none yet (driver entry points looked up once through the runtime).
+pa_status current_context_id(unsigned long long* id) {
+  static std::atomic<CtxGetCurrentFn> get_current{nullptr};
+  static std::atomic<CtxGetIdFn> get_id{nullptr};
+  CtxGetCurrentFn cur = get_current.load();
+  CtxGetIdFn gid = get_id.load();
+  if (!cur || !gid) {
+    void* p1 = nullptr;
+    void* p2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p1, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess || !p1 ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &p2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess || !p2)
+      return fail(PA_ERR_CUDA, "decode_fixed_scratch: the driver's context queries are unavailable");
+    cur = reinterpret_cast<CtxGetCurrentFn>(p1);
+    gid = reinterpret_cast<CtxGetIdFn>(p2);
+    get_current.store(cur);
+    get_id.store(gid);
+  }
+  CUcontext ctx = nullptr;
+  *id = 0;
+  if (cur(&ctx) != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "decode_fixed_scratch: cuCtxGetCurrent failed");
+  if (ctx && gid(ctx, id) != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "decode_fixed_scratch: cuCtxGetId failed");
+  return PA_OK;
+}
+
+// Device address of g_fixed_scratch in the current device's current context,
+// looked up once per (device, context), with that device current, and cached.
 pa_status fixed_scratch_address(void** addr) {
   int dev = -1;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode_fixed_scratch: cudaGetDevice: %s", cudaGetErrorString(err));
   if (dev < 0 || dev >= kMaxDevices) return fail(PA_ERR_UNSUPPORTED, "decode_fixed_scratch: device %d", dev);
+  unsigned long long ctx_id = 0;
+  pa_status st = current_context_id(&ctx_id);
+  if (st != PA_OK) return st;
   std::lock_guard<std::mutex> lock(g_fixed_scratch_mutex);
-  if (!g_fixed_scratch_addr[dev]) {
+  FixedScratchEntry& e = g_fixed_scratch_cache[dev];
+  if (ctx_id == 0 || !e.addr || e.ctx_id != ctx_id) {
     void* p = nullptr;
-    err = cudaGetSymbolAddress(&p, g_fixed_scratch);
+    err = cudaGetSymbolAddress(&p, g_fixed_scratch);  // also makes the runtime's context current
     if (err != cudaSuccess || !p)
       return fail(PA_ERR_CUDA, "decode_fixed_scratch: cudaGetSymbolAddress: %s", cudaGetErrorString(err));
-    g_fixed_scratch_addr[dev] = p;
+    if (ctx_id == 0) {
+      st = current_context_id(&ctx_id);
+      if (st != PA_OK) return st;
+    }
+    e.addr = p;
+    e.ctx_id = ctx_id;
   }
-  *addr = g_fixed_scratch_addr[dev];
+  *addr = e.addr;
   return PA_OK;
 }
 
@@ -3525,18 +4492,22 @@ extern "C" pa_status pa_decode_fixed_scratch(const void* q, const void* key_cach
                                              int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                              int32_t num_blocks, float scale, void* out, pa_dtype dtype,
                                              int32_t* dev_status, void* stream) {
+  // Calls that need no scratch (no sequences) or that pa_decode would reject
+  // anyway are handed to it without the one-time set-up.
+  if (num_seqs <= 0 || max_blocks_per_seq <= 0 || block_size <= 0 || num_q_heads <= 0 || head_dim <= 0)
+    return pa_decode(q, key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                     num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, out, dtype, nullptr, 0,
+                     dev_status, stream);
+  const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim,
+                                               (int64_t)max_blocks_per_seq * block_size);
+  if (need > (size_t)PA_FIXED_SCRATCH_BYTES)
+    return fail(PA_ERR_INVALID,
+                "decode_fixed_scratch: this call needs %zu bytes of scratch, more than the fixed %zu-byte array; "
+                "use pa_decode with a caller-provided workspace",
+                need, (size_t)PA_FIXED_SCRATCH_BYTES);
   void* scratch = nullptr;
-  pa_status st = fixed_scratch_address(&scratch);  // first call on a device: the one-time set-up
+  pa_status st = fixed_scratch_address(&scratch);  // first call in a context: the one-time set-up
   if (st != PA_OK) return st;
-  if (max_blocks_per_seq > 0 && block_size > 0 && num_seqs > 0 && num_q_heads > 0 && head_dim > 0) {
-    const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim,
-                                                 (int64_t)max_blocks_per_seq * block_size);
-    if (need > (size_t)PA_FIXED_SCRATCH_BYTES)
-      return fail(PA_ERR_INVALID,
-                  "decode_fixed_scratch: this call needs %zu bytes of scratch, more than the fixed %zu-byte array; "
-                  "use pa_decode with a caller-provided workspace",
-                  need, (size_t)PA_FIXED_SCRATCH_BYTES);
-  }
   return pa_decode(q, key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs, num_q_heads,
                    num_kv_heads, head_dim, block_size, num_blocks, scale, out, dtype, scratch,
                    (size_t)PA_FIXED_SCRATCH_BYTES, dev_status, stream);
@@ -3565,6 +4536,49 @@ extern "C" pa_status pa_decode_shared_prefix(const void* q, const void* key_cach
                      block_size % 16 == 0 && a.group <= PA_PREFIX_QUERIES_PER_CTA && partitions > 1 &&
                      num_chunks > 0 && num_members > 0 && max_shared_partitions > 0 && first_partition && chunks &&
                      members;
+  const int choice = g_shared_kernel.load();
+  // The balanced kernel's walk counts 64-token steps per kv head in 32 bits: an
+  // upper bound of the call's units must stay below kSegMaxUnits.
+  const int64_t unit_bound =
+      (int64_t)num_kv_heads * ((int64_t)num_chunks * (max_shared_partitions * 8 + 3) +
+                               (int64_t)num_seqs * ((int64_t)max_blocks_per_seq * block_size / 64 + 1 + 2));
+  // AUTO takes the balanced kernel when the members' own tokens are a small share
+  // of the shared work (beams over a long prompt): it then runs them itself at
+  // little cost.  Many long private tails of few rows each (many sequences over a
+  // common prompt) run better in the per-sequence kernel beside the per-partition
+  // joint kernel.
+  const int64_t tail_bound = (int64_t)num_members * std::max<int64_t>(
+      0, (int64_t)max_blocks_per_seq * block_size - (int64_t)min_shared_partitions * kPartition);
+  const bool tails_light = 8 * tail_bound <= (int64_t)num_chunks * max_shared_partitions * kPartition;
+  if (joint && unit_bound < kSegMaxUnits &&
+      ((choice == PA_SHARED_PREFIX_AUTO && tails_light) || choice == PA_SHARED_PREFIX_TCGEN05)) {
+    // Balanced tcgen05 kernel: the groups' shared partitions and their members'
+    // own tokens in one grid; a per-sequence kernel only for the sequences outside
+    // every group (run first, so that the joint grid fills the SMs it leaves).
+    if (!aligned16(chunks)) return fail(PA_ERR_INVALID, "decode_shared_prefix: chunks must be 16-byte aligned");
+    const bool others = num_members < num_seqs;
+    if (others) {
+      DecodeArgs ap = a;
+      ap.first_partition = first_partition;
+      ap.skip_members = 1;
+      ap.partition_base = 0;
+      st = launch_partitions(ap, dtype, head_dim, num_seqs, partitions, s);
+      if (st != PA_OK) return st;
+    }
+    cudaError_t err;
+    if (head_dim == 64)
+      err = dtype == PA_BF16 ? launch_shared_seg<__nv_bfloat16, 64>(a, dtype, num_chunks, chunks, members, num_members,
+                                                                     first_partition, num_seqs, others, s)
+                             : launch_shared_seg<__half, 64>(a, dtype, num_chunks, chunks, members, num_members,
+                                                             first_partition, num_seqs, others, s);
+    else
+      err = dtype == PA_BF16 ? launch_shared_seg<__nv_bfloat16, 128>(a, dtype, num_chunks, chunks, members, num_members,
+                                                                      first_partition, num_seqs, others, s)
+                             : launch_shared_seg<__half, 128>(a, dtype, num_chunks, chunks, members, num_members,
+                                                              first_partition, num_seqs, others, s);
+    if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode shared-prefix kernel: %s", cudaGetErrorString(err));
+    return launch_reduce_any(a, dtype, head_dim, num_seqs, s, /*dependent=*/true);
+  }
   if (joint) {
     if (!aligned16(chunks)) return fail(PA_ERR_INVALID, "decode_shared_prefix: chunks must be 16-byte aligned");
     dim3 grid(num_chunks, num_kv_heads, max_shared_partitions < partitions ? max_shared_partitions : partitions);

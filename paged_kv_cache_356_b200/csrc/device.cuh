@@ -97,6 +97,25 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, for finite x <= 127 (smaller than -125 gives 2^-125).
+// Range reduction in the manner of Cody and Waite: x = i + f with i the
+// nearest integer (adding and subtracting 1.5 * 2^23 rounds to it) and
+// f in [-1/2, 1/2]; 2^f from a cubic fitted for this code (weighted least
+// squares on a dense grid, reweighted until the relative error ripples evenly:
+// maximum relative error 7.6e-5, far below the 16-bit rounding the softmax
+// weights get next); i is added to the exponent field of the result.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float shifter = 12582912.f;  // 1.5 * 2^23
+  const float t = x + shifter;       // rint(x) in the low mantissa bits
+  const float f = x - (t - shifter);
+  float p = fmaf(0.05517031252f, f, 0.2426077873f);
+  p = fmaf(p, f, 0.6932609081f);
+  p = fmaf(p, f, 0.9999282956f);
+  // (bits(t) << 23) is rint(x) << 23 modulo 2^32: the shifter's own bits shift out.
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 // ---- async copies ---------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

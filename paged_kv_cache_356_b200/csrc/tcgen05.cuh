@@ -125,6 +125,20 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t addr, uint32_t parity
   }
   return true;
 }
+// One arrival on the mbarrier (release: the thread's earlier shared-memory
+// writes are visible to a thread that sees the phase complete).
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(mbar) : "memory");
+}
+// The mbarrier's current phase also waits for every cp.async this thread has
+// issued so far (not an arrival: the pending count is raised now and lowered
+// when the copies land).
+__device__ __forceinline__ void cp_async_arrive(uint32_t mbar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];\n" ::"r"(mbar) : "memory");
+}
+// Waits for every cp.async this thread has issued.
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+
 // Makes generic-proxy writes to shared memory (st.shared, cp.async) visible to
 // the async proxy that tcgen05.mma reads through.
 __device__ __forceinline__ void fence_proxy_async_smem() {

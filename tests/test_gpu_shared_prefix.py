@@ -11,8 +11,9 @@ from tests.parity import assert_decode_close, bits_of, host_bits
 
 pytestmark = pytest.mark.gpu
 
-JOINT = {"tcgen05": pa.PA_SHARED_PREFIX_TCGEN05, "tcgen05_2cta": pa.PA_SHARED_PREFIX_TCGEN05_2CTA,
-         "tcgen05_serial": pa.PA_SHARED_PREFIX_TCGEN05_SERIAL, "mma_sync": pa.PA_SHARED_PREFIX_MMA_SYNC}
+JOINT = {"tcgen05": pa.PA_SHARED_PREFIX_TCGEN05, "tcgen05_items": pa.PA_SHARED_PREFIX_TCGEN05_ITEMS,
+         "tcgen05_2cta": pa.PA_SHARED_PREFIX_TCGEN05_2CTA, "tcgen05_serial": pa.PA_SHARED_PREFIX_TCGEN05_SERIAL,
+         "mma_sync": pa.PA_SHARED_PREFIX_MMA_SYNC}
 
 
 @pytest.fixture(params=list(JOINT))
