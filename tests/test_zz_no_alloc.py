@@ -5,10 +5,12 @@ allocation, or a serving loop that forbids allocation after start-up) pass
 inputs and outputs only; the split-context partials live in the library's
 fixed 32 MiB device array.  These tests call the entry point through the C
 ABI (ctypes) and compare it with pa_decode, which takes a caller-provided
-workspace, within the bf16 decode tolerance used by every decode test.  Two
-calls in a row on different inputs check that what the array keeps from the
-previous call does not leak into the next.  This file is collected last, so a
-run that stops at the first failure has run every other test before it.
+workspace, and with the fp64 oracle, within the bf16 decode tolerance used by
+every decode test.  Two calls in a row on different inputs check that what
+the array keeps from the previous call does not leak into the next; a call
+after the first is checked to leave the device's free memory and torch's
+allocated bytes unchanged.  This file is collected last, so a run that stops
+at the first failure has run every other test before it.
 """
 import ctypes
 import math
@@ -16,10 +18,11 @@ import math
 import numpy as np
 import pytest
 
+from oracle import attention
 from paged_kv_cache_356_b200 import _lib
 from paged_kv_cache_356_b200 import binding as pa
 from paged_kv_cache_356_b200 import workloads
-from tests.parity import BF16_ATOL, BF16_RTOL
+from tests.parity import BF16_ATOL, BF16_RTOL, assert_decode_close
 
 pytestmark = pytest.mark.gpu
 
@@ -43,8 +46,9 @@ def _case(seed, ctx, hq=32, hkv=8, d=128, bs=16):
     kc = dev_bf16(nb * hkv * bs * d, (nb, hkv, bs, d))
     vc = dev_bf16(nb * hkv * bs * d, (nb, hkv, bs, d))
     q = dev_bf16(len(ctx) * hq * d, (len(ctx), hq, d))
-    return dict(q=q, kc=kc, vc=vc, tables=torch.from_numpy(tables).cuda(),
-                ctx=torch.tensor(ctx, dtype=torch.int32).cuda(), scale=1.0 / math.sqrt(d))
+    return dict(q=q, kc=kc, vc=vc, tables=torch.from_numpy(tables).cuda(), tables_np=tables,
+                ctx=torch.tensor(ctx, dtype=torch.int32).cuda(), ctx_np=np.array(ctx, dtype=np.int32),
+                scale=1.0 / math.sqrt(d))
 
 
 def _fixed_scratch_call(c, out):
@@ -61,6 +65,13 @@ def _fixed_scratch_call(c, out):
 
 def _reference(c):
     return pa.pa_decode(c["q"], c["kc"], c["vc"], c["tables"], c["ctx"], c["scale"])
+
+
+def _oracle(c):
+    """fp64 textbook attention over the same stored bf16 bits."""
+    bits = lambda t: t.view(__import__("torch").int16).cpu().numpy().view(np.uint16)
+    return attention.decode_attention(bits(c["q"]), bits(c["kc"]), bits(c["vc"]), c["tables_np"], c["ctx_np"],
+                                      c["scale"], "bf16")
 
 
 def _assert_close(got, want):
@@ -80,6 +91,33 @@ def test_two_calls_in_a_row_match_pa_decode():
         assert _fixed_scratch_call(c, out) == 0, _lib.last_error()
         torch.cuda.synchronize()
         _assert_close(out, _reference(c))
+        assert_decode_close(out, _oracle(c), "bf16", "pa_decode_fixed_scratch vs oracle")
+
+
+def test_a_call_after_the_first_allocates_no_device_memory():
+    """After the first call has done its one-time set-up, a call changes neither the device's free
+    memory nor torch's allocated bytes; the same holds through the Python binding."""
+    import torch
+    c = _case(3, [1500, 40, 2600])
+    out = torch.empty_like(c["q"])
+    assert _fixed_scratch_call(c, out) == 0, _lib.last_error()
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    assert _fixed_scratch_call(c, out) == 0, _lib.last_error()
+    pa.pa_decode_fixed_scratch(c["q"], c["kc"], c["vc"], c["tables"], c["ctx"], c["scale"], out)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert torch.cuda.memory_allocated() == alloc0
+    assert_decode_close(out, _oracle(c), "bf16", "binding pa_decode_fixed_scratch vs oracle")
+
+
+def test_empty_batch_returns_before_any_work():
+    import torch
+    c = _case(4, [5])
+    empty = dict(c, q=c["q"][:0], tables=c["tables"][:0], ctx=c["ctx"][:0])
+    out = torch.empty_like(empty["q"])
+    assert _fixed_scratch_call(empty, out) == 0, _lib.last_error()
 
 
 def test_call_beyond_the_fixed_scratch_is_rejected():
