@@ -53,6 +53,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true", help="skip the nvidia-smi clock record (profiler runs)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="measure the headline workload only (by default a 1-GPU run also measures every other "
+                         "workload, the verification step at T = 4 and 8, and the cache-write and page-copy "
+                         "kernels, each with its own clock record, under the line's configs key)")
     ap.add_argument("--micro", action="store_true",
                     help="instead of the decode step, time the cache write (65,536 tokens) and the page copy "
                          "(4,096 pairs of 16-token pages) and print one JSON line each")
@@ -63,7 +67,7 @@ def parse_args(argv=None):
                     help="decode shared leading pages once per group (auto: on for prefix/beam32k)")
     ap.add_argument("--no-graph", action="store_true",
                     help="time eager launches instead of replaying the step as a CUDA graph")
-    ap.add_argument("--joint-kernel", choices=["auto", "tcgen05", "tcgen05_2cta", "tcgen05_serial", "mma_sync"],
+    ap.add_argument("--joint-kernel", choices=["auto", "tcgen05", "tcgen05_items", "tcgen05_2cta", "tcgen05_serial", "mma_sync"],
                     default="auto",
                     help="kernel for the shared partitions of a prefix group")
     ap.add_argument("--verify-tokens", type=int, default=0,
@@ -136,21 +140,23 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profiled_traffic(kernel_hash):
-    """DRAM bytes per launch of the partition kernel from the committed ncu summary, if still current."""
-    path = os.path.join(ROOT, "profiles", "decode_partitions_llama70b.md")
+def profiled_traffic(key, kernel_hash):
+    """DRAM bytes per launch of a kernel on a workload, from the committed counters in
+    profiles/traffic.json, if they were taken on the current sources.
+
+    Returns (bytes or None, record or None); the record carries the source hash the counters were
+    taken on and, when the capture ran on a smaller case, the case it was scaled from."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
-        text = open(path).read()
-    except OSError:
+        with open(path) as f:
+            rec = json.load(f).get(key)
+    except (OSError, ValueError):
         return None, None
-    vals = {}
-    for line in text.splitlines():
-        if ":" in line and line.strip().startswith("- "):
-            k, v = line.strip()[2:].split(":", 1)
-            vals[k.strip()] = v.strip().split()[0].replace(",", "")
-    if vals.get("kernel_source_sha256") != kernel_hash or "dram_bytes_per_launch_full_size" not in vals:
-        return None, vals.get("kernel_source_sha256")
-    return int(float(vals["dram_bytes_per_launch_full_size"])), kernel_hash
+    if not rec:
+        return None, None
+    if rec.get("kernel_source_sha256") != kernel_hash:
+        return None, rec
+    return int(rec["dram_bytes_per_launch"]), rec
 
 
 def kernel_source_hash():
@@ -367,33 +373,70 @@ def rank_workload(name: str, rank: int):
     return base if rank == 0 else workloads.by_name(name, seed=base.seed + 1000 * rank)
 
 
+def apply_kernel_settings(pa, args):
+    """Process-wide kernel choices of the C library, from the command line."""
+    pa.pa_set_decode_kernel({"auto": pa.PA_DECODE_AUTO, "tc": pa.PA_DECODE_TENSOR_CORES,
+                             "cc": pa.PA_DECODE_CUDA_CORES}[args.kernel])
+    warps, stages = (int(x) for x in args.tiling.split("x"))
+    pa.pa_set_decode_tiling(warps, stages)
+    pa.pa_set_verify_tiling(args.verify_rows)
+    pa.pa_set_verify_path({"auto": pa.PA_VERIFY_AUTO, "per_sequence": pa.PA_VERIFY_PER_SEQUENCE,
+                           "joint": pa.PA_VERIFY_JOINT}[args.verify_path])
+    pa.pa_set_shared_prefix_kernel({"auto": pa.PA_SHARED_PREFIX_AUTO, "tcgen05": pa.PA_SHARED_PREFIX_TCGEN05,
+                                    "tcgen05_items": pa.PA_SHARED_PREFIX_TCGEN05_ITEMS,
+                                    "tcgen05_2cta": pa.PA_SHARED_PREFIX_TCGEN05_2CTA,
+                                    "tcgen05_serial": pa.PA_SHARED_PREFIX_TCGEN05_SERIAL,
+                                    "mma_sync": pa.PA_SHARED_PREFIX_MMA_SYNC}[args.joint_kernel])
+
+
+def timed_with_clocks(torch, local, no_clocks, body):
+    """Run ``body()`` (which returns the timed region's milliseconds) while nvidia-smi samples the
+    clocks; the record is extended by re-running ``body`` until it spans at least ~1.5 s under load."""
+    sampler = None
+    if not no_clocks:
+        sampler = ClockSampler(gpu_smi_id(torch, local))
+        sampler.start()
+        time.sleep(0.3)
+    ms = body()
+    clocks = None
+    if sampler is not None:
+        soak_until = time.perf_counter() + 1.5
+        while time.perf_counter() < soak_until:
+            body()
+        clocks = sampler.stop()
+        clocks["window"] = "timed region, extended by identical timed regions to >= 1.5 s of samples"
+    return ms, clocks
+
+
 # ---------------------------------------------------------------------------------------------
 # cache write / page copy bandwidth
 # ---------------------------------------------------------------------------------------------
 
-def run_micro(args):
-    import torch
-    from paged_kv_cache_356_b200 import binding as pa
-    from paged_kv_cache_356_b200 import build as pa_build
-    pa_build.build()
-    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+def micro_results(args, torch, pa, local):
+    """Cache write (65,536 tokens) and page copy (4,096 pairs of 16-token pages) alone, each timed
+    with CUDA events over ``args.steps`` calls after warm-up, with its own clock record."""
     peak, peak_kind = measured_peak()
     g = torch.Generator(device="cuda").manual_seed(7)
     hkv, d, bs = 8, 128, 16
     stream = torch.cuda.current_stream()
+    steps = max(args.steps, 20)
 
-    def timed(fn, iters):
+    def timed(fn):
         for _ in range(max(args.warmup, 3)):
             fn()
         torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(iters):
-            fn()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / iters
 
+        def body():
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(steps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / steps
+        return timed_with_clocks(torch, local, args.no_clocks, body)
+
+    rows = []
     # cache write: 65,536 tokens into a shuffled 4,160-page pool
     t = 65536
     nb = t // bs + 64
@@ -402,13 +445,15 @@ def run_micro(args):
     slots = torch.randperm(nb * bs, generator=g, device="cuda")[:t].to(torch.int64)
     kc = torch.zeros(nb, hkv, bs, d, dtype=torch.bfloat16, device="cuda")
     vc = torch.zeros_like(kc)
-    ms = timed(lambda: pa.pa_reshape_and_cache(key, value, slots, kc, vc), args.steps)
+    ms, clocks = timed(lambda: pa.pa_reshape_and_cache(key, value, slots, kc, vc))
     nbytes = 2 * 2 * t * hkv * d * 2
-    print(json.dumps({"metric": "reshape_and_cache GB/s", "value": nbytes / ms / 1e6, "unit": "GB/s",
-                      "ms_per_call": ms, "bytes_per_call": nbytes, "frac_of_hbm": nbytes / ms / 1e6 / peak,
-                      "peak": peak, "peak_kind": peak_kind,
-                      "config": {"tokens": t, "num_kv_heads": hkv, "head_dim": d, "block_size": bs,
-                                 "dtype": "bf16", "l2": "no flush: 537 MB moved per call"}}), flush=True)
+    rows.append({"metric": "reshape_and_cache GB/s", "value": nbytes / ms / 1e6, "unit": "GB/s",
+                 "ms_per_call": ms, "calls": steps, "bytes_per_call": nbytes,
+                 "frac_of_hbm": {"measured": nbytes / ms / 1e6 / peak, "nominal_8000": nbytes / ms / 1e6 / NOMINAL_HBM_GBS},
+                 "peak": peak, "peak_kind": peak_kind, "kernel": "reshape_and_cache_kernel", "clocks": clocks,
+                 "config": {"workload": "cache write of 65,536 tokens to random slots of a 4,160-page pool",
+                            "tokens": t, "num_kv_heads": hkv, "head_dim": d, "block_size": bs,
+                            "dtype": "bf16", "l2": "no flush: 537 MB moved per call, over four times the 126 MB L2"}})
     del key, value, slots, kc, vc
 
     # page copy: 4,096 (src, dst) pairs of 16-token pages
@@ -418,94 +463,91 @@ def run_micro(args):
     vc = torch.randn(nb, hkv, bs, d, generator=g, device="cuda").to(torch.bfloat16)
     perm = torch.randperm(nb, generator=g, device="cuda")
     mapping = torch.stack([perm[:pairs], perm[pairs:2 * pairs]], dim=1).to(torch.int64).contiguous()
-    ms = timed(lambda: pa.pa_copy_blocks(kc, vc, mapping), args.steps)
+    ms, clocks = timed(lambda: pa.pa_copy_blocks(kc, vc, mapping))
     nbytes = 2 * 2 * pairs * hkv * bs * d * 2
-    print(json.dumps({"metric": "copy_blocks GB/s", "value": nbytes / ms / 1e6, "unit": "GB/s",
-                      "ms_per_call": ms, "bytes_per_call": nbytes, "frac_of_hbm": nbytes / ms / 1e6 / peak,
-                      "peak": peak, "peak_kind": peak_kind,
-                      "config": {"pairs": pairs, "num_kv_heads": hkv, "head_dim": d, "block_size": bs,
-                                 "dtype": "bf16", "l2": "no flush: 537 MB moved per call"}}), flush=True)
+    rows.append({"metric": "copy_blocks GB/s", "value": nbytes / ms / 1e6, "unit": "GB/s",
+                 "ms_per_call": ms, "calls": steps, "bytes_per_call": nbytes,
+                 "frac_of_hbm": {"measured": nbytes / ms / 1e6 / peak, "nominal_8000": nbytes / ms / 1e6 / NOMINAL_HBM_GBS},
+                 "peak": peak, "peak_kind": peak_kind, "kernel": "copy_blocks_kernel", "clocks": clocks,
+                 "config": {"workload": "page copy of 4,096 random (src, dst) pairs of 16-token pages",
+                            "pairs": pairs, "num_kv_heads": hkv, "head_dim": d, "block_size": bs,
+                            "dtype": "bf16", "l2": "no flush: 537 MB moved per call, over four times the 126 MB L2"}})
+    del kc, vc, perm, mapping
+    torch.cuda.empty_cache()
+    return rows
+
+
+def run_micro(args):
+    import torch
+    from paged_kv_cache_356_b200 import binding as pa
+    from paged_kv_cache_356_b200 import build as pa_build
+    pa_build.build()
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    for row in micro_results(args, torch, pa, local):
+        print(json.dumps(row), flush=True)
     return 0
 
 
 # ---------------------------------------------------------------------------------------------
-# our arm
+# one workload's step, as the bench times it
 # ---------------------------------------------------------------------------------------------
 
-def run_ours(args):
-    import torch
-    import torch.distributed as dist
+class StepBench:
+    """A workload's step on resident inputs: the step's cache write, then decode (the partition
+    kernel(s) and the merge) -- or, with ``T`` > 0, the write of T draft tokens per sequence and their
+    verification.  ``run`` reuses a TraceRunner whose trace has already run."""
 
-    from paged_kv_cache_356_b200 import binding as pa
-    from paged_kv_cache_356_b200 import build as pa_build
-    from paged_kv_cache_356_b200 import workloads
-    from paged_kv_cache_356_b200.runner import TraceRunner
+    def __init__(self, args, w, shared, T=0, run=None):
+        import torch
+        from paged_kv_cache_356_b200 import binding as pa
+        from paged_kv_cache_356_b200.runner import TraceRunner
+        self.args, self.torch, self.pa, self.w, self.T = args, torch, pa, w, T
+        if run is None:
+            run = TraceRunner(w, shared_prefix=shared)
+            run.run(decode=False)
+            torch.cuda.synchronize()
+            if run.status() != 0:
+                raise RuntimeError(f"device status {run.status()} after setup")
+        self.run = run
+        tables_np = run.block_tables.cpu().numpy()
+        self.ctx_np = ctx_np = run.context_lens.cpu().numpy()
+        self.unique, self.logical = kv_bytes(w, tables_np, ctx_np)
+        self.part_bytes = partition_kernel_bytes(w, ctx_np, self.unique)
+        self.max_ctx = max_ctx = w.max_blocks_per_seq * w.block_size
+        self.kd, self.vd, self.sd = run.step_write
+        self.q, self.out, self.ws = run.q, run.out, run.workspace
+        self.verify_joint = False
+        if T > 0:
+            # draft verification: the step overwrites each sequence's last T positions with the draft
+            # tokens' K/V, then attends with T causal query tokens per sequence
+            if run.plan is not None or int(ctx_np.min()) < T:
+                raise SystemExit("--verify-tokens needs a workload without a shared-prefix plan and contexts >= T")
+            slots = np.concatenate([run.alloc.slot_mapping(b, int(ctx_np[b]) - T, T) for b in range(w.num_seqs)])
+            dk, dv = w.draft_kv(T)
+            self.kd, self.vd = run._to_device(dk), run._to_device(dv)
+            self.sd = torch.from_numpy(slots.astype(np.int64)).cuda()
+            self.q = run._to_device(w.draft_query(T))
+            self.out = torch.empty_like(self.q)
+            need = pa.pa_decode_verify_workspace_size(w.num_seqs, T, w.num_q_heads, w.head_dim, max_ctx)
+            self.ws = torch.empty(need, dtype=torch.uint8, device="cuda") if need > 0 else None
+            self.part_bytes = verify_call_bytes(w, ctx_np, self.unique, T)
+            self.verify_joint = (args.verify_path == "joint" or
+                                 (args.verify_path == "auto" and T * w.group_size > 16 and args.kernel != "cc" and
+                                  w.dtype in ("bf16", "f16") and w.head_dim in (64, 128) and
+                                  w.block_size % 16 == 0 and max_ctx > 512))
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
-    pa_build.build()
-    pa.pa_set_decode_kernel({"auto": pa.PA_DECODE_AUTO, "tc": pa.PA_DECODE_TENSOR_CORES,
-                             "cc": pa.PA_DECODE_CUDA_CORES}[args.kernel])
-    warps, stages = (int(x) for x in args.tiling.split("x"))
-    pa.pa_set_decode_tiling(warps, stages)
-    pa.pa_set_verify_tiling(args.verify_rows)
-    pa.pa_set_verify_path({"auto": pa.PA_VERIFY_AUTO, "per_sequence": pa.PA_VERIFY_PER_SEQUENCE,
-                           "joint": pa.PA_VERIFY_JOINT}[args.verify_path])
-    pa.pa_set_shared_prefix_kernel({"auto": pa.PA_SHARED_PREFIX_AUTO, "tcgen05": pa.PA_SHARED_PREFIX_TCGEN05,
-                                    "tcgen05_2cta": pa.PA_SHARED_PREFIX_TCGEN05_2CTA,
-                                    "tcgen05_serial": pa.PA_SHARED_PREFIX_TCGEN05_SERIAL,
-                                    "mma_sync": pa.PA_SHARED_PREFIX_MMA_SYNC}[args.joint_kernel])
-
-    w = rank_workload(args.workload, rank)
-    shared = args.shared_prefix == "on" or (args.shared_prefix == "auto" and w.kind in ("prefix", "beam"))
-    run = TraceRunner(w, shared_prefix=shared)
-    run.run(decode=False)
-    torch.cuda.synchronize()
-    if run.status() != 0:
-        raise RuntimeError(f"device status {run.status()} after setup")
-    tables_np = run.block_tables.cpu().numpy()
-    ctx_np = run.context_lens.cpu().numpy()
-    unique, logical = kv_bytes(w, tables_np, ctx_np)
-    part_bytes = partition_kernel_bytes(w, ctx_np, unique)
-    max_ctx = w.max_blocks_per_seq * w.block_size
-    stream = torch.cuda.current_stream()
-    kd, vd, sd = run.step_write
-    q_step, out_step, ws_step = run.q, run.out, run.workspace
-    T = args.verify_tokens
-    verify_joint = False
-    if T > 0:
-        # draft verification: the step overwrites each sequence's last T positions with the draft
-        # tokens' K/V, then attends with T causal query tokens per sequence
-        if run.plan is not None or int(ctx_np.min()) < T:
-            raise SystemExit("--verify-tokens needs a workload without a shared-prefix plan and contexts >= T")
-        slots = np.concatenate([run.alloc.slot_mapping(b, int(ctx_np[b]) - T, T) for b in range(w.num_seqs)])
-        dk, dv = w.draft_kv(T)
-        kd, vd = run._to_device(dk), run._to_device(dv)
-        sd = torch.from_numpy(slots.astype(np.int64)).cuda()
-        q_step = run._to_device(w.draft_query(T))
-        out_step = torch.empty_like(q_step)
-        need = pa.pa_decode_verify_workspace_size(w.num_seqs, T, w.num_q_heads, w.head_dim, max_ctx)
-        ws_step = torch.empty(need, dtype=torch.uint8, device="cuda") if need > 0 else None
-        part_bytes = verify_call_bytes(w, ctx_np, unique, T)
-        verify_joint = (args.verify_path == "joint" or
-                        (args.verify_path == "auto" and T * w.group_size > 16 and args.kernel != "cc" and
-                         w.dtype in ("bf16", "f16") and w.head_dim in (64, 128) and w.block_size % 16 == 0 and
-                         max_ctx > 512))
-
-    def step(evs=None, stream=stream):
+    def step(self, evs=None, stream=None):
+        pa, run, w = self.pa, self.run, self.w
+        stream = stream if stream is not None else self.torch.cuda.current_stream()
         if evs is not None:
             evs[0].record(stream)
-        pa.pa_reshape_and_cache(kd, vd, sd, run.key_cache, run.value_cache, stream=stream)
+        pa.pa_reshape_and_cache(self.kd, self.vd, self.sd, run.key_cache, run.value_cache, stream=stream)
         if evs is not None:
             evs[1].record(stream)
-        if T > 0:                    # partition kernel and merge, one call
-            pa.pa_decode_verify(q_step, run.key_cache, run.value_cache, run.block_tables, run.context_lens,
-                                w.scale, out=out_step, workspace=ws_step, stream=stream)
+        if self.T > 0:               # partition kernel and merge, one call
+            pa.pa_decode_verify(self.q, run.key_cache, run.value_cache, run.block_tables, run.context_lens,
+                                w.scale, out=self.out, workspace=self.ws, stream=stream)
             if evs is not None:
                 evs[2].record(stream)
         elif run.plan is not None:   # joint + per-sequence partition kernels and the merge, one call
@@ -518,98 +560,207 @@ def run_ours(args):
                                     w.scale, run.out, run.workspace, stream=stream)
             if evs is not None:
                 evs[2].record(stream)
-            pa.pa_decode_reduce(run.context_lens, max_ctx, run.out, run.workspace, stream=stream)
+            pa.pa_decode_reduce(run.context_lens, self.max_ctx, run.out, run.workspace, stream=stream)
         if evs is not None:
             evs[3].record(stream)
 
-    for _ in range(max(args.warmup, 3)):
-        step()
-    torch.cuda.synchronize()
+    def launches_per_step(self):
+        if self.T > 0:
+            return 2 + (self.max_ctx > 512) + 2 * self.verify_joint
+        return 4 if self.run.plan is not None and self.run.plan["num_chunks"] > 0 else 3
 
-    # Per-kernel breakdown: one eager pass of the same steps with events between the kernels.
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    for i in range(args.steps):
-        step(evs[i])
-    torch.cuda.synchronize()
+    def measure(self, steps, warmup, world, local):
+        """Warm-up, an eager pass with events between the kernels, then ``steps`` timed steps (a
+        replayed CUDA graph unless --no-graph), with an L2 flush before each timed step when the step
+        reads under twice the L2.  Returns the timings and the clock record."""
+        torch, args = self.torch, self.args
+        import torch.distributed as dist
+        stream = torch.cuda.current_stream()
+        for _ in range(max(warmup, 3)):
+            self.step()
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        for i in range(steps):
+            self.step(evs[i])
+        torch.cuda.synchronize()
 
-    # The timed region replays the step as a CUDA graph (as a decode loop would), unless disabled.
-    graph, launch_mode = None, "eager"
-    if not args.no_graph:
-        try:
-            side = torch.cuda.Stream()
-            side.wait_stream(stream)
-            with torch.cuda.stream(side):
-                step(stream=side)
-            stream.wait_stream(side)
-            torch.cuda.synchronize()
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph):
-                step(stream=torch.cuda.current_stream())
-            for _ in range(3):
+        graph, launch_mode = None, "eager"
+        if not args.no_graph:
+            try:
+                side = torch.cuda.Stream()
+                side.wait_stream(stream)
+                with torch.cuda.stream(side):
+                    self.step(stream=side)
+                stream.wait_stream(side)
+                torch.cuda.synchronize()
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph):
+                    self.step(stream=torch.cuda.current_stream())
+                for _ in range(3):
+                    graph.replay()
+                torch.cuda.synchronize()
+                launch_mode = "CUDA graph of one step (write + decode), replayed"
+            except Exception as exc:  # capture unsupported here: time eager launches
+                graph = None
+                launch_mode = f"eager (graph capture failed: {type(exc).__name__})"
+                torch.cuda.synchronize()
+
+        def one():
+            if graph is not None:
                 graph.replay()
-            torch.cuda.synchronize()
-            launch_mode = "CUDA graph of one step (write + decode), replayed"
-        except Exception as exc:  # capture unsupported here: time eager launches
-            graph = None
-            launch_mode = f"eager (graph capture failed: {type(exc).__name__})"
-            torch.cuda.synchronize()
+            else:
+                self.step()
 
-    def timed_step():
-        if graph is not None:
-            graph.replay()
+        # A step that reads less than twice the 126 MB L2 could find part of its KV still cached from
+        # the previous step: then every timed step is preceded by writing a 256 MB buffer, and only
+        # the step itself is timed.
+        flush_l2 = self.unique < 2 * L2_BYTES
+        scrub = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if flush_l2 else None
+
+        def body():
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            if flush_l2:
+                tev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+                for i in range(steps):
+                    scrub.fill_(i & 0xFF)
+                    tev[i][0].record(stream)
+                    one()
+                    tev[i][1].record(stream)
+            else:
+                t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                t0.record(stream)
+                for _ in range(steps):
+                    one()
+                t1.record(stream)
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            return sum(e[0].elapsed_time(e[1]) for e in tev) if flush_l2 else t0.elapsed_time(t1)
+
+        if world > 1:   # every rank soaks the same number of timed regions: no data-dependent loop
+            total_ms = body()
+            clocks = None
+            if not args.no_clocks:
+                total_ms, clocks = timed_with_clocks(torch, local, False, body)
         else:
-            step()
+            total_ms, clocks = timed_with_clocks(torch, local, args.no_clocks, body)
+        if graph is not None:
+            del graph
+        del scrub
+        return {"total_ms": total_ms, "ms_per_step": total_ms / steps,
+                "eager_ms": evs[0][0].elapsed_time(evs[-1][3]) / steps,
+                "write_ms": sum(e[0].elapsed_time(e[1]) for e in evs) / steps,
+                "part_ms": sum(e[1].elapsed_time(e[2]) for e in evs) / steps,
+                "reduce_ms": sum(e[2].elapsed_time(e[3]) for e in evs) / steps,
+                "launch": launch_mode, "flush_l2": flush_l2, "clocks": clocks}
 
-    # A step that reads less than twice the 126 MB L2 could find part of its KV still cached from
-    # the previous step: then every timed step is preceded by writing a 256 MB buffer, and only
-    # the step itself is timed.
-    flush_l2 = unique < 2 * L2_BYTES
-    scrub = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if flush_l2 else None
+    def l2_policy(self, flush_l2):
+        return ("flushed: a 256 MB buffer is written before each timed step (its unique KV is under twice the "
+                "126 MB L2); only the step is timed" if flush_l2 else
+                "no flush: each step reads its whole KV, more than twice the 126 MB L2")
 
-    sampler = None
-    if not args.no_clocks:
-        sampler = ClockSampler(gpu_smi_id(torch, local))
-        sampler.start()
-        time.sleep(0.3)
+    def kernel_ms(self, m):
+        if self.T > 0:
+            return {"reshape_and_cache": m["write_ms"], "decode_verify (partition kernel + merge)": m["part_ms"]}
+        if self.run.plan is None:
+            return {"reshape_and_cache": m["write_ms"], "decode_partitions": m["part_ms"],
+                    "decode_reduce": m["reduce_ms"]}
+        return {"reshape_and_cache": m["write_ms"],
+                "decode_shared_prefix (joint + per-sequence + merge)": m["part_ms"]}
+
+
+def config_entry(sb, m, peak, peak_kind):
+    """A summary of one workload's measurement for the bench line's ``configs`` key."""
+    w, T = sb.w, sb.T
+    ms = m["ms_per_step"]
+    gbs = sb.unique / ms / 1e6
+    e = {"workload": describe(w)["workload"] + (f"; {T} draft tokens per sequence verified per step (causal)"
+                                                if T else ""),
+         "ms_per_step": ms,
+         "kv_gbs_unique": gbs, "kv_gbs_logical": sb.logical / ms / 1e6,
+         "kv_bytes_per_step": {"unique": sb.unique, "logical": sb.logical},
+         "frac_of_hbm": {"measured": gbs / peak, "nominal_8000": gbs / NOMINAL_HBM_GBS, "peak": peak,
+                         "peak_kind": peak_kind},
+         "seqs_per_s": w.num_seqs * 1000.0 / ms,
+         "eager_ms_per_step": m["eager_ms"], "kernel_ms": sb.kernel_ms(m),
+         "l2": sb.l2_policy(m["flush_l2"]), "launch": m["launch"], "clocks": m["clocks"]}
+    if T:
+        e["query_tokens"] = T
+        e["query_tokens_per_s"] = w.num_seqs * T * 1000.0 / ms
+        e["verify_path"] = "joint + per-sequence" if sb.verify_joint else "per-sequence"
+    if sb.run.plan is not None:
+        e["shared_prefix_plan"] = {"chunks": sb.run.plan["num_chunks"], "members": sb.run.plan["num_members"],
+                                   "shared_partitions": sb.run.plan["max_shared_partitions"]}
+    return e
+
+
+# Every configuration the benchmark carries beside the headline, in the order they run.
+EXTRA_CONFIGS = ("verify4", "verify8", "llama8b", "prefix", "beam32k", "micro")
+
+
+def extra_configs(args, head, peak, peak_kind, local):
+    """Every other configuration of the decode path, measured in the same run with its own clock
+    record: the draft-verification step at T = 4 and 8 on the headline batch (which it then
+    modifies), the other decode workloads, and the cache-write and page-copy kernels alone."""
+    import torch
+    from paged_kv_cache_356_b200 import binding as pa
+    from paged_kv_cache_356_b200 import workloads
+    out = {}
+    steps = args.steps
+    for name in EXTRA_CONFIGS:
+        if name.startswith("verify"):
+            T = int(name[len("verify"):])
+            if head.run.plan is not None or head.T:
+                continue
+            sb = StepBench(args, head.w, False, T=T, run=head.run)
+            out[f"{head.w.name}_verify_T{T}"] = dict(config_entry(sb, sb.measure(steps, args.warmup, 1, local),
+                                                                  peak, peak_kind), steps=steps)
+            del sb
+        elif name == "micro":
+            for row in micro_results(args, torch, pa, local):
+                out[row["kernel"]] = row
+        elif name != head.w.name:
+            w = workloads.by_name(name)
+            sb = StepBench(args, w, w.kind in ("prefix", "beam"))
+            out[name] = dict(config_entry(sb, sb.measure(steps, args.warmup, 1, local), peak, peak_kind),
+                             steps=steps)
+            del sb
+            torch.cuda.empty_cache()
+    return out
+
+
+# ---------------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from paged_kv_cache_356_b200 import binding as pa
+    from paged_kv_cache_356_b200 import build as pa_build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
     if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    if flush_l2:
-        tev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-        for i in range(args.steps):
-            scrub.fill_(i & 0xFF)
-            tev[i][0].record(stream)
-            timed_step()
-            tev[i][1].record(stream)
-    else:
-        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        for i in range(args.steps):
-            timed_step()
-        t1.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    total_ms = sum(e[0].elapsed_time(e[1]) for e in tev) if flush_l2 else t0.elapsed_time(t1)
-    eager_ms = evs[0][0].elapsed_time(evs[-1][3]) / args.steps
-    clocks = None
-    if sampler is not None:
-        # keep identical steps running until the clock record spans at least ~1.5 s under load
-        soak_until = time.perf_counter() + max(0.0, 1.5 - total_ms / 1000)
-        while time.perf_counter() < soak_until:
-            for _ in range(20):
-                timed_step()
-            torch.cuda.synchronize()
-        clocks = sampler.stop()
-        clocks["window"] = "timed region, extended by identical steps to >= 1.5 s of samples"
-    if graph is not None:
-        del graph
-    del scrub
-    write_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
-    part_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
-    reduce_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    pa_build.build()
+    apply_kernel_settings(pa, args)
 
-    total_ms_max, (all_unique, all_seqs) = reduce_over_ranks(total_ms, [unique, w.num_seqs], world, "cuda")
+    w = rank_workload(args.workload, rank)
+    shared = args.shared_prefix == "on" or (args.shared_prefix == "auto" and w.kind in ("prefix", "beam"))
+    T = args.verify_tokens
+    sb = StepBench(args, w, shared, T=T)
+    run = sb.run
+    m = sb.measure(args.steps, args.warmup, world, local)
+    total_ms = m["total_ms"]
+
+    total_ms_max, (all_unique, all_seqs) = reduce_over_ranks(total_ms, [sb.unique, w.num_seqs], world, "cuda")
     seconds = total_ms_max / 1000.0
     value = all_unique * args.steps / seconds / 1e9
     seqs_per_s = all_seqs * args.steps / seconds
@@ -619,7 +770,7 @@ def run_ours(args):
     if not args.no_e2e:
         if T > 0:
             decode = lambda d_q, d_tab, d_ctx, d_out: pa.pa_decode_verify(
-                d_q, run.key_cache, run.value_cache, d_tab, d_ctx, w.scale, out=d_out, workspace=ws_step)
+                d_q, run.key_cache, run.value_cache, d_tab, d_ctx, w.scale, out=d_out, workspace=sb.ws)
         elif run.plan is not None:
             decode = lambda d_q, d_tab, d_ctx, d_out: pa.pa_decode_shared_prefix(
                 d_q, run.key_cache, run.value_cache, d_tab, d_ctx, w.scale, run.plan, out=d_out,
@@ -627,30 +778,35 @@ def run_ours(args):
         else:
             decode = lambda d_q, d_tab, d_ctx, d_out: pa.pa_decode(
                 d_q, run.key_cache, run.value_cache, d_tab, d_ctx, w.scale, out=d_out, workspace=run.workspace)
-        e2e = end_to_end(args, torch, pa, run, w, unique, world, dist, (q_step, kd, vd, sd, out_step), decode)
+        e2e = end_to_end(args, torch, pa, run, w, sb.unique, world, dist, (sb.q, sb.kd, sb.vd, sb.sd, sb.out),
+                         decode)
 
     peak, peak_kind = measured_peak()
-    achieved = part_bytes / (part_ms / 1000.0) / 1e9
+    achieved = sb.part_bytes / (m["part_ms"] / 1000.0) / 1e9
     khash = kernel_source_hash()
-    traffic, _ = profiled_traffic(khash)
+    traffic_key = f"decode_tc_kernel {args.workload}"
+    traffic, traffic_rec = (profiled_traffic(traffic_key, khash)
+                            if run.plan is None and T == 0 and args.kernel != "cc" else (None, None))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.workload, args.cpu_seconds, verify_tokens=T)
 
+    configs = None
+    if world == 1 and not args.no_configs:
+        configs = extra_configs(args, sb, peak, peak_kind, local)
+
     if rank == 0:
         cfg = describe(w)
         cfg.update({"parallelism": f"dp{world} (independent batches per GPU, no collective)",
-                    "l2": ("flushed: a 256 MB buffer is written before each timed step (its unique KV is under "
-                           "twice the 126 MB L2); only the step is timed" if flush_l2 else
-                           "no flush: each step reads its whole KV, more than twice the 126 MB L2"),
+                    "l2": sb.l2_policy(m["flush_l2"]),
                     "kernel": args.kernel, "tiling": args.tiling, "global_batch": w.num_seqs * world,
-                    "launch": launch_mode})
+                    "launch": m["launch"]})
         if run.plan is not None:
             cfg["joint_kernel"] = args.joint_kernel
         if T > 0:
             cfg["query_tokens"] = T
-            cfg["verify_path"] = f"{args.verify_path} ({'joint + per-sequence' if verify_joint else 'per-sequence'})"
+            cfg["verify_path"] = f"{args.verify_path} ({'joint + per-sequence' if sb.verify_joint else 'per-sequence'})"
             cfg["verify_rows_per_cta"] = args.verify_rows or "default"
             cfg["workload"] += f"; {T} draft tokens per sequence verified per step (causal)"
         line = {
@@ -660,39 +816,36 @@ def run_ours(args):
             "data": "synthetic", "config": cfg,
             "seqs_per_s": seqs_per_s,
             **({"query_tokens_per_s": seqs_per_s * T} if T > 0 else {}),
-            "eager": {"ms_per_step": eager_ms, "seqs_per_s": w.num_seqs * 1000.0 / eager_ms,
+            "eager": {"ms_per_step": m["eager_ms"], "seqs_per_s": w.num_seqs * 1000.0 / m["eager_ms"],
                       "note": "same steps launched one call at a time, events between the kernels"},
-            "kv_bytes_per_step": {"unique": unique, "logical": logical},
+            "kv_bytes_per_step": {"unique": sb.unique, "logical": sb.logical},
             "frac_of_hbm": {"measured": value / world / peak, "nominal_8000": value / world / NOMINAL_HBM_GBS},
-            "kernel_ms": ({"reshape_and_cache": write_ms, "decode_verify (partition kernel + merge)": part_ms}
-                          if T > 0 else
-                          {"reshape_and_cache": write_ms, "decode_partitions": part_ms, "decode_reduce": reduce_ms}
-                          if run.plan is None else
-                          {"reshape_and_cache": write_ms, "decode_shared_prefix (joint + per-sequence + merge)": part_ms}),
+            "kernel_ms": sb.kernel_ms(m),
             "shared_prefix_plan": (None if run.plan is None else
                                    {"chunks": run.plan["num_chunks"], "members": run.plan["num_members"],
                                     "shared_partitions": run.plan["max_shared_partitions"]}),
             "roofline": {"bound": "hbm",
                          "kernel": (("pa_decode_verify call: plan kernel + joint tcgen05 kernel (partitions all "
                                      "tokens see) + decode_verify_tc_kernel (the rest) + merge, timed together"
-                                     if verify_joint else
+                                     if sb.verify_joint else
                                      "pa_decode_verify call: decode_verify_tc_kernel + merge (timed together)")
                                     if T > 0 else
                                     "decode_tc_kernel (pa_decode_partitions)" if run.plan is None else
-                                    "pa_decode_shared_prefix call: decode_shared_tc05p_kernel + per-sequence "
+                                    "pa_decode_shared_prefix call: joint tcgen05 kernel + per-sequence "
                                     "decode_tc_kernel + merge (timed together)"),
                          "achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} (copy bandwidth)",
                          "unit": "GB/s", "frac": achieved / peak,
-                         # the committed counters are per launch of the Llama-3-70B-shaped batch
-                         "traffic": (traffic if (args.workload == "llama70b" and run.plan is None and T == 0)
-                                     else None),
-                         "algorithmic_bytes_per_launch": part_bytes, "kernel_source_sha256": khash},
+                         "traffic": traffic,
+                         **({"traffic_scaled_from": traffic_rec["scaled_from"]}
+                            if traffic is not None and traffic_rec.get("scaled_from") else {}),
+                         "algorithmic_bytes_per_launch": sb.part_bytes, "kernel_source_sha256": khash},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": ((4 if run.plan is not None and run.plan["num_chunks"] > 0 else 3) if T == 0 else
-                             2 + (max_ctx > 512) + 2 * verify_joint) * args.steps,
-            "clocks": clocks,
+            "gpu_launches": sb.launches_per_step() * args.steps,
+            "clocks": m["clocks"],
         }
+        if configs is not None:
+            line["configs"] = configs
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

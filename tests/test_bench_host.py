@@ -1,6 +1,8 @@
 """Host-side pieces of bench.py that need no GPU: the partition kernel's source hash resolves its
 anchors, the committed ncu summary parses and still matches the sources, and the byte accounting of a
 decode step counts shared pages once."""
+import os
+
 import numpy as np
 
 import bench
@@ -10,12 +12,21 @@ from paged_kv_cache_356_b200 import workloads
 def test_kernel_hash_and_committed_traffic_are_consistent():
     h = bench.kernel_source_hash()
     assert len(h) == 16 and int(h, 16) >= 0
-    traffic, committed = bench.profiled_traffic(h)
-    assert committed is not None and len(committed) == 16
-    if committed == h:   # counters taken on these sources: a plausible DRAM figure for the full batch
-        assert traffic is not None and 0.9 < traffic / 2965942736 < 1.1
-    else:                # the kernel changed since: the bench must report no traffic
+    traffic, rec = bench.profiled_traffic("decode_tc_kernel llama70b", h)
+    assert rec is not None and len(rec["kernel_source_sha256"]) == 16
+    assert rec["summary"].startswith("profiles/") and os.path.exists(os.path.join(bench.ROOT, rec["summary"]))
+    if rec["kernel_source_sha256"] == h:   # counters taken on these sources: a plausible DRAM figure
+        assert traffic is not None and 0.9 < traffic / rec["algorithmic_bytes_per_launch"] < 1.1
+    else:                                   # the kernel changed since: the bench must report no traffic
         assert traffic is None
+    assert bench.profiled_traffic("no such kernel", h) == (None, None)
+
+
+def test_configs_cover_every_workload_and_kernel():
+    """The default run carries every other workload, both verification sizes and both copy kernels."""
+    names = set(bench.EXTRA_CONFIGS)
+    assert {"llama8b", "prefix", "beam32k", "micro", "verify4", "verify8"} <= names
+    assert bench.parse_args([]).no_configs is False and bench.parse_args(["--no-configs"]).no_configs
 
 
 def test_unique_and_logical_kv_bytes():
