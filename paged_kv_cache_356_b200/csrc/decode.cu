@@ -2998,12 +2998,14 @@ __global__ void __launch_bounds__(Tc05dShape<D, STAGES>::kThreads, 2)
 // grows with the partition count).  Warp w of an item merges partitions w,
 // w + WPI, ... with its own running maximum (the lanes compute 32 weights per
 // round; partial rows are loaded in prefetched groups), then the item's warps
-// merge through shared memory the same way.  A partition whose l is 0 (no
-// token, or a slot a shared-prefix segment marked empty) adds nothing and its
-// row is not read.  Launched as a programmatic dependent of the kernel that
-// writes the partials, it waits for that grid before reading them.
+// merge through shared memory the same way.  A partition whose l is 0 adds
+// nothing; with SPARSE (the balanced shared-prefix kernel leaves slots it
+// marks empty, l = 0, unwritten) such a row is not read at all -- otherwise
+// rows are requested before their l is known.  Launched as a programmatic
+// dependent of the kernel that writes the partials, it waits for that grid
+// before reading them.
 // ---------------------------------------------------------------------------
-template <typename T, int D, int WPI>
+template <typename T, int D, int WPI, bool SPARSE>
 __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel(const DecodeArgs a, int num_seqs) {
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
   constexpr int VPL = D / 32;
@@ -3034,8 +3036,8 @@ __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel
   auto load_rows = [&](float (&x)[UNROLL][VPL], int p0, int k, int cnt, float lw) {
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {
-      const float lu = __shfl_sync(kFull, lw, min(k + u, 31));
-      if (k + u < cnt && lu > 0.f) {
+      const bool present = SPARSE ? __shfl_sync(kFull, lw, min(k + u, 31)) > 0.f : true;
+      if (k + u < cnt && present) {
         const float* src = a.o_part + (base + p0 + WPI * (k + u)) * D + lane * VPL;
         if constexpr (VPL % 4 == 0) {
 #pragma unroll
@@ -3960,27 +3962,30 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-template <typename T, int D>
+template <typename T, int D, bool SPARSE>
 cudaError_t launch_reduce_dim(const DecodeArgs& a, int num_seqs, cudaStream_t stream, bool dependent) {
   const int64_t items = (int64_t)num_seqs * a.num_q_heads;
   auto grid = [&](int ipc) { return dim3((unsigned)((items + ipc - 1) / ipc)); };
   // Warps per (sequence, query head), by partition count (an 8-warp form,
   // tried for more than 32 partitions, measured no faster).
   if (a.max_partitions <= 16)
-    return launch_pdl(decode_reduce_kernel<T, D, 1>, grid(4), dim3(128), 0, stream, dependent, a, num_seqs);
+    return launch_pdl(decode_reduce_kernel<T, D, 1, SPARSE>, grid(4), dim3(128), 0, stream, dependent, a, num_seqs);
   if (a.max_partitions <= 48)
-    return launch_pdl(decode_reduce_kernel<T, D, 2>, grid(2), dim3(128), 0, stream, dependent, a, num_seqs);
-  return launch_pdl(decode_reduce_kernel<T, D, 4>, grid(1), dim3(128), 0, stream, dependent, a, num_seqs);
+    return launch_pdl(decode_reduce_kernel<T, D, 2, SPARSE>, grid(2), dim3(128), 0, stream, dependent, a, num_seqs);
+  return launch_pdl(decode_reduce_kernel<T, D, 4, SPARSE>, grid(1), dim3(128), 0, stream, dependent, a, num_seqs);
 }
 
 template <typename T>
 cudaError_t launch_reduce(const DecodeArgs& a, int head_dim, int num_seqs, cudaStream_t stream,
-                          bool dependent = false) {
+                          bool dependent = false, bool sparse = false) {
   if ((int64_t)num_seqs * a.num_q_heads > 0x7fffffffLL) return cudaErrorInvalidValue;
   switch (head_dim) {
-    case 64: return launch_reduce_dim<T, 64>(a, num_seqs, stream, dependent);
-    case 128: return launch_reduce_dim<T, 128>(a, num_seqs, stream, dependent);
-    case 256: return launch_reduce_dim<T, 256>(a, num_seqs, stream, dependent);
+    case 64: return sparse ? launch_reduce_dim<T, 64, true>(a, num_seqs, stream, dependent)
+                           : launch_reduce_dim<T, 64, false>(a, num_seqs, stream, dependent);
+    case 128: return sparse ? launch_reduce_dim<T, 128, true>(a, num_seqs, stream, dependent)
+                            : launch_reduce_dim<T, 128, false>(a, num_seqs, stream, dependent);
+    case 256: return sparse ? launch_reduce_dim<T, 256, true>(a, num_seqs, stream, dependent)
+                            : launch_reduce_dim<T, 256, false>(a, num_seqs, stream, dependent);
   }
   return cudaErrorInvalidValue;
 }
@@ -4203,10 +4208,11 @@ pa_status launch_partitions(const DecodeArgs& a, pa_dtype dtype, int head_dim, i
 }
 
 pa_status launch_reduce_any(const DecodeArgs& a, pa_dtype dtype, int head_dim, int num_seqs, cudaStream_t s,
-                            bool dependent = false) {
-  const cudaError_t err = dtype == PA_F32    ? launch_reduce<float>(a, head_dim, num_seqs, s, dependent)
-                          : dtype == PA_BF16 ? launch_reduce<__nv_bfloat16>(a, head_dim, num_seqs, s, dependent)
-                                             : launch_reduce<__half>(a, head_dim, num_seqs, s, dependent);
+                            bool dependent = false, bool sparse = false) {
+  const cudaError_t err =
+      dtype == PA_F32    ? launch_reduce<float>(a, head_dim, num_seqs, s, dependent, sparse)
+      : dtype == PA_BF16 ? launch_reduce<__nv_bfloat16>(a, head_dim, num_seqs, s, dependent, sparse)
+                         : launch_reduce<__half>(a, head_dim, num_seqs, s, dependent, sparse);
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode reduce kernel: %s", cudaGetErrorString(err));
   return PA_OK;
 }
@@ -4577,7 +4583,7 @@ extern "C" pa_status pa_decode_shared_prefix(const void* q, const void* key_cach
                              : launch_shared_seg<__half, 128>(a, dtype, num_chunks, chunks, members, num_members,
                                                               first_partition, num_seqs, others, s);
     if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode shared-prefix kernel: %s", cudaGetErrorString(err));
-    return launch_reduce_any(a, dtype, head_dim, num_seqs, s, /*dependent=*/true);
+    return launch_reduce_any(a, dtype, head_dim, num_seqs, s, /*dependent=*/true, /*sparse=*/true);
   }
   if (joint) {
     if (!aligned16(chunks)) return fail(PA_ERR_INVALID, "decode_shared_prefix: chunks must be 16-byte aligned");
