@@ -2053,7 +2053,8 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
     decode_shared_seg_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k, int tma_k,
                              const int32_t* __restrict__ chunks, int num_chunks,
                              const int32_t* __restrict__ members, int num_members,
-                             const int32_t* __restrict__ first_partition, int num_seqs, int fault) {
+                             const int32_t* __restrict__ first_partition, int num_seqs, int wait_at_start,
+                             int fault) {
   using S = SegShape<D, STAGES>;
   constexpr int E = S::kEpilogueSteps;
   extern __shared__ uint8_t smem_raw[];
@@ -2122,6 +2123,10 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
   // three steps before the current one ends without waiting for the table.
   int win_cur = -1, win_nxt = -1, nxt_cur = -1, nxt_nxt = -1;
   if (producer) {
+    // Launched as a programmatic dependent of an arbitrary kernel: nothing is read
+    // before that grid has finished (its launch and the set-up below overlap it).
+    // Every global write of this grid follows a producer's load, hence this wait.
+    if (wait_at_start) asm volatile("griddepcontrol.wait;\n" ::: "memory");
     seg_walk_init<E>(walk, a, chunks, num_chunks, members, num_members, first_partition, num_seqs,
                      pw == 0 && lane == 0 && blockIdx.x == 0);
     have = next_seg(seg);
@@ -2999,11 +3004,12 @@ __global__ void __launch_bounds__(Tc05dShape<D, STAGES>::kThreads, 2)
 // w + WPI, ... with its own running maximum (the lanes compute 32 weights per
 // round; partial rows are loaded in prefetched groups), then the item's warps
 // merge through shared memory the same way.  A partition whose l is 0 adds
-// nothing; with SPARSE (the balanced shared-prefix kernel leaves slots it
-// marks empty, l = 0, unwritten) such a row is not read at all -- otherwise
-// rows are requested before their l is known.  Launched as a programmatic
-// dependent of the kernel that writes the partials, it waits for that grid
-// before reading them.
+// nothing.  With SPARSE (the balanced shared-prefix kernel marks slots empty,
+// l = 0, without writing their rows) a row's contribution is selected rather
+// than multiplied by its weight, so that whatever an unwritten row holds never
+// reaches the sum; rows are requested before the weights are known either
+// way.  Launched as a programmatic dependent of the kernel that writes the
+// partials, it waits for that grid before reading them.
 // ---------------------------------------------------------------------------
 template <typename T, int D, int WPI, bool SPARSE>
 __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel(const DecodeArgs a, int num_seqs) {
@@ -3031,13 +3037,11 @@ __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel
   // This warp's partitions are p = sub + WPI * (lane + 32 c), c = 0, 1, ...
   // Lane `lane` holds m and l of its first one; the first UNROLL partial rows
   // are requested before the max is known, and each group of rows is
-  // accumulated while the next group is in flight.  `lw` is the lane's l of
-  // the current group: rows with l = 0 are not read.
-  auto load_rows = [&](float (&x)[UNROLL][VPL], int p0, int k, int cnt, float lw) {
+  // accumulated while the next group is in flight.
+  auto load_rows = [&](float (&x)[UNROLL][VPL], int p0, int k, int cnt) {
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {
-      const bool present = SPARSE ? __shfl_sync(kFull, lw, min(k + u, 31)) > 0.f : true;
-      if (k + u < cnt && present) {
+      if (k + u < cnt) {
         const float* src = a.o_part + (base + p0 + WPI * (k + u)) * D + lane * VPL;
         if constexpr (VPL % 4 == 0) {
 #pragma unroll
@@ -3065,7 +3069,7 @@ __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel
     l_first = a.l_part[base + pf];
   }
   float x[UNROLL][VPL];
-  load_rows(x, sub, 0, merge ? min(32, (np - sub + WPI - 1) / WPI) : 0, l_first);
+  load_rows(x, sub, 0, merge ? min(32, (np - sub + WPI - 1) / WPI) : 0);
   float mx = m_first;
   if (merge)
     for (int p = pf + WPI * 32; p < np; p += WPI * 32) mx = fmaxf(mx, a.m_part[base + p]);
@@ -3087,16 +3091,19 @@ __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel
       }
       lsum += wt;
       const int cnt = min(32, (np - p0 + WPI - 1) / WPI);
-      if (c > 0) load_rows(x, p0, 0, cnt, lcur);
+      if (c > 0) load_rows(x, p0, 0, cnt);
       for (int k = 0; k < cnt; k += UNROLL) {
         float xn[UNROLL][VPL];
         const bool more = k + UNROLL < cnt;
-        if (more) load_rows(xn, p0, k + UNROLL, cnt, lcur);
+        if (more) load_rows(xn, p0, k + UNROLL, cnt);
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
           const float wk = __shfl_sync(kFull, wt, min(k + u, 31));
 #pragma unroll
-          for (int i = 0; i < VPL; ++i) acc[i] = fmaf(k + u < cnt ? wk : 0.f, x[u][i], acc[i]);
+          for (int i = 0; i < VPL; ++i) {
+            if constexpr (SPARSE) acc[i] = (k + u < cnt && wk > 0.f) ? fmaf(wk, x[u][i], acc[i]) : acc[i];
+            else acc[i] = fmaf(k + u < cnt ? wk : 0.f, x[u][i], acc[i]);
+          }
         }
         if (more) {
 #pragma unroll
@@ -3885,8 +3892,12 @@ cudaError_t launch_shared_seg(const DecodeArgs& a, pa_dtype dtype, int num_chunk
   std::memset(&mk, 0, sizeof(mk));
   const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * a.block_size;
   const int tma_k = rows < (1ll << 31) && encode_cache_map(&mk, a.key_cache, dtype, rows, D) ? 1 : 0;
-  return launch_pdl(kernel, dim3(sm_count()), dim3(S::kThreads), S::kSmemBytes, stream, dependent, a, mk, tma_k,
-                    chunks, num_chunks, members, num_members, first_partition, num_seqs, (int)g_fault.load());
+  // Always a programmatic dependent: after a per-sequence kernel (`dependent`) it
+  // reads inputs that kernel does not write and only waits for it at the end; after
+  // any other kernel it waits before its first read.
+  return launch_pdl(kernel, dim3(sm_count()), dim3(S::kThreads), S::kSmemBytes, stream, true, a, mk, tma_k,
+                    chunks, num_chunks, members, num_members, first_partition, num_seqs, dependent ? 0 : 1,
+                    (int)g_fault.load());
 }
 
 std::atomic<int> g_shared_kernel{PA_SHARED_PREFIX_AUTO};

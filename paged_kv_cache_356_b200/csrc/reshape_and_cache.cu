@@ -23,6 +23,10 @@ __global__ void __launch_bounds__(kThreads)
                              int chunks_per_row, int rows_per_cta, int64_t num_slots, int block_size,
                              uint4* __restrict__ key_cache, uint4* __restrict__ value_cache,
                              int32_t* status) {
+  // A kernel launched after this one as a programmatic dependent (the decode
+  // that reads these rows waits for this grid before it reads anything) may
+  // start its own set-up now.
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   const int local_row = threadIdx.x / chunks_per_row;
   const int chunk = threadIdx.x - local_row * chunks_per_row;
   if (local_row >= rows_per_cta) return;
