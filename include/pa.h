@@ -366,6 +366,16 @@ PA_API pa_status pa_set_shared_prefix_kernel(pa_shared_prefix_kernel kernel);
 #define PA_FAULT_WITHHOLD_FIRST_ITEM 1
 PA_API pa_status pa_set_fault_injection(int32_t mode);
 
+/* Test hook for an arithmetic helper of the decode kernels (the pages have no
+ * counterpart).  y[i] = 2^x[i] for i < n, evaluated on the device as the
+ * softmax of the shared-prefix kernel evaluates it: method 0 = the FMA-pipe
+ * form (range reduction to x = i + f, f in [-1/2, 1/2], and a fitted cubic
+ * for 2^f; maximum relative error 7.6e-5 for -125 <= x <= 127, inputs below
+ * -125 clamped), method 1 = the special-function unit (ex2.approx.ftz.f32).
+ * x and y are device arrays of n floats (16-byte aligned); asynchronous on
+ * the stream; PA_ERR_INVALID for a NULL array, n < 0 or another method. */
+PA_API pa_status pa_eval_exp2(const float* x, float* y, int64_t n, int32_t method, void* stream);
+
 /* Which partition kernel pa_decode runs (process-wide; default AUTO).
  * AUTO picks the tensor-core kernel whenever it supports the call (bf16/f16,
  * head_dim 64/128/256, G <= 8, block_size a multiple of 16 up to 256) and the

@@ -65,6 +65,7 @@ SIGNATURES = {
     "pa_set_decode_kernel": (_i32, [_i32]),
     "pa_set_shared_prefix_kernel": (_i32, [_i32]),
     "pa_set_fault_injection": (_i32, [_i32]),
+    "pa_eval_exp2": (_i32, [_vp, _vp, _i64, _i32, _vp]),
     "pa_set_decode_tiling": (_i32, [_i32, _i32]),
     "pa_block_alloc_create": (_i32, [_i32, _i32, _pi32, _c.POINTER(_vp)]),
     "pa_block_alloc_destroy": (None, [_vp]),

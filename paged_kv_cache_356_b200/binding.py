@@ -296,6 +296,16 @@ def pa_set_fault_injection(mode: int) -> None:
     _check(_lib.load().pa_set_fault_injection(int(mode)))
 
 
+def pa_eval_exp2(x, method: int = 0, stream=None):
+    """2^x on the device as the decode kernels evaluate it (method 0: FMA-pipe cubic, 1: the
+    special-function unit); ``x`` a contiguous float32 CUDA tensor.  Test hook."""
+    torch = _torch()
+    y = torch.empty_like(x)
+    _check(_lib.load().pa_eval_exp2(_cuda(x, "x", torch.float32), _cuda(y, "y", torch.float32), x.numel(),
+                                    int(method), _stream_handle(stream, x.device)))
+    return y
+
+
 def pa_set_decode_tiling(warps: int, stages: int) -> None:
     _check(_lib.load().pa_set_decode_tiling(int(warps), int(stages)))
 

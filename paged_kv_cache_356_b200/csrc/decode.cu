@@ -4104,6 +4104,26 @@ extern "C" pa_status pa_set_fault_injection(int32_t mode) {
   return PA_OK;
 }
 
+namespace pa {
+namespace {
+__global__ void eval_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n, int method) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    y[i] = method == 0 ? exp2_poly(x[i]) : ex2_approx(x[i]);
+}
+}  // namespace
+}  // namespace pa
+
+extern "C" pa_status pa_eval_exp2(const float* x, float* y, int64_t n, int32_t method, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y)) || (method != 0 && method != 1))
+    return fail(PA_ERR_INVALID, "eval_exp2: bad arguments");
+  if (n == 0) return PA_OK;
+  const int64_t blocks = std::min<int64_t>((n + 255) / 256, 4096);
+  eval_exp2_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n, method);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "eval_exp2: %s", cudaGetErrorString(err));
+  return PA_OK;
+}
+
 extern "C" pa_status pa_set_shared_prefix_kernel(pa_shared_prefix_kernel k) {
   if (k != PA_SHARED_PREFIX_AUTO && k != PA_SHARED_PREFIX_TCGEN05 && k != PA_SHARED_PREFIX_MMA_SYNC &&
       k != PA_SHARED_PREFIX_TCGEN05_SERIAL && k != PA_SHARED_PREFIX_TCGEN05_2CTA &&
