@@ -1916,7 +1916,8 @@ __device__ __forceinline__ int seg_cut(const SegWalk& w, int k, const DecodeArgs
 template <int E>
 __device__ __forceinline__ void seg_walk_init(SegWalk& w, const DecodeArgs& a, const int32_t* __restrict__ chunks,
                                               int num_chunks, const int32_t* __restrict__ members, int num_members,
-                                              const int32_t* __restrict__ first_partition, int num_seqs, bool report) {
+                                              const int32_t* __restrict__ first_partition, int num_seqs,
+                                              bool fold_tails, bool report) {
   const int lane = threadIdx.x & 31;
   // Shared units per kv head and the tail weight per kv head.  The chunk, member
   // and sequence loads of one pass are independent (one round trip); plans of up
@@ -1929,8 +1930,8 @@ __device__ __forceinline__ void seg_walk_init(SegWalk& w, const DecodeArgs& a, c
     const int i = i0 + lane;
     const SegChunk ci = i < num_chunks ? seg_chunk(a, chunks, i, num_members, num_seqs, report) : SegChunk{0, 0, 0, 0};
     const int n = seg_lane_units(ci.sp);
-    int T, fp, ctx;
-    seg_tail_of(a, first_partition, i, num_seqs, T, fp, ctx);
+    int T = 0, fp, ctx;
+    if (fold_tails) seg_tail_of(a, first_partition, i, num_seqs, T, fp, ctx);
     const int incl = warp_incl_sum(n);
     if (i0 == 0) {
       w.cl = ci;
@@ -2053,8 +2054,8 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
     decode_shared_seg_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k, int tma_k,
                              const int32_t* __restrict__ chunks, int num_chunks,
                              const int32_t* __restrict__ members, int num_members,
-                             const int32_t* __restrict__ first_partition, int num_seqs, int wait_at_start,
-                             int fault) {
+                             const int32_t* __restrict__ first_partition, int num_seqs, int fold_tails,
+                             int wait_at_start, int fault) {
   using S = SegShape<D, STAGES>;
   constexpr int E = S::kEpilogueSteps;
   extern __shared__ uint8_t smem_raw[];
@@ -2127,7 +2128,7 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
     // before that grid has finished (its launch and the set-up below overlap it).
     // Every global write of this grid follows a producer's load, hence this wait.
     if (wait_at_start) asm volatile("griddepcontrol.wait;\n" ::: "memory");
-    seg_walk_init<E>(walk, a, chunks, num_chunks, members, num_members, first_partition, num_seqs,
+    seg_walk_init<E>(walk, a, chunks, num_chunks, members, num_members, first_partition, num_seqs, fold_tails != 0,
                      pw == 0 && lane == 0 && blockIdx.x == 0);
     have = next_seg(seg);
     if (have) {
@@ -3879,7 +3880,7 @@ cudaError_t launch_shared_tc05d(const DecodeArgs& a, const CUtensorMap& mk, cons
 template <typename T, int D>
 cudaError_t launch_shared_seg(const DecodeArgs& a, pa_dtype dtype, int num_chunks, const int32_t* chunks,
                               const int32_t* members, int num_members, const int32_t* first_partition, int num_seqs,
-                              bool dependent, cudaStream_t stream) {
+                              bool dependent, cudaStream_t stream, bool fold_tails = true) {
   constexpr int kStages = D == 128 ? 5 : 8;
   using S = SegShape<D, kStages>;
   static std::atomic<uint64_t> done{0};
@@ -3896,8 +3897,8 @@ cudaError_t launch_shared_seg(const DecodeArgs& a, pa_dtype dtype, int num_chunk
   // reads inputs that kernel does not write and only waits for it at the end; after
   // any other kernel it waits before its first read.
   return launch_pdl(kernel, dim3(sm_count()), dim3(S::kThreads), S::kSmemBytes, stream, true, a, mk, tma_k,
-                    chunks, num_chunks, members, num_members, first_partition, num_seqs, dependent ? 0 : 1,
-                    (int)g_fault.load());
+                    chunks, num_chunks, members, num_members, first_partition, num_seqs, fold_tails ? 1 : 0,
+                    dependent ? 0 : 1, (int)g_fault.load());
 }
 
 std::atomic<int> g_shared_kernel{PA_SHARED_PREFIX_AUTO};
@@ -4401,6 +4402,7 @@ extern "C" pa_status pa_decode_verify(const void* q, const void* key_cache, cons
                                     "%% 16 == 0, G <= %d and contexts beyond one partition", PA_PREFIX_QUERIES_PER_CTA);
   const bool joint = joint_ok && (path == PA_VERIFY_JOINT ||
                                   (path == PA_VERIFY_AUTO && (int64_t)num_query_tokens * G > kVerifyJointRows));
+  bool balanced = false;  // the balanced joint kernel ran (its merge skips the slots it leaves empty)
   if (joint) {
     const VerifyLayout lay = verify_layout(num_seqs, num_query_tokens, num_q_heads, head_dim, partitions);
     if (workspace_bytes < lay.total)
@@ -4417,11 +4419,32 @@ extern "C" pa_status pa_decode_verify(const void* q, const void* key_cache, cons
     // The joint kernel indexes q, the partials and its members with H_q heads per member.
     DecodeArgs aj = a;
     aj.num_q_heads = num_q_heads;
-    const dim3 grid(num_seqs * cps, num_kv_heads, max_visible);
-    err = dtype == PA_BF16 ? launch_shared_dim<__nv_bfloat16>(aj, head_dim, grid, chunks, members, num_members,
-                                                              num_members, dtype, s)
-                           : launch_shared_dim<__half>(aj, head_dim, grid, chunks, members, num_members, num_members,
-                                                       dtype, s);
+    const int shared_choice = g_shared_kernel.load();
+    const int64_t units = (int64_t)num_kv_heads * num_seqs * cps * ((int64_t)max_visible * 8 + 3);
+    balanced = (shared_choice == PA_SHARED_PREFIX_AUTO || shared_choice == PA_SHARED_PREFIX_TCGEN05) &&
+               units < kSegMaxUnits;
+    if (balanced) {
+      // The balanced kernel over the visible partitions only (the per-sequence kernel
+      // keeps the partitions the causal limits cut); it waits for the plan kernel first.
+      // Its members are token ids b * T + t, so they are checked against num_members.
+      const int nc = num_seqs * cps;
+      err = head_dim == 64
+                ? (dtype == PA_BF16 ? launch_shared_seg<__nv_bfloat16, 64>(aj, dtype, nc, chunks, members, num_members,
+                                                                           nullptr, num_members, false, s, false)
+                                    : launch_shared_seg<__half, 64>(aj, dtype, nc, chunks, members, num_members,
+                                                                    nullptr, num_members, false, s, false))
+                : (dtype == PA_BF16 ? launch_shared_seg<__nv_bfloat16, 128>(aj, dtype, nc, chunks, members,
+                                                                            num_members, nullptr, num_members, false,
+                                                                            s, false)
+                                    : launch_shared_seg<__half, 128>(aj, dtype, nc, chunks, members, num_members,
+                                                                     nullptr, num_members, false, s, false));
+    } else {
+      const dim3 grid(num_seqs * cps, num_kv_heads, max_visible);
+      err = dtype == PA_BF16 ? launch_shared_dim<__nv_bfloat16>(aj, head_dim, grid, chunks, members, num_members,
+                                                                num_members, dtype, s)
+                             : launch_shared_dim<__half>(aj, head_dim, grid, chunks, members, num_members,
+                                                         num_members, dtype, s);
+    }
     if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode_verify joint kernel: %s", cudaGetErrorString(err));
     v.skip_visible = 1;
   }
@@ -4434,7 +4457,7 @@ extern "C" pa_status pa_decode_verify(const void* q, const void* key_cache, cons
                              : launch_verify_cc<__half>(a, v, head_dim, num_seqs, partitions, s);
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode_verify partition kernel: %s", cudaGetErrorString(err));
   if (partitions <= 1) return PA_OK;
-  return launch_reduce_any(a, dtype, head_dim, num_seqs, s);
+  return launch_reduce_any(a, dtype, head_dim, num_seqs, s, /*dependent=*/false, /*sparse=*/balanced);
 }
 
 // ---------------------------------------------------------------------------

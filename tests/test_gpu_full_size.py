@@ -135,9 +135,16 @@ def test_verify_step_on_sampled_sequences(verify_run, num_tokens):
     saved = run.key_cache[pages, :, offs, :].clone(), run.value_cache[pages, :, offs, :].clone()
     pa.pa_reshape_and_cache(run._to_device(dk), run._to_device(dv), torch.from_numpy(slots.astype(np.int64)).cuda(),
                             run.key_cache, run.value_cache)
+    # NaN bytes in the workspace: a partial that no kernel wrote shows up in the sampled rows
+    need = pa.pa_decode_verify_workspace_size(w.num_seqs, T, w.num_q_heads, w.head_dim,
+                                              run.block_tables.shape[1] * w.block_size)
+    ws = torch.full((max(need, 1),), 0xFF, dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = pa.pa_decode_verify(run._to_device(q), run.key_cache, run.value_cache, run.block_tables,
-                              run.context_lens, w.scale)
+                              run.context_lens, w.scale, workspace=ws, dev_status=status)
     torch.cuda.synchronize()
+    assert status.item() == 0, f"device status {status.item():#x}"
+    del ws
     # the trace's own K/V back in place for the next case
     run.key_cache[pages, :, offs, :] = saved[0]
     run.value_cache[pages, :, offs, :] = saved[1]

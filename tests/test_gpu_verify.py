@@ -73,10 +73,21 @@ def _run(case, kernel, tables=None, ctx=None, status=None, path="auto"):
     dt = case["dtype"]
     t = case["tables"] if tables is None else tables
     c = case["ctx"] if ctx is None else ctx
-    out = pa.pa_decode_verify(_dev(case["q"], dt), _dev(case["kc"], dt), _dev(case["vc"], dt),
+    q = _dev(case["q"], dt)
+    # The workspace starts as NaN bytes, so a partial that no kernel wrote cannot pass for a stale
+    # correct one left by an earlier call.
+    need = pa.pa_decode_verify_workspace_size(q.shape[0], q.shape[1], q.shape[2], q.shape[3],
+                                              t.shape[1] * case["kc"].shape[2])
+    ws = torch.full((max(need, 1),), 0xFF, dtype=torch.uint8, device="cuda")
+    own_status = status is None
+    if own_status:
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = pa.pa_decode_verify(q, _dev(case["kc"], dt), _dev(case["vc"], dt),
                               torch.from_numpy(t).cuda(), torch.from_numpy(np.asarray(c, np.int32)).cuda(),
-                              case["scale"], dev_status=status)
+                              case["scale"], workspace=ws, dev_status=status)
     torch.cuda.synchronize()
+    if own_status:
+        assert status.item() == 0, f"device status {status.item():#x}"
     return out
 
 
@@ -124,13 +135,15 @@ def _edge_contexts(num_tokens):
     return [c for c in out if c > 0]
 
 
-@pytest.mark.parametrize("joint_kernel", ["tcgen05", "mma_sync"])
+@pytest.mark.parametrize("joint_kernel", ["tcgen05", "tcgen05_items", "mma_sync"])
 @pytest.mark.parametrize("num_tokens,hq,hkv,d", [(4, 64, 8, 128), (3, 8, 2, 64), (5, 32, 1, 128), (9, 16, 1, 64)],
                          ids=["T4-G8", "T3-G4-d64", "T5-G32-two-chunks", "T9-G16-two-chunks"])
 def test_joint_path_partition_edges(num_tokens, hq, hkv, d, joint_kernel):
     """The joint kernel's plan (built on the device) against the causal limits; G * T above 128
-    splits a sequence's tokens over several chunks."""
+    splits a sequence's tokens over several chunks.  tcgen05 is the balanced kernel (equal ranges of
+    steps per CTA), tcgen05_items the one-CTA-per-partition kernel."""
     pa.pa_set_shared_prefix_kernel({"tcgen05": pa.PA_SHARED_PREFIX_TCGEN05,
+                                    "tcgen05_items": pa.PA_SHARED_PREFIX_TCGEN05_ITEMS,
                                     "mma_sync": pa.PA_SHARED_PREFIX_MMA_SYNC}[joint_kernel])
     case = _case(300 + num_tokens, _edge_contexts(num_tokens), num_tokens, hq, hkv, d, 16, "bf16")
     assert_decode_close(_run(case, "tc", path="joint"), _oracle(case), "bf16", joint_kernel)
