@@ -52,6 +52,9 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle time budget for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-slices", type=int, default=5,
+                    help="decode workloads: runs of sequences whose copies overlap the other runs' kernels in "
+                         "the end-to-end step (1: copy in, compute, copy out in turn)")
     ap.add_argument("--no-clocks", action="store_true", help="skip the nvidia-smi clock record (profiler runs)")
     ap.add_argument("--no-configs", action="store_true",
                     help="measure the headline workload only (by default a 1-GPU run also measures every other "
@@ -767,7 +770,9 @@ def run_ours(args):
 
     # end to end through the API, host buffers: export tables, copy inputs in, decode, read the output back
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and T == 0 and run.plan is None and w.kind == "independent":
+        e2e = end_to_end_decode(args, torch, pa, run, w, world, dist, (sb.q, sb.kd, sb.vd), args.e2e_slices)
+    elif not args.no_e2e:
         if T > 0:
             decode = lambda d_q, d_tab, d_ctx, d_out: pa.pa_decode_verify(
                 d_q, run.key_cache, run.value_cache, d_tab, d_ctx, w.scale, out=d_out, workspace=sb.ws)
@@ -904,6 +909,195 @@ def end_to_end(args, torch, pa, run, w, unique, world, dist, inputs, decode):
             "d2h_bytes_per_step": d2h, "ms_per_step": 1000 * elapsed / args.steps,
             "includes": "host table export (C ABI), pinned H2D of q/new K,V/slots/tables/lengths, "
                         "reshape_and_cache + decode, D2H of out, stream sync"}
+
+
+def end_to_end_decode(args, torch, pa, run, w, world, dist, inputs, slices):
+    """Decode steps through the public API from pinned host buffers, each growing every sequence by one
+    token as a serving loop does; wall clock, each step synchronised (its output in host memory) before
+    the next is launched.
+
+    Host, per step: ``pa_block_alloc_append_tokens`` (the new tokens' slots) and
+    ``pa_block_alloc_table_updates`` (the table entries that changed), done for step i + 1 while step
+    i runs on the device (the allocator never waits for attention outputs), into one of two sets of
+    pinned buffers.  Device, per step, one CUDA graph: copies in of the updates, lengths, slots, q and
+    the new tokens' K/V; ``pa_block_tables_apply`` on a device copy of the tables; then, per slice of
+    the batch, ``pa_reshape_and_cache`` + ``pa_decode`` once the slice's inputs have landed and the
+    copy out of its rows on a third stream, so the copies of one slice overlap the kernels of another.
+    ``inputs`` = (q, new K, new V) of the device-resident step."""
+    q_dev, kd, vd = inputs
+    n, bs = w.num_seqs, w.block_size
+    warm = 3
+    mb = -(-(w.max_context_len + warm + args.steps + 2) // bs)   # room for the tokens the steps add
+    kmax = 2 * n   # updates a captured step carries; a step with more applies them before its launch
+    pin = dict(pin_memory=True)
+
+    def pinned(shape, dtype, fill=None):
+        h = torch.empty(shape, dtype=dtype, **pin)
+        if fill is not None:
+            h.fill_(fill)
+        return h
+
+    h_q, h_k, h_v = (pinned(x.shape, x.dtype) for x in (q_dev, kd, vd))
+    for h, x in ((h_q, q_dev), (h_k, kd), (h_v, vd)):
+        h.copy_(x)
+    h_s = [pinned(n, torch.int64) for _ in range(2)]
+    h_ctx = [pinned(n, torch.int32) for _ in range(2)]
+    h_upd = [pinned((kmax, 3), torch.int32, -1) for _ in range(2)]     # the graph's fixed-size buffer
+    h_big = [pinned((n * mb, 3), torch.int32) for _ in range(2)]       # what table_updates writes
+    h_pairs = [pinned((n, 2), torch.int64) for _ in range(2)]
+    h_out = pinned(q_dev.shape, q_dev.dtype)
+    d_q, d_k, d_v = (torch.empty_like(x, device="cuda") for x in (h_q, h_k, h_v))
+    d_s, d_ctx = torch.empty(n, dtype=torch.int64, device="cuda"), torch.empty(n, dtype=torch.int32, device="cuda")
+    d_upd = torch.empty((kmax, 3), dtype=torch.int32, device="cuda")
+    d_big = torch.empty((n * mb, 3), dtype=torch.int32, device="cuda")
+    d_pairs = torch.empty((n, 2), dtype=torch.int64, device="cuda")
+    d_tab = torch.full((n, mb), -1, dtype=torch.int32, device="cuda")
+    d_out = torch.empty_like(q_dev)
+    need = pa.pa_decode_workspace_size(n, w.num_q_heads, w.head_dim, mb * bs)
+    ws = [torch.empty(max(need, 256), dtype=torch.uint8, device="cuda") for _ in range(2)]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    seqs = np.arange(n, dtype=np.int64)
+    filled = [0, 0]            # non-padding rows written last into each h_upd
+    # Slices: the first and the last half the size of the others (the copy in before the first kernel
+    # and the copy out after the last one are what the overlap cannot hide).
+    weights = [1] if slices == 1 else [1] + [2] * (slices - 2) + [1]
+    cuts = np.rint(np.cumsum([0] + weights) / sum(weights) * n).astype(int)
+    bounds = [(int(a), int(b)) for a, b in zip(cuts[:-1], cuts[1:]) if b > a]
+    s_in, s_out, s_alt = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    moved = {"extra": 0}
+
+    def prep(b):
+        """Host half of the next step, into buffer set b."""
+        slots, cow = run.alloc.append_tokens(seqs)
+        h_s[b].numpy()[:] = slots
+        upd, _ = run.alloc.table_updates(seqs, mb, out=h_big[b].numpy(), lens_out=h_ctx[b].numpy())
+        k = len(upd)
+        u = h_upd[b].numpy()
+        small = k <= kmax
+        if small:
+            u[:k] = upd
+        u[k if small else 0:filled[b]] = -1
+        filled[b] = k if small else 0
+        return k, cow[cow[:, 0] >= 0]
+
+    def device_step(b):
+        """Device half of a step from buffer set b, on the current stream (captured or eager)."""
+        cs = torch.cuda.current_stream()
+        fork = torch.cuda.Event()
+        fork.record(cs)
+        s_in.wait_event(fork)
+        s_out.wait_event(fork)
+        ev_meta, ev_in, ev_done = torch.cuda.Event(), [torch.cuda.Event() for _ in bounds], []
+        with torch.cuda.stream(s_in):
+            d_upd.copy_(h_upd[b], non_blocking=True)
+            d_ctx.copy_(h_ctx[b], non_blocking=True)
+            d_s.copy_(h_s[b], non_blocking=True)
+            ev_meta.record(s_in)
+            for (r0, r1), ev in zip(bounds, ev_in):
+                d_q[r0:r1].copy_(h_q[r0:r1], non_blocking=True)
+                d_k[r0:r1].copy_(h_k[r0:r1], non_blocking=True)
+                d_v[r0:r1].copy_(h_v[r0:r1], non_blocking=True)
+                ev.record(s_in)
+        cs.wait_event(ev_meta)
+        pa.pa_block_tables_apply(d_tab, d_upd, kmax, dev_status=status, stream=cs)
+        applied = torch.cuda.Event()
+        applied.record(cs)
+        s_alt.wait_event(applied)
+        # Slices alternate between two compute streams (each with its own workspace), so that one
+        # slice's kernels start while the previous slice's last CTAs and merge finish.
+        for i, ((r0, r1), ev) in enumerate(zip(bounds, ev_in)):
+            st = cs if i % 2 == 0 else s_alt
+            st.wait_event(ev)
+            pa.pa_reshape_and_cache(d_k[r0:r1], d_v[r0:r1], d_s[r0:r1], run.key_cache, run.value_cache,
+                                    dev_status=status, stream=st)
+            pa.pa_decode(d_q[r0:r1], run.key_cache, run.value_cache, d_tab[r0:r1], d_ctx[r0:r1], w.scale,
+                         out=d_out[r0:r1], workspace=ws[i % 2], dev_status=status, stream=st)
+            done = torch.cuda.Event()
+            done.record(st)
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                h_out[r0:r1].copy_(d_out[r0:r1], non_blocking=True)
+            ev_done.append(done)
+        join = torch.cuda.Event()
+        join.record(s_out)
+        cs.wait_event(join)
+        alt_done = torch.cuda.Event()
+        alt_done.record(s_alt)
+        cs.wait_event(alt_done)
+
+    def launch(b, pending, graphs):
+        """Work the captured step cannot carry (many updates, copy-on-write pairs), then the step."""
+        k, forked = pending
+        cs = torch.cuda.current_stream()
+        if k > kmax:
+            d_big[:k].copy_(h_big[b][:k], non_blocking=True)
+            pa.pa_block_tables_apply(d_tab, d_big, k, dev_status=status, stream=cs)
+            moved["extra"] += k * 12
+        if len(forked):
+            h_pairs[b][:len(forked)].copy_(torch.from_numpy(forked.astype(np.int64)))
+            d_pairs[:len(forked)].copy_(h_pairs[b][:len(forked)], non_blocking=True)
+            pa.pa_copy_blocks(run.key_cache, run.value_cache, d_pairs[:len(forked)], dev_status=status, stream=cs)
+            moved["extra"] += len(forked) * 16
+        if graphs is None:
+            device_step(b)
+        else:
+            graphs[b].replay()
+
+    def steps(count, graphs, b0):
+        pending = prep(b0)
+        for i in range(count):
+            b = (b0 + i) % 2
+            launch(b, pending, graphs)
+            if i + 1 < count:
+                pending = prep(1 - b)
+            torch.cuda.current_stream().synchronize()
+        return (b0 + count) % 2
+
+    b = steps(warm, None, 0)           # eager: sets up the device tables (whole rows) and warms the calls
+    graphs = []
+    for p in range(2):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            device_step(p)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    moved["extra"] = 0
+    ctx0 = np.array([run.alloc.num_tokens(int(x)) for x in seqs], dtype=np.int64)
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    steps(args.steps, graphs, b)
+    elapsed = time.perf_counter() - t0
+    torch.cuda.synchronize()
+    # The device tables equal the full export, and the last output equals one device-resident call on
+    # the same state.
+    full, lens = run.alloc.block_tables(seqs, mb)
+    if not np.array_equal(d_tab.cpu().numpy(), full):
+        raise RuntimeError("end-to-end: the device tables differ from the full export")
+    ref = torch.empty_like(d_out)
+    pa.pa_decode(d_q, run.key_cache, run.value_cache, torch.from_numpy(full).cuda(), torch.from_numpy(lens).cuda(),
+                 w.scale, out=ref, workspace=ws[0])
+    torch.cuda.synchronize()
+    if not torch.equal(h_out.view(torch.int16), ref.cpu().view(torch.int16)):
+        raise RuntimeError("end-to-end: output differs from the device-resident call")
+    if status.item() != 0:
+        raise RuntimeError(f"end-to-end: device status {status.item():#x}")
+    del graphs
+    per_token = 2 * w.num_kv_heads * w.head_dim * w.elem_bytes
+    # timed step j reads ctx0 + j tokens per sequence (independent pages: unique bytes = logical bytes)
+    kv = sum(int(ctx0.sum()) + j * n for j in range(1, args.steps + 1)) * per_token
+    elapsed, (kv,) = reduce_over_ranks(elapsed, [kv], world, "cuda")
+    h2d = (sum(x.numel() * x.element_size() for x in (h_q, h_k, h_v, h_s[0], h_ctx[0], h_upd[0]))
+           + moved["extra"] / args.steps)
+    d2h = h_out.numel() * h_out.element_size()
+    return {"value": kv / elapsed / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": 1000 * elapsed / args.steps, "slices": slices,
+            "includes": "per step: host append_tokens + table_updates (C ABI; for step i + 1 while step i runs), "
+                        "then one CUDA graph: pinned H2D of table updates (fixed buffer of "
+                        f"{kmax}), lengths, slots, q and new K/V, pa_block_tables_apply, and per slice of the "
+                        f"batch (sizes {[b - a for a, b in bounds]}, on two alternating compute streams) "
+                        "reshape_and_cache + decode with its rows copied back on a copy-out stream; stream sync "
+                        "before the next step; every sequence grows one token per step"}
 
 
 # ---------------------------------------------------------------------------------------------

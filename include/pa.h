@@ -68,6 +68,7 @@ typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1, PA_F16 = 2 } pa_dtype;
 #define PA_DEV_BAD_PAIR 8 /* copy_blocks: a source or destination page is outside the pool  */
 #define PA_DEV_BAD_PLAN 16 /* decode_shared_prefix: a prefix-plan entry is out of range       */
 #define PA_DEV_TIMEOUT 32  /* a bounded wait inside a kernel gave up (the CTA's rows are not written) */
+#define PA_DEV_BAD_UPDATE 64 /* block_tables_apply: an update's row or column is outside the tables */
 
 /* Tokens per split-context partition of pa_decode. */
 #define PA_PARTITION_TOKENS 512
@@ -115,6 +116,31 @@ PA_API pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_
                          int32_t num_pairs, int32_t num_blocks, int32_t block_size,
                          int32_t num_kv_heads, int32_t head_dim, pa_dtype dtype,
                          int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------
+ * pa_block_tables_apply -- write block-table updates into a device copy of
+ * the padded tables (int32 [num_rows][max_blocks_per_seq], row-major).
+ *
+ * [Internals] "2. The Dynamic Block Table": a table gains an entry when a
+ * token starts a new block; [Internals] "Copy-on-Write and Prefix Sharing":
+ * an entry changes when a shared page is forked.  The updates come from
+ * pa_block_alloc_table_updates, so a decode step moves a few entries to the
+ * device instead of every table.
+ *
+ * updates       device int32 [num_updates][3] = (row, column, page); the
+ *               updates of one call must name distinct entries (they are
+ *               written in parallel).  Row -1 marks padding: the triple is
+ *               skipped (a buffer of fixed size, e.g. in a CUDA graph, may
+ *               hold fewer updates).  Any other row outside [0, num_rows), or
+ *               a column outside [0, max_blocks_per_seq), is skipped and
+ *               flagged PA_DEV_BAD_UPDATE.  Pages are written as given (the
+ *               decode kernels check them against the pool).
+ * num_updates   0 returns PA_OK at once.
+ * Asynchronous on `stream`; the caller keeps `updates` alive until it runs.
+ * ---------------------------------------------------------------------- */
+PA_API pa_status pa_block_tables_apply(int32_t* block_tables, int32_t num_rows, int32_t max_blocks_per_seq,
+                                       const int32_t* updates, int32_t num_updates, int32_t* dev_status,
+                                       void* stream);
 
 /* ------------------------------------------------------------------------
  * pa_decode -- one decode step of scaled dot-product attention over the
@@ -487,6 +513,32 @@ PA_API pa_status pa_block_alloc_prefix_plan(const pa_block_alloc* a, const int64
                                             int32_t group_size, int32_t* first_partition, int32_t* chunks,
                                             int32_t* members, int32_t* num_chunks, int32_t* num_members,
                                             int32_t* max_shared_partitions, int32_t* min_shared_partitions);
+
+/* Incremental form of pa_block_alloc_block_tables, for a device copy of the
+ * padded tables of a batch that is updated in place with
+ * pa_block_tables_apply.  The allocator logs, per sequence, the table entries
+ * that changed since the sequence was last exported by this call (a page
+ * taken at a block boundary, a copy-on-write replacement).  For the batch
+ * seqs[n] (row i holds seqs[i]) it writes into updates[cap][3] triples
+ * (row, column, page):
+ *   - every entry of row i, and pad for the entries the row held before past
+ *     the new table (all of them up to max_blocks_per_seq for a row this call
+ *     has not exported yet), when the row is not known to hold seqs[i]'s
+ *     logged state: a row new to this call, a row last exported for another
+ *     sequence, a sequence last exported at another row (or at several), a
+ *     sequence allocated or forked since, or one whose log outgrew its table;
+ *   - otherwise each logged entry of seqs[i] once, with the page it holds now.
+ * *n_out (required) receives the number of triples.  If it is above cap, the
+ * call returns PA_ERR_INVALID and changes nothing: call again with room for
+ * *n_out.  On success the logs of the batch are cleared and the rows
+ * recorded; context_lens_out[n] (may be NULL) receives the token counts.
+ * Applying the triples to the tables this call last produced for the same
+ * max_blocks_per_seq (any contents for rows it has not produced) gives what
+ * pa_block_alloc_block_tables writes.  Changing max_blocks_per_seq starts
+ * over (every row whole).  One consumer per handle: the logs are shared. */
+PA_API pa_status pa_block_alloc_table_updates(pa_block_alloc* a, const int64_t* seqs, int32_t n,
+                                              int32_t max_blocks_per_seq, int32_t pad, int32_t* updates,
+                                              int32_t cap, int32_t* n_out, int32_t* context_lens_out);
 
 /* The free pool front to back into out[cap]; *n_out receives its length. */
 PA_API pa_status pa_block_alloc_free_pool(const pa_block_alloc* a, int32_t* out, int32_t cap,

@@ -15,6 +15,7 @@ PA_F32, PA_BF16, PA_F16 = 0, 1, 2
 PA_DEV_BAD_SLOT, PA_DEV_BAD_PAGE, PA_DEV_BAD_CTX, PA_DEV_BAD_PAIR, PA_DEV_BAD_PLAN = 1, 2, 4, 8, 16
 PA_PREFIX_QUERIES_PER_CTA = 128
 PA_DEV_TIMEOUT = 32
+PA_DEV_BAD_UPDATE = 64
 PA_DECODE_AUTO, PA_DECODE_CUDA_CORES, PA_DECODE_TENSOR_CORES = 0, 1, 2
 PA_SHARED_PREFIX_AUTO, PA_SHARED_PREFIX_TCGEN05, PA_SHARED_PREFIX_MMA_SYNC, PA_SHARED_PREFIX_TCGEN05_SERIAL = 0, 1, 2, 3
 PA_SHARED_PREFIX_TCGEN05_2CTA = 4
@@ -47,6 +48,7 @@ SIGNATURES = {
     "pa_reshape_and_cache": (_i32, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                     _vp, _vp]),
     "pa_copy_blocks": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
+    "pa_block_tables_apply": (_i32, [_vp, _i32, _i32, _vp, _i32, _vp, _vp]),
     "pa_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i64]),
     "pa_decode": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _i32,
                          _vp, _sz, _vp, _vp]),
@@ -76,6 +78,7 @@ SIGNATURES = {
     "pa_block_alloc_slot_mapping": (_i32, [_vp, _i64, _i64, _i64, _pi64]),
     "pa_block_alloc_block_table": (_i32, [_vp, _i64, _pi32, _i32, _pi32]),
     "pa_block_alloc_block_tables": (_i32, [_vp, _pi64, _i32, _pi32, _i32, _i32, _pi32]),
+    "pa_block_alloc_table_updates": (_i32, [_vp, _pi64, _i32, _i32, _i32, _pi32, _i32, _pi32, _pi32]),
     "pa_block_alloc_num_tokens": (_i64, [_vp, _i64]),
     "pa_block_alloc_num_free": (_i32, [_vp]),
     "pa_block_alloc_num_sequences": (_i32, [_vp]),

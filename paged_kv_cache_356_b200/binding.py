@@ -20,6 +20,7 @@ from ._lib import (PA_BF16, PA_DECODE_AUTO, PA_DECODE_CUDA_CORES, PA_DECODE_TENS
                    PA_SHARED_PREFIX_TCGEN05_ITEMS, PA_FAULT_NONE,
                    PA_FAULT_WITHHOLD_FIRST_ITEM, PA_VERIFY_AUTO, PA_VERIFY_JOINT, PA_VERIFY_PER_SEQUENCE,
                    PA_DEV_BAD_CTX, PA_DEV_BAD_PAGE, PA_DEV_BAD_PAIR, PA_DEV_BAD_PLAN, PA_DEV_BAD_SLOT, PA_ERR_NOT_FOUND,
+                   PA_DEV_BAD_UPDATE,
                    PA_ERR_OOM, PA_F16, PA_F32, PA_PARTITION_TOKENS)
 
 
@@ -121,6 +122,23 @@ def pa_copy_blocks(key_cache, value_cache, block_mapping, dev_status=None, strea
         _cuda(key_cache, "key_cache"), _cuda(value_cache, "value_cache"),
         _cuda(block_mapping, "block_mapping", torch.int64), int(block_mapping.shape[0]), nb, bs, hkv, d,
         dtype_code(key_cache.dtype), _opt_status(dev_status), _stream_handle(stream, key_cache.device)))
+
+
+def pa_block_tables_apply(block_tables, updates, num_updates=None, dev_status=None, stream=None) -> None:
+    """Write (row, column, page) updates (device int32 [k, 3], the first num_updates rows) into the
+    device int32 [num_rows, max_blocks_per_seq] tables in place."""
+    torch = _torch()
+    if block_tables.dim() != 2 or block_tables.dtype != torch.int32 or not block_tables.is_contiguous():
+        raise ValueError("block_tables must be a contiguous int32 [num_rows, max_blocks_per_seq] tensor")
+    if updates.dim() != 2 or updates.shape[1] != 3:
+        raise ValueError("updates must be [k, 3]")
+    k = int(updates.shape[0]) if num_updates is None else int(num_updates)
+    if k < 0 or k > updates.shape[0]:
+        raise ValueError("num_updates outside [0, updates.shape[0]]")
+    _check(_lib.load().pa_block_tables_apply(
+        _cuda(block_tables, "block_tables", torch.int32), int(block_tables.shape[0]), int(block_tables.shape[1]),
+        _cuda(updates, "updates", torch.int32), k, _opt_status(dev_status),
+        _stream_handle(stream, block_tables.device)))
 
 
 def pa_decode_workspace_size(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int) -> int:
@@ -408,6 +426,30 @@ def pa_block_alloc_block_tables(handle, seqs: Sequence[int], max_blocks_per_seq:
     return tables, lens
 
 
+def pa_block_alloc_table_updates(handle, seqs: Sequence[int], max_blocks_per_seq: int, pad: int = -1,
+                                 out: Optional[np.ndarray] = None, lens_out: Optional[np.ndarray] = None):
+    """(row, column, page) updates since the last call for the batch `seqs` (int32 [k, 3], a view of
+    `out` when given) and the [n] int32 token counts.  Without `out` the array is sized to fit; a
+    given `out` too small raises (the allocator is left unchanged)."""
+    ids = np.ascontiguousarray(seqs, dtype=np.int64)
+    lens = np.empty(len(ids), dtype=np.int32) if lens_out is None else lens_out
+    if lens.shape != (len(ids),) or lens.dtype != np.int32:
+        raise ValueError("lens_out must be an int32 [n] array")
+    lib = _lib.load()
+    n_out = ctypes.c_int32(0)
+    if out is None:
+        st = lib.pa_block_alloc_table_updates(handle, _i64p(ids), len(ids), max_blocks_per_seq, pad, None, 0,
+                                              ctypes.byref(n_out), None)
+        if st not in (_lib.PA_OK, _lib.PA_ERR_INVALID):
+            _check(st)
+        out = np.empty((max(1, n_out.value), 3), dtype=np.int32)
+    if out.ndim != 2 or out.shape[1] != 3 or out.dtype != np.int32 or not out.flags.c_contiguous:
+        raise ValueError("out must be a C-contiguous int32 [cap, 3] array")
+    _check(lib.pa_block_alloc_table_updates(handle, _i64p(ids), len(ids), max_blocks_per_seq, pad, _i32p(out),
+                                            int(out.shape[0]), ctypes.byref(n_out), _i32p(lens)))
+    return out[:n_out.value], lens
+
+
 def pa_block_alloc_num_tokens(handle, seq: int) -> int:
     return int(_lib.load().pa_block_alloc_num_tokens(handle, seq))
 
@@ -508,6 +550,9 @@ class BlockAllocator:
 
     def block_tables(self, seqs, max_blocks_per_seq, pad=-1, out=None, lens_out=None):
         return pa_block_alloc_block_tables(self.handle, seqs, max_blocks_per_seq, pad, out, lens_out)
+
+    def table_updates(self, seqs, max_blocks_per_seq, pad=-1, out=None, lens_out=None):
+        return pa_block_alloc_table_updates(self.handle, seqs, max_blocks_per_seq, pad, out, lens_out)
 
     def num_tokens(self, seq):
         return pa_block_alloc_num_tokens(self.handle, seq)

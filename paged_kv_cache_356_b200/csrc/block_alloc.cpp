@@ -15,6 +15,7 @@
 // The pool is a fixed ring of num_blocks ids (it can never hold more), so
 // taking from the front and returning to the back are O(1).
 #include <algorithm>
+#include <climits>
 #include <unordered_map>
 #include <vector>
 
@@ -30,8 +31,28 @@ struct pa_block_alloc {
   struct Seq {
     std::vector<int32_t> pages;
     int64_t tokens = 0;
+    // Change log for pa_block_alloc_table_updates: table entries changed since
+    // the sequence was last exported there, or the whole table.
+    std::vector<int32_t> changed;
+    bool whole = true;
+    int32_t row = -1;  // the export row the log is relative to
+    void log(int32_t logical) {
+      if (whole) return;
+      if (changed.size() >= pages.size()) {  // more entries logged than held: export it whole
+        whole = true;
+        changed.clear();
+        return;
+      }
+      changed.push_back(logical);
+    }
   };
   std::unordered_map<int64_t, Seq> seqs;
+  // Rows of the incremental export: the sequence each row was last exported
+  // for (kNoOwner: unknown contents) and how many leading entries it holds.
+  static constexpr int64_t kNoOwner = INT64_MIN;
+  std::vector<int64_t> row_owner;
+  std::vector<int32_t> row_len;
+  int32_t rows_width = -1;  // max_blocks_per_seq of the recorded rows
 
   int32_t take_front() {
     int32_t page = ring[head];
@@ -113,6 +134,7 @@ pa_status pa_block_alloc_append_token(pa_block_alloc* a, int64_t seq, int64_t* s
   if (offset == 0) {
     if (a->count == 0) return fail(PA_ERR_OOM, "append_token: no free page for the next block");
     s.pages.push_back(a->take_front());
+    s.log((int32_t)logical);
   } else if (a->refs[s.pages[logical]] > 1) {
     if (!cow_src || !cow_dst)
       return fail(PA_ERR_INVALID, "append_token: page %d is shared but cow_src/cow_dst are NULL",
@@ -122,6 +144,7 @@ pa_status pa_block_alloc_append_token(pa_block_alloc* a, int64_t seq, int64_t* s
     dst = a->take_front();
     a->release(src);
     s.pages[logical] = dst;
+    s.log((int32_t)logical);
   }
   s.tokens = pos + 1;
   if (slot_out) *slot_out = (int64_t)s.pages[logical] * a->block_size + offset;
@@ -150,6 +173,8 @@ pa_status pa_block_alloc_fork(pa_block_alloc* a, int64_t parent, int64_t child) 
   if (it == a->seqs.end()) return fail(PA_ERR_NOT_FOUND, "fork: unknown parent %lld", (long long)parent);
   if (a->seqs.count(child)) return fail(PA_ERR_INVALID, "fork: sequence %lld exists", (long long)child);
   pa_block_alloc::Seq copy = it->second;  // copy before inserting (rehash may move `it`)
+  copy.changed.clear();
+  copy.whole = true;  // a new sequence: its whole table is exported
   for (int32_t p : copy.pages) ++a->refs[p];
   a->seqs.emplace(child, std::move(copy));
   return PA_OK;
@@ -339,6 +364,86 @@ pa_status pa_block_alloc_prefix_plan(const pa_block_alloc* a, const int64_t* seq
   *num_members = nm;
   *max_shared_partitions = max_sp;
   *min_shared_partitions = min_sp;
+  return PA_OK;
+}
+
+// Incremental export.  A row is exported whole (pad included) when its
+// contents are not known to belong to the sequence's logged state: a row never
+// exported, a row last exported for another sequence, a sequence last exported
+// at another row, a sequence new since (allocated or forked), or one whose log
+// overflowed.  Otherwise only its logged entries go out, each once, with the
+// page the table holds now.  Logs are cleared and rows recorded only once the
+// whole batch fits in the caller's buffer.
+pa_status pa_block_alloc_table_updates(pa_block_alloc* a, const int64_t* seqs, int32_t n,
+                                       int32_t max_blocks_per_seq, int32_t pad, int32_t* updates, int32_t cap,
+                                       int32_t* n_out, int32_t* context_lens_out) {
+  if (n_out) *n_out = 0;
+  if (!a || n < 0 || max_blocks_per_seq < 0 || cap < 0 || !n_out || (n > 0 && !seqs) || (cap > 0 && !updates))
+    return fail(PA_ERR_INVALID, "table_updates: bad argument");
+  const bool same_width = a->rows_width == max_blocks_per_seq;
+  std::vector<pa_block_alloc::Seq*> batch(n);
+  std::vector<char> whole(n);
+  int64_t count = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = a->seqs.find(seqs[i]);
+    if (it == a->seqs.end())
+      return fail(PA_ERR_NOT_FOUND, "table_updates: unknown sequence %lld", (long long)seqs[i]);
+    pa_block_alloc::Seq& sq = it->second;
+    if ((int64_t)sq.pages.size() > max_blocks_per_seq)
+      return fail(PA_ERR_INVALID, "table_updates: sequence %lld holds %zu pages > %d", (long long)seqs[i],
+                  sq.pages.size(), max_blocks_per_seq);
+    batch[i] = &sq;
+    const bool known = same_width && i < (int32_t)a->row_owner.size();
+    const int64_t owner = known ? a->row_owner[i] : pa_block_alloc::kNoOwner;
+    whole[i] = sq.whole || sq.row != i || owner != seqs[i];
+    if (whole[i]) {
+      const int64_t held = owner == pa_block_alloc::kNoOwner ? max_blocks_per_seq : a->row_len[i];
+      count += std::max<int64_t>((int64_t)sq.pages.size(), held);
+    } else {
+      std::sort(sq.changed.begin(), sq.changed.end());
+      sq.changed.erase(std::unique(sq.changed.begin(), sq.changed.end()), sq.changed.end());
+      count += (int64_t)sq.changed.size();
+    }
+  }
+  *n_out = count > INT32_MAX ? INT32_MAX : (int32_t)count;
+  if (count > cap)
+    return fail(PA_ERR_INVALID, "table_updates: %lld updates, capacity %d", (long long)count, cap);
+  if (!same_width) {
+    a->row_owner.clear();
+    a->row_len.clear();
+    a->rows_width = max_blocks_per_seq;
+  }
+  if ((int32_t)a->row_owner.size() < n) {
+    a->row_owner.resize(n, pa_block_alloc::kNoOwner);
+    a->row_len.resize(n, 0);
+  }
+  int32_t* u = updates;
+  auto put = [&](int32_t row, int32_t col, int32_t page) {
+    u[0] = row;
+    u[1] = col;
+    u[2] = page;
+    u += 3;
+  };
+  for (int32_t i = 0; i < n; ++i) {
+    const pa_block_alloc::Seq& sq = *batch[i];
+    const int32_t len = (int32_t)sq.pages.size();
+    if (whole[i]) {
+      const int32_t held =
+          a->row_owner[i] == pa_block_alloc::kNoOwner ? max_blocks_per_seq : a->row_len[i];
+      for (int32_t j = 0; j < len; ++j) put(i, j, sq.pages[j]);
+      for (int32_t j = len; j < held; ++j) put(i, j, pad);
+    } else {
+      for (int32_t j : sq.changed) put(i, j, sq.pages[j]);
+    }
+    a->row_owner[i] = seqs[i];
+    a->row_len[i] = len;
+    if (context_lens_out) context_lens_out[i] = (int32_t)sq.tokens;
+  }
+  for (int32_t i = 0; i < n; ++i) {
+    batch[i]->changed.clear();
+    batch[i]->whole = false;
+    batch[i]->row = i;  // a sequence at several rows: the last one
+  }
   return PA_OK;
 }
 

@@ -124,7 +124,8 @@ class TraceRunner:
         self.out = torch.empty_like(self.q)
         need = pa.pa_decode_workspace_size(w.num_seqs, w.num_q_heads, w.head_dim,
                                            w.max_blocks_per_seq * w.block_size)
-        self.workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
+        # NaN bytes to start with: a partial that no kernel wrote reaches the output as NaN.
+        self.workspace = torch.full((max(need, 256),), 0xFF, dtype=torch.uint8, device=self.device)
         if self.shared_prefix:
             host = self.alloc.prefix_plan(list(range(w.num_seqs)), w.group_size)
             self.plan = pa.prefix_plan_to_device(host, self.device)

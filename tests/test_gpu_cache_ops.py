@@ -168,3 +168,75 @@ def test_copy_blocks_many_pairs():
     ref[mapping[:, 1]] = kc[mapping[:, 0]]
     np.testing.assert_array_equal(bits_of(kd), ref)
     np.testing.assert_array_equal(bits_of(vd), ref)
+
+
+# -- block-table updates --------------------------------------------------------------------------
+
+def test_block_tables_apply_writes_each_update():
+    """Distinct random (row, column, page) triples, more than one CTA of them, against numpy."""
+    import torch
+    rng = _rng(11)
+    rows, mb = 300, 70
+    tables = rng.integers(-5, 10_000, size=(rows, mb)).astype(np.int32)
+    flat = rng.choice(rows * mb, size=5_000, replace=False)
+    upd = np.stack([flat // mb, flat % mb, rng.integers(0, 10_000, size=len(flat))], axis=1).astype(np.int32)
+    dt = torch.from_numpy(tables.copy()).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_block_tables_apply(dt, torch.from_numpy(upd).cuda(), dev_status=status)
+    tables[upd[:, 0], upd[:, 1]] = upd[:, 2]
+    np.testing.assert_array_equal(dt.cpu().numpy(), tables)
+    assert status.item() == 0
+    pa.pa_block_tables_apply(dt, torch.from_numpy(upd).cuda(), num_updates=0)   # nothing to do
+    np.testing.assert_array_equal(dt.cpu().numpy(), tables)
+
+
+def test_block_tables_apply_bad_update_is_skipped_and_flagged():
+    import torch
+    tables = np.zeros((4, 5), np.int32)
+    upd = np.array([[0, 0, 7], [4, 0, 9], [1, 5, 9], [-2, 2, 9], [3, 4, 8], [2, -3, 9]], np.int32)
+    dt = torch.from_numpy(tables.copy()).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_block_tables_apply(dt, torch.from_numpy(upd).cuda(), dev_status=status)
+    tables[0, 0], tables[3, 4] = 7, 8
+    np.testing.assert_array_equal(dt.cpu().numpy(), tables)
+    assert status.item() == pa.PA_DEV_BAD_UPDATE
+
+
+def test_block_tables_apply_skips_padding_rows():
+    """Row -1 is padding: skipped without a flag, whatever the column and page."""
+    import torch
+    tables = np.arange(12, dtype=np.int32).reshape(3, 4)
+    upd = np.array([[-1, 0, 50], [1, 2, 60], [-1, 99, 70], [-1, -1, -1]], np.int32)
+    dt = torch.from_numpy(tables.copy()).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_block_tables_apply(dt, torch.from_numpy(upd).cuda(), dev_status=status)
+    tables[1, 2] = 60
+    np.testing.assert_array_equal(dt.cpu().numpy(), tables)
+    assert status.item() == 0
+
+
+def test_device_tables_follow_decode_steps():
+    """The allocator's updates, applied on the device step after step (new blocks, a fork with
+    copy-on-write, a freed and replaced sequence), keep the device copy equal to the full export."""
+    import torch
+    bs, mb = 16, 32
+    alloc = pa.BlockAllocator(2_000, bs, _rng(3).permutation(2_000))
+    for s, n in enumerate([5, 16, 200, 31, 47]):
+        alloc.allocate_sequence(s, n)
+    batch = list(range(5))
+    dev = torch.full((len(batch), mb), 12345, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for step in range(60):
+        if step == 20:
+            alloc.fork(2, 9)
+            batch[4] = 9            # row 4 now holds the fork
+        if step == 40:
+            alloc.free_sequence(1)
+            alloc.allocate_sequence(1, 3)
+        for s in batch:
+            alloc.append_token(s)
+        upd, lens = alloc.table_updates(batch, mb)
+        pa.pa_block_tables_apply(dev, torch.from_numpy(upd.copy()).cuda(), dev_status=status)
+        full, _ = alloc.block_tables(batch, mb)
+        np.testing.assert_array_equal(dev.cpu().numpy(), full)
+    assert status.item() == 0

@@ -69,6 +69,10 @@ def _run_gpu(case, kernel="auto", tables=None, ctx=None, workspace=None, status=
     dt = case["dtype"]
     t = case["tables"] if tables is None else tables
     c = case["ctx"] if ctx is None else ctx
+    if workspace is None:  # NaN bytes: a partial that no kernel wrote cannot pass for a stale one
+        q = case["q"]
+        need = pa.pa_decode_workspace_size(q.shape[0], q.shape[1], q.shape[2], t.shape[1] * case["kc"].shape[2])
+        workspace = torch.full((max(need, 256),), 0xFF, dtype=torch.uint8, device="cuda")
     out = pa.pa_decode(_dev(case["q"], dt), _dev(case["kc"], dt), _dev(case["vc"], dt),
                        torch.from_numpy(t).cuda(), torch.from_numpy(np.asarray(c, np.int32)).cuda(), case["scale"],
                        workspace=workspace, dev_status=status)

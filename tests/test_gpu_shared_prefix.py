@@ -81,8 +81,12 @@ def test_shared_shapes(hq, hkv, d, bs, dtype, joint):
     plan = pa.prefix_plan_to_device(a.prefix_plan(list(range(nseq)), hq // hkv))
     assert plan["num_chunks"] >= 1
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    # NaN bytes in the workspace: a partial that no kernel wrote cannot pass for a stale one
+    ws = torch.full((max(pa.pa_decode_workspace_size(nseq, hq, d, mb * bs), 256),), 0xFF, dtype=torch.uint8,
+                    device="cuda")
     out = pa.pa_decode_shared_prefix(dev(q), dev(kc), dev(vc), torch.from_numpy(tables).cuda(),
-                                     torch.from_numpy(lens).cuda(), 1 / math.sqrt(d), plan, dev_status=status)
+                                     torch.from_numpy(lens).cuda(), 1 / math.sqrt(d), plan, workspace=ws,
+                                     dev_status=status)
     torch.cuda.synchronize()
     assert status.item() == 0
     ref = attention.decode_attention(q, kc, vc, tables, lens, 1 / math.sqrt(d), dtype)
