@@ -2051,7 +2051,8 @@ __device__ __forceinline__ bool seg_walk_next(SegWalk& w, Seg& s, const DecodeAr
 
 template <typename T, int D, int STAGES>
 __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
-    decode_shared_seg_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k, int tma_k,
+    decode_shared_seg_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
+                             const __grid_constant__ CUtensorMap tmap_v, int tma_k,
                              const int32_t* __restrict__ chunks, int num_chunks,
                              const int32_t* __restrict__ members, int num_members,
                              const int32_t* __restrict__ first_partition, int num_seqs, int fold_tails,
@@ -2156,7 +2157,10 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
     tc05::mbar_init(mma_drain, 1);
     *abort_flag = 0;
     tc05::fence_mbar_init();
-    if (tma_k) tc05::prefetch_tensormap(&tmap_k);
+    if (tma_k) {
+      tc05::prefetch_tensormap(&tmap_k);
+      tc05::prefetch_tensormap(&tmap_v);
+    }
   }
   if (warp == 0) {
     tc05::alloc(taddr_slot, S::kTmemCols);
@@ -2246,12 +2250,17 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
         if (lane == 0 && tok < seg.ctx && !page_ok) flag_status(a.status, PA_DEV_BAD_PAGE);
         const int64_t slab = ((int64_t)(page_ok ? page : 0) * a.num_kv_heads + seg.kvh) * bs + tok % bs;
         const uint32_t stage = base + S::kStageOff + st * S::kStageBytes;
-        // V (and K without the tensor map): 16-byte cp.async copies, zero past the
-        // context and on an out-of-range page; their completion joins the stage's
-        // phase before this warp's arrival below.
+        // V by the tensor map too when the whole group lies in the context (or the
+        // page is out of range: the box then starts past the tensor and loads zeros);
+        // a group the context ends inside needs zeros in its later rows, since a
+        // weight of 0 times a stale slot's NaN would still reach O.
+        const bool tma_v = tma_k && (!page_ok || tok + 16 <= seg.ctx);
+        // The rest (V of such a group, and K and V without the tensor maps): 16-byte
+        // cp.async copies, zero past the context and on an out-of-range page; their
+        // completion joins the stage's phase before this warp's arrival below.
 #pragma unroll
         for (int kv = 0; kv < 2; ++kv) {
-          if (kv == 0 && tma_k) continue;
+          if (kv == 0 ? tma_k : tma_v) continue;
           const T* cache = kv ? vcache : kcache;
 #pragma unroll
           for (int i2 = 0; i2 < S::kCopiesPerGroup; ++i2) {
@@ -2272,11 +2281,17 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
             // K by the tensor-memory-access unit: one 16-row box per 64-column block
             // (an out-of-range page loads as zeros; rows past the context are masked
             // by the softmax).  The arrival announces the bytes before the copies start.
-            tc05::mbar_arrive_expect_tx(kv_full(st), S::kBlocks * 16 * 128);
+            tc05::mbar_arrive_expect_tx(kv_full(st), (tma_v ? 2 : 1) * S::kBlocks * 16 * 128);
             const int32_t y = page_ok ? (int32_t)slab : (int32_t)((int64_t)a.num_blocks * a.num_kv_heads * bs);
 #pragma unroll
             for (int blk = 0; blk < S::kBlocks; ++blk)
               tc05::tma_load_2d(stage + blk * S::kKVBlockBytes + 16 * pw * 128, &tmap_k, kv_full(st), 64 * blk, y);
+            if (tma_v) {
+#pragma unroll
+              for (int blk = 0; blk < S::kBlocks; ++blk)
+                tc05::tma_load_2d(stage + S::kTileBytes + blk * S::kKVBlockBytes + 16 * pw * 128, &tmap_v,
+                                  kv_full(st), 64 * blk, y);
+            }
           } else {
             tc05::mbar_arrive(kv_full(st));
           }
@@ -3887,16 +3902,20 @@ cudaError_t launch_shared_seg(const DecodeArgs& a, pa_dtype dtype, int num_chunk
   auto kernel = decode_shared_seg_kernel<T, D, kStages>;
   cudaError_t err = ensure_smem(kernel, S::kSmemBytes, done);
   if (err != cudaSuccess) return err;
-  // K goes through the tensor-memory-access unit when the cache fits a tensor map
-  // (V, and K otherwise, through cp.async).
-  CUtensorMap mk;
+  // K and V go through the tensor-memory-access unit when the caches fit tensor
+  // maps (cp.async otherwise, and for V groups the context ends inside).
+  CUtensorMap mk, mv;
   std::memset(&mk, 0, sizeof(mk));
+  std::memset(&mv, 0, sizeof(mv));
   const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * a.block_size;
-  const int tma_k = rows < (1ll << 31) && encode_cache_map(&mk, a.key_cache, dtype, rows, D) ? 1 : 0;
+  const int tma_k = rows < (1ll << 31) && encode_cache_map(&mk, a.key_cache, dtype, rows, D) &&
+                            encode_cache_map(&mv, a.value_cache, dtype, rows, D)
+                        ? 1
+                        : 0;
   // Always a programmatic dependent: after a per-sequence kernel (`dependent`) it
   // reads inputs that kernel does not write and only waits for it at the end; after
   // any other kernel it waits before its first read.
-  return launch_pdl(kernel, dim3(sm_count()), dim3(S::kThreads), S::kSmemBytes, stream, true, a, mk, tma_k,
+  return launch_pdl(kernel, dim3(sm_count()), dim3(S::kThreads), S::kSmemBytes, stream, true, a, mk, mv, tma_k,
                     chunks, num_chunks, members, num_members, first_partition, num_seqs, fold_tails ? 1 : 0,
                     dependent ? 0 : 1, (int)g_fault.load());
 }
