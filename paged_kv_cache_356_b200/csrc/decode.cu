@@ -3020,11 +3020,11 @@ __global__ void __launch_bounds__(Tc05dShape<D, STAGES>::kThreads, 2)
 // w + WPI, ... with its own running maximum (the lanes compute 32 weights per
 // round; partial rows are loaded in prefetched groups), then the item's warps
 // merge through shared memory the same way.  A partition whose l is 0 adds
-// nothing.  With SPARSE (the balanced shared-prefix kernel marks slots empty,
-// l = 0, without writing their rows) a row's contribution is selected rather
-// than multiplied by its weight, so that whatever an unwritten row holds never
-// reaches the sum; rows are requested before the weights are known either
-// way.  Launched as a programmatic dependent of the kernel that writes the
+// nothing.  Dense form: rows are requested before the weights are known (one
+// round trip less).  SPARSE form (the balanced shared-prefix kernel marks slots
+// empty, l = 0, without writing their rows, and most slots are such marks):
+// the weights first, then only the rows of the slots with a contribution, so
+// an unwritten row is never read.  Launched as a programmatic dependent of the kernel that writes the
 // partials, it waits for that grid before reading them.
 // ---------------------------------------------------------------------------
 template <typename T, int D, int WPI, bool SPARSE>
@@ -3085,7 +3085,7 @@ __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel
     l_first = a.l_part[base + pf];
   }
   float x[UNROLL][VPL];
-  load_rows(x, sub, 0, merge ? min(32, (np - sub + WPI - 1) / WPI) : 0);
+  if constexpr (!SPARSE) load_rows(x, sub, 0, merge ? min(32, (np - sub + WPI - 1) / WPI) : 0);
   float mx = m_first;
   if (merge)
     for (int p = pf + WPI * 32; p < np; p += WPI * 32) mx = fmaxf(mx, a.m_part[base + p]);
@@ -3106,6 +3106,47 @@ __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel
         wt = lcur > 0.f ? lcur * expf(mp - mx) : 0.f;
       }
       lsum += wt;
+      if constexpr (SPARSE) {
+        // Only the slots with a contribution are read, UNROLL rows at a time.
+        uint32_t present = __ballot_sync(kFull, wt > 0.f);
+        while (present) {
+          int idx[UNROLL];
+#pragma unroll
+          for (int u = 0; u < UNROLL; ++u) {
+            idx[u] = present ? __ffs(present) - 1 : -1;
+            present &= present - 1;
+          }
+          float xs[UNROLL][VPL];
+#pragma unroll
+          for (int u = 0; u < UNROLL; ++u) {
+            if (idx[u] >= 0) {
+              const float* src = a.o_part + (base + p0 + WPI * idx[u]) * D + lane * VPL;
+              if constexpr (VPL % 4 == 0) {
+#pragma unroll
+                for (int v = 0; v < VPL / 4; ++v) {
+                  const float4 f = reinterpret_cast<const float4*>(src)[v];
+                  xs[u][4 * v] = f.x;
+                  xs[u][4 * v + 1] = f.y;
+                  xs[u][4 * v + 2] = f.z;
+                  xs[u][4 * v + 3] = f.w;
+                }
+              } else {
+#pragma unroll
+                for (int i = 0; i < VPL; ++i) xs[u][i] = src[i];
+              }
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < UNROLL; ++u) {
+            const float wk = __shfl_sync(kFull, wt, idx[u] < 0 ? 0 : idx[u]);
+            if (idx[u] >= 0) {
+#pragma unroll
+              for (int i = 0; i < VPL; ++i) acc[i] = fmaf(wk, xs[u][i], acc[i]);
+            }
+          }
+        }
+        continue;
+      }
       const int cnt = min(32, (np - p0 + WPI - 1) / WPI);
       if (c > 0) load_rows(x, p0, 0, cnt);
       for (int k = 0; k < cnt; k += UNROLL) {
@@ -3116,10 +3157,7 @@ __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel
         for (int u = 0; u < UNROLL; ++u) {
           const float wk = __shfl_sync(kFull, wt, min(k + u, 31));
 #pragma unroll
-          for (int i = 0; i < VPL; ++i) {
-            if constexpr (SPARSE) acc[i] = (k + u < cnt && wk > 0.f) ? fmaf(wk, x[u][i], acc[i]) : acc[i];
-            else acc[i] = fmaf(k + u < cnt ? wk : 0.f, x[u][i], acc[i]);
-          }
+          for (int i = 0; i < VPL; ++i) acc[i] = fmaf(k + u < cnt ? wk : 0.f, x[u][i], acc[i]);
         }
         if (more) {
 #pragma unroll
