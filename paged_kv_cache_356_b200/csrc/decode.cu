@@ -1765,32 +1765,38 @@ struct SegShape {
   __host__ __device__ static constexpr int producer_of(int w) { return w < kMmaWarp ? w - 4 : w - 5; }
 };
 
-// Chunk c of a shared-prefix plan; an entry that would index outside an array
+// Chunk c of a plan, its lane length in 64-token steps: a shared-prefix plan
+// gives whole partitions (8 steps each), a verify plan (vt = T > 0) the steps
+// that cover the leader's context.  An entry that would index outside an array
 // is reported (when `report`) and read as an empty chunk.
 struct SegChunk {
-  int leader, moff, mcount, sp;
+  int leader, moff, mcount, ns;
 };
 __device__ __forceinline__ SegChunk seg_chunk(const DecodeArgs& a, const int32_t* __restrict__ chunks, int c,
-                                             int num_members, int num_seqs, bool report) {
+                                             int num_members, int num_seqs, bool report, int vt) {
   SegChunk k{__ldg(chunks + 4 * c), __ldg(chunks + 4 * c + 1), __ldg(chunks + 4 * c + 2), __ldg(chunks + 4 * c + 3)};
+  const int64_t steps = vt > 0 ? (int64_t)k.ns : 8 * (int64_t)k.ns;
   const bool ok = (unsigned)k.leader < (unsigned)num_seqs && k.moff >= 0 && k.mcount >= 0 &&
-                  (int64_t)k.moff + k.mcount <= num_members && (int64_t)k.mcount * a.group <= 128 && k.sp >= 0 &&
-                  (int64_t)k.sp * kPartition <= (int64_t)a.max_blocks_per_seq * a.block_size &&
-                  k.sp <= a.max_partitions;
+                  (int64_t)k.moff + k.mcount <= num_members && (int64_t)k.mcount * a.group <= 128 && steps >= 0 &&
+                  64 * (steps - 1) < (int64_t)a.max_blocks_per_seq * a.block_size &&
+                  (steps + 7) / 8 <= a.max_partitions;
   if (!ok) {
     if (report) flag_status(a.status, PA_DEV_BAD_PLAN);
     k.mcount = 0;
   }
-  if (k.mcount == 0) k.sp = 0;
+  k.ns = k.mcount == 0 ? 0 : (int)steps;
   return k;
 }
 
 // A segment: steps [s0, s1) of one lane.  kind 0 = shared (rows: the chunk's
 // members), 1 = tail (rows: member `b`); `leader` is the sequence whose block
-// table gives the pages; tokens at or past `ctx` are masked.  Its partial goes
-// to workspace slot `slot`; slots [slot + 1, mark_end) are marked empty.
+// table gives the pages; tokens at or past `ctx` are read as nothing.  Row r
+// (member mi = r / G) sees the tokens before ctx - max(0, causal - mi): a verify
+// chunk's tokens first .. first + count - 1 of T sit at the context's last T
+// positions, so causal = T - 1 - first; 0 elsewhere.  Its partial goes to
+// workspace slot `slot`; slots [slot + 1, mark_end) are marked empty.
 struct Seg {
-  int kind, kvh, leader, moff, mcount, b, s0, s1, ctx, slot, mark_end;
+  int kind, kvh, leader, moff, mcount, b, s0, s1, ctx, slot, mark_end, causal;
 };
 
 // The segments of one CTA, in order.  Every lane of a producer warp runs the
@@ -1816,6 +1822,7 @@ struct SegWalk {
   uint32_t tmask;      // members of the loaded batch still to hand out
   bool tloaded, tdone;
   int tT, tfp, tctx;      // per lane: tail steps, first tail partition and context of sequence tm0 + lane
+  int vt;                 // verify plans: query tokens per sequence (0: a shared-prefix plan)
 };
 
 // Tail of batch sequence b: its steps from the end of its shared partitions
@@ -1847,9 +1854,9 @@ __device__ __forceinline__ int warp_incl_sum(int v) {
 
 // Units of shared lane (kv head, c): kSegLeadIn units that carry no step (the
 // cost of starting a segment: the previous one's epilogue and the switch of
-// query rows), then one unit per 64-token step of the chunk's shared partitions.
+// query rows), then one unit per 64-token step of the lane.
 constexpr int kSegLeadIn = 3;
-__device__ __forceinline__ int seg_lane_units(int sp) { return sp > 0 ? 8 * sp + kSegLeadIn : 0; }
+__device__ __forceinline__ int seg_lane_units(int ns) { return ns > 0 ? ns + kSegLeadIn : 0; }
 
 // Chunk c of the plan from the lane registers of the walk (plans of at most 32
 // chunks: lane c holds chunk c) or from global memory.
@@ -1858,30 +1865,30 @@ __device__ __forceinline__ SegChunk seg_chunk_of(const SegWalk& w, int c, const 
                                                  int num_members, int num_seqs) {
   if (num_chunks <= 32) {
     return SegChunk{__shfl_sync(kFull, w.cl.leader, c), __shfl_sync(kFull, w.cl.moff, c),
-                    __shfl_sync(kFull, w.cl.mcount, c), __shfl_sync(kFull, w.cl.sp, c)};
+                    __shfl_sync(kFull, w.cl.mcount, c), __shfl_sync(kFull, w.cl.ns, c)};
   }
-  return seg_chunk(a, chunks, c, num_members, num_seqs, false);
+  return seg_chunk(a, chunks, c, num_members, num_seqs, false, w.vt);
 }
 
-// Lane (kv head, chunk), unit offset within the lane and the chunk's shared
-// partitions of shared unit u (warp-collective; u < H_kv * s_sh).
+// Lane (kv head, chunk), unit offset within the lane and the lane's steps of
+// shared unit u (warp-collective; u < H_kv * s_sh).
 __device__ __forceinline__ void seg_locate(const SegWalk& w, int u, const DecodeArgs& a,
                                            const int32_t* __restrict__ chunks, int num_chunks, int num_members,
-                                           int num_seqs, int& kvh, int& c, int& off, int& sp) {
+                                           int num_seqs, int& kvh, int& c, int& off, int& ns) {
   const int lane = threadIdx.x & 31;
   kvh = u / w.s_sh;
   int r = u - kvh * w.s_sh;
   c = 0;
   off = 0;
-  sp = 0;
+  ns = 0;
   for (int c0 = 0; c0 < num_chunks; c0 += 32) {
     int n, incl;
     if (num_chunks <= 32) {
-      n = seg_lane_units(w.cl.sp);
+      n = seg_lane_units(w.cl.ns);
       incl = w.cl_incl;
     } else {
       const int cc = c0 + lane;
-      n = cc < num_chunks ? seg_lane_units(seg_chunk(a, chunks, cc, num_members, num_seqs, false).sp) : 0;
+      n = cc < num_chunks ? seg_lane_units(seg_chunk(a, chunks, cc, num_members, num_seqs, false, w.vt).ns) : 0;
       incl = warp_incl_sum(n);
     }
     const uint32_t hit = __ballot_sync(kFull, incl > r);
@@ -1890,7 +1897,7 @@ __device__ __forceinline__ void seg_locate(const SegWalk& w, int u, const Decode
       const int nl = __shfl_sync(kFull, n, l);
       c = c0 + l;
       off = r - (__shfl_sync(kFull, incl, l) - nl);
-      sp = (nl - kSegLeadIn) / 8;
+      ns = nl - kSegLeadIn;
       return;
     }
     r -= __shfl_sync(kFull, incl, 31);
@@ -1898,17 +1905,17 @@ __device__ __forceinline__ void seg_locate(const SegWalk& w, int u, const Decode
 }
 
 // Start of CTA k's range: total * k / ctas, except that a range never ends
-// inside the steps of a lane of one partition (such a cut moves to the nearer
-// end of them).
+// inside the steps of a lane of one partition, at most 8 steps (such a cut moves
+// to the nearer end of them): such a lane has one slot.
 __device__ __forceinline__ int seg_cut(const SegWalk& w, int k, const DecodeArgs& a,
                                        const int32_t* __restrict__ chunks, int num_chunks, int num_members,
                                        int num_seqs) {
   int u = (int)((unsigned)w.total * (unsigned)k / (unsigned)w.ctas);
   if (u < w.base && w.s_sh > 0) {
-    int kvh, c, off, sp;
-    seg_locate(w, u, a, chunks, num_chunks, num_members, num_seqs, kvh, c, off, sp);
+    int kvh, c, off, ns;
+    seg_locate(w, u, a, chunks, num_chunks, num_members, num_seqs, kvh, c, off, ns);
     const int step = off - kSegLeadIn;
-    if (sp == 1 && step > 0) u += step < 4 ? -step : 8 - step;
+    if (ns <= 8 && step > 0) u += 2 * step < ns ? -step : ns - step;
   }
   return u;
 }
@@ -1917,8 +1924,9 @@ template <int E>
 __device__ __forceinline__ void seg_walk_init(SegWalk& w, const DecodeArgs& a, const int32_t* __restrict__ chunks,
                                               int num_chunks, const int32_t* __restrict__ members, int num_members,
                                               const int32_t* __restrict__ first_partition, int num_seqs,
-                                              bool fold_tails, bool report) {
+                                              bool fold_tails, int vt, bool report) {
   const int lane = threadIdx.x & 31;
+  w.vt = vt;
   // Shared units per kv head and the tail weight per kv head.  The chunk, member
   // and sequence loads of one pass are independent (one round trip); plans of up
   // to 32 chunks keep their chunks in lane registers.
@@ -1928,8 +1936,9 @@ __device__ __forceinline__ void seg_walk_init(SegWalk& w, const DecodeArgs& a, c
   w.cl_incl = 0;
   for (int i0 = 0; i0 < num_chunks || i0 < num_seqs; i0 += 32) {
     const int i = i0 + lane;
-    const SegChunk ci = i < num_chunks ? seg_chunk(a, chunks, i, num_members, num_seqs, report) : SegChunk{0, 0, 0, 0};
-    const int n = seg_lane_units(ci.sp);
+    const SegChunk ci =
+        i < num_chunks ? seg_chunk(a, chunks, i, num_members, num_seqs, report, vt) : SegChunk{0, 0, 0, 0};
+    const int n = seg_lane_units(ci.ns);
     int T = 0, fp, ctx;
     if (fold_tails) seg_tail_of(a, first_partition, i, num_seqs, T, fp, ctx);
     const int incl = warp_incl_sum(n);
@@ -1961,8 +1970,8 @@ __device__ __forceinline__ void seg_walk_init(SegWalk& w, const DecodeArgs& a, c
   if (w.u0 < w.base && s_sh > 0) {
     w.su = w.u0;
     w.su_end = w.u1 < w.base ? w.u1 : w.base;
-    int sp;
-    seg_locate(w, w.u0, a, chunks, num_chunks, num_members, num_seqs, w.skvh, w.sc, w.soff, sp);
+    int ns;
+    seg_locate(w, w.u0, a, chunks, num_chunks, num_members, num_seqs, w.skvh, w.sc, w.soff, ns);
     w.sci = seg_chunk_of(w, w.sc, a, chunks, num_chunks, num_members, num_seqs);
   }
   // Tail cursor: the first kv head whose tail lanes can start in [u0, u1).
@@ -1982,8 +1991,8 @@ __device__ __forceinline__ bool seg_walk_next(SegWalk& w, Seg& s, const DecodeAr
                                               const int32_t* __restrict__ first_partition, int num_seqs) {
   const int lane = threadIdx.x & 31;
   while (w.su < w.su_end) {
-    const int units = seg_lane_units(w.sci.sp);
-    const int len = 8 * w.sci.sp;
+    const int units = seg_lane_units(w.sci.ns);
+    const int len = w.sci.ns;
     const int lane0 = w.su - w.soff;
     const int off1 = units - w.soff < w.su_end - w.su ? units : w.soff + (w.su_end - w.su);
     const int s0 = max(0, w.soff - kSegLeadIn), s1 = max(0, off1 - kSegLeadIn);
@@ -1998,7 +2007,7 @@ __device__ __forceinline__ bool seg_walk_next(SegWalk& w, Seg& s, const DecodeAr
           ++w.skvh;
         }
         w.sci = seg_chunk_of(w, w.sc, a, chunks, num_chunks, num_members, num_seqs);
-      } while (w.sci.sp == 0 && w.skvh < a.num_kv_heads);
+      } while (w.sci.ns == 0 && w.skvh < a.num_kv_heads);
       w.soff = 0;
     }
     if (s1 <= s0) continue;  // the range held only lead-in units of this lane
@@ -2010,8 +2019,11 @@ __device__ __forceinline__ bool seg_walk_next(SegWalk& w, Seg& s, const DecodeAr
       const int first = lane0 + kSegLeadIn;
       slot = (int)blockIdx.x - (int)(((unsigned)w.ctas * (unsigned)(first + 1) - 1u) / (unsigned)w.total);
     }
-    const int mark_end = s1 == len ? ci.sp : slot + 1;
-    s = Seg{0, kvh, ci.leader, ci.moff, ci.mcount, -1, s0, s1, INT_MAX, slot, mark_end};
+    const int mark_end = s1 == len ? (ci.ns + 7) / 8 : slot + 1;
+    // A verify lane reads its leader's whole context, each row up to its own token.
+    const int ctx = w.vt > 0 ? context_of(a, ci.leader, false) : INT_MAX;
+    const int causal = w.vt > 0 ? w.vt - 1 - (ci.moff - ci.leader * w.vt) : 0;
+    s = Seg{0, kvh, ci.leader, ci.moff, ci.mcount, -1, s0, s1, ctx, slot, mark_end, causal};
     return true;
   }
   while (true) {
@@ -2020,7 +2032,7 @@ __device__ __forceinline__ bool seg_walk_next(SegWalk& w, Seg& s, const DecodeAr
       w.tmask &= w.tmask - 1;
       const int T = __shfl_sync(kFull, w.tT, l), b = w.tm0 + l;
       const int fp = __shfl_sync(kFull, w.tfp, l), ctx = __shfl_sync(kFull, w.tctx, l);
-      s = Seg{1, w.tkvh, b, 0, 1, b, 8 * fp, 8 * fp + T, ctx, fp, (ctx + kPartition - 1) / kPartition};
+      s = Seg{1, w.tkvh, b, 0, 1, b, 8 * fp, 8 * fp + T, ctx, fp, (ctx + kPartition - 1) / kPartition, 0};
       return true;
     }
     if (w.tdone) return false;
@@ -2056,7 +2068,7 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
                              const int32_t* __restrict__ chunks, int num_chunks,
                              const int32_t* __restrict__ members, int num_members,
                              const int32_t* __restrict__ first_partition, int num_seqs, int fold_tails,
-                             int wait_at_start, int fault) {
+                             int verify_tokens, int wait_at_start, int fault) {
   using S = SegShape<D, STAGES>;
   constexpr int E = S::kEpilogueSteps;
   extern __shared__ uint8_t smem_raw[];
@@ -2130,7 +2142,7 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
     // Every global write of this grid follows a producer's load, hence this wait.
     if (wait_at_start) asm volatile("griddepcontrol.wait;\n" ::: "memory");
     seg_walk_init<E>(walk, a, chunks, num_chunks, members, num_members, first_partition, num_seqs, fold_tails != 0,
-                     pw == 0 && lane == 0 && blockIdx.x == 0);
+                     verify_tokens, pw == 0 && lane == 0 && blockIdx.x == 0);
     have = next_seg(seg);
     if (have) {
       win_cur = window(seg, seg.s0);
@@ -2214,6 +2226,7 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
           desc[qb * 16 + 6] = s.slot;
           desc[qb * 16 + 7] = s.mark_end;
           desc[qb * 16 + 8] = s.leader;
+          desc[qb * 16 + 13] = s.causal;
           desc[qb * 16 + 0] = 1;
         }
       }
@@ -2386,6 +2399,8 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
       const int s0 = desc[qb * 16 + 2], s1 = desc[qb * 16 + 3];
       const int nrows = desc[qb * 16 + 4], ctx = desc[qb * 16 + 5];
       const int slot = desc[qb * 16 + 6], mark_end = desc[qb * 16 + 7], leader = desc[qb * 16 + 8];
+      // This thread's row sees the tokens before ctx_row (its own causal limit).
+      const int ctx_row = ctx - max(0, desc[qb * 16 + 13] - (32 * warp + lane) / a.group);
       const bool busy = 32 * warp < nrows;
       // Out-of-range pages: bit i of bad_w[k] is group k of step mw0 + i.  The
       // producers publish the first 32 steps; later windows of 32 steps are
@@ -2427,7 +2442,7 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
         const int sh = step - mw0;
         const int bad = (int)(((bad_w[0] >> sh) & 1u) | (((bad_w[1] >> sh) & 1u) << 1) |
                               (((bad_w[2] >> sh) & 1u) << 2) | (((bad_w[3] >> sh) & 1u) << 3));
-        const int lim = ctx - 64 * step;  // tokens of this step inside the context
+        const int lim = ctx_row - 64 * step;  // tokens of this step this row sees
         uint32_t pk[32];
         float alpha = 1.f;
         if (busy) {
@@ -3219,7 +3234,8 @@ struct VerifyArgs {
   int num_tokens;    // T
   int q_heads;       // H_q
   int row_groups;    // CTAs per kv head along grid y
-  int skip_visible;  // 1: the partitions every token sees in full come from the joint kernel
+  int skip_visible;  // 1: the partitions every token sees in full come from the joint kernel;
+                     // 2: every partition of sequences longer than one partition does
 };
 
 // Partitions [0, n) of a sequence that all T tokens see in full (none for a
@@ -3230,14 +3246,18 @@ __device__ __forceinline__ int verify_visible_partitions(int ctx, int num_tokens
 
 // Work plan of the joint kernel for a verify call, from the context lengths:
 // sequence b's T tokens are T members (ids b * T + t, query rows of T * H_q
-// per sequence) reading b's table, in chunks of at most `per_chunk` tokens,
-// over its visible partitions.  chunks[b * cps + k] = (b, b * T + k * per_chunk,
-// count, visible partitions); members[i] = i.
+// per sequence) reading b's table, in chunks of at most `per_chunk` tokens.
+// chunks[b * cps + k] = (b, b * T + k * per_chunk, count, extent); members[i] = i.
+// The extent is the partitions every token sees in full (`whole` = 0: the
+// per-partition kernels), or the 64-token steps of the whole context for a
+// sequence longer than one partition (`whole` = 1: the balanced kernel, which
+// applies each row's causal limit).
 __global__ void verify_plan_kernel(const DecodeArgs a, int num_seqs, int num_tokens, int per_chunk, int cps,
-                                   int32_t* __restrict__ chunks, int32_t* __restrict__ members) {
+                                   int whole, int32_t* __restrict__ chunks, int32_t* __restrict__ members) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= num_seqs) return;
-  const int sp = verify_visible_partitions(context_of(a, b, false), num_tokens);
+  const int ctx = context_of(a, b, false);
+  const int sp = whole ? (ctx > kPartition ? (ctx + 63) / 64 : 0) : verify_visible_partitions(ctx, num_tokens);
   for (int k = 0; k < cps; ++k) {
     const int first = k * per_chunk;
     int4 c;
@@ -3349,9 +3369,10 @@ __global__ void __launch_bounds__(NW * 32) decode_verify_tc_kernel(const DecodeA
 
   const int ctx = context_of(a, b, threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0);
   const int np = (ctx + kPartition - 1) / kPartition;
-  // With the joint kernel on the partitions every token sees, grid z counts the ones after them.
-  const int p = blockIdx.z + (v.skip_visible ? verify_visible_partitions(ctx, v.num_tokens) : 0);
-  if (p >= max(np, 1)) return;
+  // With the joint kernel on the partitions every token sees, grid z counts the ones after them;
+  // with the balanced kernel on every sequence longer than one partition, only the others are left.
+  const int p = blockIdx.z + (v.skip_visible == 1 ? verify_visible_partitions(ctx, v.num_tokens) : 0);
+  if (p >= max(np, 1) || (v.skip_visible == 2 && np > 1)) return;
   if (ctx == 0) {
     verify_zero_rows<T, D>(a, v, b, kvh, r0, nr);
     return;
@@ -3933,7 +3954,7 @@ cudaError_t launch_shared_tc05d(const DecodeArgs& a, const CUtensorMap& mk, cons
 template <typename T, int D>
 cudaError_t launch_shared_seg(const DecodeArgs& a, pa_dtype dtype, int num_chunks, const int32_t* chunks,
                               const int32_t* members, int num_members, const int32_t* first_partition, int num_seqs,
-                              bool dependent, cudaStream_t stream, bool fold_tails = true) {
+                              bool dependent, cudaStream_t stream, bool fold_tails = true, int verify_tokens = 0) {
   constexpr int kStages = D == 128 ? 5 : 8;
   using S = SegShape<D, kStages>;
   static std::atomic<uint64_t> done{0};
@@ -3955,7 +3976,7 @@ cudaError_t launch_shared_seg(const DecodeArgs& a, pa_dtype dtype, int num_chunk
   // any other kernel it waits before its first read.
   return launch_pdl(kernel, dim3(sm_count()), dim3(S::kThreads), S::kSmemBytes, stream, true, a, mk, mv, tma_k,
                     chunks, num_chunks, members, num_members, first_partition, num_seqs, fold_tails ? 1 : 0,
-                    dependent ? 0 : 1, (int)g_fault.load());
+                    verify_tokens, dependent ? 0 : 1, (int)g_fault.load());
 }
 
 std::atomic<int> g_shared_kernel{PA_SHARED_PREFIX_AUTO};
@@ -4073,7 +4094,7 @@ cudaError_t launch_verify_tc(const DecodeArgs& a, VerifyArgs v, int num_seqs, in
   // After the visible partitions a sequence has at most 1 + ceil((T - 1) / 512) left.
   const int tail = 1 + (v.num_tokens - 1 + kPartition - 1) / kPartition;
   const dim3 grid(num_seqs, a.num_kv_heads * v.row_groups,
-                  v.skip_visible ? std::min(partitions, tail) : partitions);
+                  v.skip_visible == 2 ? 1 : v.skip_visible ? std::min(partitions, tail) : partitions);
   if (!v.skip_visible) {
     kernel<<<grid, NW * 32, S::kSmemBytes, stream>>>(a, v);
     return cudaGetLastError();
@@ -4469,32 +4490,38 @@ extern "C" pa_status pa_decode_verify(const void* q, const void* key_cache, cons
     int32_t* members = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.members_off);
     const int cps = (num_query_tokens + per_chunk - 1) / per_chunk;
     const int num_members = num_seqs * num_query_tokens;
-    verify_plan_kernel<<<(num_seqs + 127) / 128, 128, 0, s>>>(a, num_seqs, num_query_tokens, per_chunk, cps, chunks,
-                                                                members);
+    // The balanced kernel takes every partition of the sequences longer than one
+    // partition, each row up to its own causal limit (its lanes counted in 64-token
+    // steps); the per-sequence kernel is left the one-partition sequences.  The
+    // per-partition kernels take the partitions every token sees in full.
+    const int shared_choice = g_shared_kernel.load();
+    const int64_t max_steps = std::min<int64_t>(((int64_t)max_blocks_per_seq * block_size + 63) / 64,
+                                                (int64_t)partitions * 8);
+    const int64_t units = (int64_t)num_kv_heads * num_seqs * cps * (max_steps + 3);
+    balanced = (shared_choice == PA_SHARED_PREFIX_AUTO || shared_choice == PA_SHARED_PREFIX_TCGEN05) &&
+               units < kSegMaxUnits;
+    verify_plan_kernel<<<(num_seqs + 127) / 128, 128, 0, s>>>(a, num_seqs, num_query_tokens, per_chunk, cps,
+                                                                balanced ? 1 : 0, chunks, members);
     err = cudaGetLastError();
     if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode_verify plan kernel: %s", cudaGetErrorString(err));
     // The joint kernel indexes q, the partials and its members with H_q heads per member.
     DecodeArgs aj = a;
     aj.num_q_heads = num_q_heads;
-    const int shared_choice = g_shared_kernel.load();
-    const int64_t units = (int64_t)num_kv_heads * num_seqs * cps * ((int64_t)max_visible * 8 + 3);
-    balanced = (shared_choice == PA_SHARED_PREFIX_AUTO || shared_choice == PA_SHARED_PREFIX_TCGEN05) &&
-               units < kSegMaxUnits;
     if (balanced) {
-      // The balanced kernel over the visible partitions only (the per-sequence kernel
-      // keeps the partitions the causal limits cut); it waits for the plan kernel first.
-      // Its members are token ids b * T + t, so they are checked against num_members.
+      // It waits for the plan kernel first.  Its members are token ids b * T + t,
+      // so they are checked against num_members.
       const int nc = num_seqs * cps;
+      const int T = num_query_tokens;
       err = head_dim == 64
                 ? (dtype == PA_BF16 ? launch_shared_seg<__nv_bfloat16, 64>(aj, dtype, nc, chunks, members, num_members,
-                                                                           nullptr, num_members, false, s, false)
+                                                                           nullptr, num_members, false, s, false, T)
                                     : launch_shared_seg<__half, 64>(aj, dtype, nc, chunks, members, num_members,
-                                                                    nullptr, num_members, false, s, false))
+                                                                    nullptr, num_members, false, s, false, T))
                 : (dtype == PA_BF16 ? launch_shared_seg<__nv_bfloat16, 128>(aj, dtype, nc, chunks, members,
                                                                             num_members, nullptr, num_members, false,
-                                                                            s, false)
+                                                                            s, false, T)
                                     : launch_shared_seg<__half, 128>(aj, dtype, nc, chunks, members, num_members,
-                                                                     nullptr, num_members, false, s, false));
+                                                                     nullptr, num_members, false, s, false, T));
     } else {
       const dim3 grid(num_seqs * cps, num_kv_heads, max_visible);
       err = dtype == PA_BF16 ? launch_shared_dim<__nv_bfloat16>(aj, head_dim, grid, chunks, members, num_members,
@@ -4503,7 +4530,7 @@ extern "C" pa_status pa_decode_verify(const void* q, const void* key_cache, cons
                                                          num_members, dtype, s);
     }
     if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode_verify joint kernel: %s", cudaGetErrorString(err));
-    v.skip_visible = 1;
+    v.skip_visible = balanced ? 2 : 1;
   }
   if (tc_ok && choice != PA_DECODE_CUDA_CORES)
     err = dtype == PA_BF16 ? launch_verify_tc_any<__nv_bfloat16>(a, v, head_dim, num_seqs, partitions, s)
