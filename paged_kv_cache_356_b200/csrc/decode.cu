@@ -4344,7 +4344,9 @@ extern "C" pa_status pa_decode(const void* q, const void* key_cache, const void*
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = launch_partitions(a, dtype, head_dim, num_seqs, partitions, s);
   if (st != PA_OK || partitions <= 1) return st;
-  return launch_reduce_any(a, dtype, head_dim, num_seqs, s);
+  // A programmatic dependent: its CTAs take the SMs the partition kernel's last
+  // wave leaves idle and wait there for that grid to finish.
+  return launch_reduce_any(a, dtype, head_dim, num_seqs, s, /*dependent=*/true);
 }
 
 extern "C" pa_status pa_decode_partitions(const void* q, const void* key_cache, const void* value_cache,
@@ -4391,7 +4393,7 @@ extern "C" pa_status pa_decode_reduce(const int32_t* context_lens, int32_t num_s
   a.o_part = reinterpret_cast<float*>(ws + w.o_off);
   a.m_part = reinterpret_cast<float*>(ws + w.m_off);
   a.l_part = reinterpret_cast<float*>(ws + w.l_off);
-  return launch_reduce_any(a, dtype, head_dim, num_seqs, static_cast<cudaStream_t>(stream));
+  return launch_reduce_any(a, dtype, head_dim, num_seqs, static_cast<cudaStream_t>(stream), /*dependent=*/true);
 }
 
 // ---------------------------------------------------------------------------
