@@ -241,18 +241,21 @@ PA_API pa_status pa_decode_reduce(const int32_t* context_lens, int32_t num_seqs,
  * and the error returns, is as for pa_decode; in addition
  * num_query_tokens >= 1 and num_query_tokens * num_q_heads <= 2^24.
  * bf16 / f16 caches with block_size a multiple of 16 run on tensor cores:
- * when T * G > 16 (head_dim 64 or 128), the partitions that all T tokens see
- * in full go to the shared-prefix joint kernel (the T tokens of a sequence
- * are members of one group: each page is read once for all T * G rows; the
- * plan is built on the device from context_lens, inside the workspace), and
- * the rest -- each sequence's last partition or two, where the causal limits
- * fall -- to a per-sequence kernel with 8 to 32 (token, query head) rows of
- * one kv head per CTA; f32 or other block sizes use CUDA cores.
+ * when T * G > 16 (head_dim 64 or 128) the joint path runs (the T tokens of
+ * a sequence are members of one group: each page is read once for all T * G
+ * rows; the plan is built on the device from context_lens, inside the
+ * workspace).  With the default shared-prefix kernel, the balanced tcgen05
+ * kernel covers the whole context of every sequence longer than one
+ * partition, each row masked at its own causal limit, and a per-sequence
+ * kernel the one-partition sequences; with the per-partition kernels, those
+ * take the partitions all T tokens see in full and the per-sequence kernel
+ * (8 to 32 (token, query head) rows of one kv head per CTA) the rest, where
+ * the causal limits fall.  f32 or other block sizes use CUDA cores.
  * pa_set_decode_kernel, pa_set_shared_prefix_kernel and pa_set_verify_path
  * apply.
  * ---------------------------------------------------------------------- */
 typedef enum {
-  PA_VERIFY_AUTO = 0,          /* joint kernel for the visible partitions when T * G > 16 */
+  PA_VERIFY_AUTO = 0,          /* joint path when T * G > 16 */
   PA_VERIFY_PER_SEQUENCE = 1,  /* per-sequence partition kernels only */
   PA_VERIFY_JOINT = 2          /* joint kernel whenever the call allows it; PA_ERR_UNSUPPORTED otherwise */
 } pa_verify_path;
@@ -354,20 +357,29 @@ PA_API pa_status pa_decode_shared_prefix(const void* q, const void* key_cache, c
                                          int32_t* dev_status, void* stream);
 
 /* Which joint kernel pa_decode_shared_prefix runs (process-wide; default
- * AUTO = TCGEN05).  TCGEN05 is the balanced persistent kernel on the 5th-
- * generation tensor cores (one CTA per SM, cp.async loads into swizzled
- * shared memory, tcgen05.mma with Tensor Memory accumulators): it covers the
- * groups' shared partitions and also every member's own tokens, split evenly
- * over the SMs in runs of 64-token steps, so a per-sequence kernel runs only
- * for sequences outside every group; a run writes one partial per query row
- * into the slot of the partition where it starts and marks the slots of the
- * later partitions it covers empty (l = 0).  The other kernels compute the
- * partials of each shared partition and leave the members' other partitions
- * to the per-sequence kernel: TCGEN05_ITEMS the persistent per-partition
- * tcgen05 kernel (TMA loads); TCGEN05_2CTA the same pipeline in a leaner form
- * that runs two CTAs per SM; TCGEN05_SERIAL the one-partition-per-CTA tcgen05
- * kernel without the software pipeline; MMA_SYNC the mma.sync kernel.  All
- * give the same output; the switch exists for testing and measurement. */
+ * AUTO).  TCGEN05 is the balanced persistent kernel on the 5th-generation
+ * tensor cores (one CTA per SM; K and V pages by the tensor-memory-access
+ * unit, with zero-filling cp.async where a context ends inside a 16-token
+ * group; tcgen05.mma with Tensor Memory accumulators): it covers the groups'
+ * shared partitions and also every member's own tokens, split evenly over the
+ * SMs in runs of 64-token steps, so a per-sequence kernel runs only for
+ * sequences outside every group.  Each run writes one partial per query row
+ * into a slot of its lane (slots counted from the lane's first run) and marks
+ * the lane's slots that no run takes empty (l = 0); the merge reads only the
+ * slots with a contribution.  AUTO takes that form when the members' own
+ * tokens are a small share of the shared work (beams over a long prompt);
+ * otherwise it runs the balanced kernel on the shared partitions only and the
+ * per-sequence kernel on every partition from each sequence's first_partition
+ * (many sequences with long tails over a common prompt).  The other kernels
+ * compute the partials of each shared partition and leave the members' other
+ * partitions to the per-sequence kernel: TCGEN05_ITEMS the persistent
+ * per-partition tcgen05 kernel; TCGEN05_2CTA the same pipeline in a leaner
+ * form that runs two CTAs per SM; TCGEN05_SERIAL the one-partition-per-CTA
+ * tcgen05 kernel without the software pipeline; MMA_SYNC the mma.sync kernel.
+ * All give the same output up to rounding; the switch exists for testing and
+ * measurement.  pa_decode_verify's joint path follows the same switch: AUTO
+ * and TCGEN05 run the balanced kernel over each sequence's whole context with
+ * per-row causal limits, the others the per-partition kernels. */
 typedef enum pa_shared_prefix_kernel {
   PA_SHARED_PREFIX_AUTO = 0,
   PA_SHARED_PREFIX_TCGEN05 = 1,

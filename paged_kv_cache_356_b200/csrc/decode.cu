@@ -1794,9 +1794,11 @@ __device__ __forceinline__ SegChunk seg_chunk(const DecodeArgs& a, const int32_t
 // (member mi = r / G) sees the tokens before ctx - max(0, causal - mi): a verify
 // chunk's tokens first .. first + count - 1 of T sit at the context's last T
 // positions, so causal = T - 1 - first; 0 elsewhere.  Its partial goes to
-// workspace slot `slot`; slots [slot + 1, mark_end) are marked empty.
+// workspace slot `slot`; slots [slot + 1, mark_end) are marked empty.  A verify
+// segment that covers its whole lane (`final`) writes its rows' outputs instead
+// and marks slot 0 done (l = -1), so that the merge leaves those rows alone.
 struct Seg {
-  int kind, kvh, leader, moff, mcount, b, s0, s1, ctx, slot, mark_end, causal;
+  int kind, kvh, leader, moff, mcount, b, s0, s1, ctx, slot, mark_end, causal, final;
 };
 
 // The segments of one CTA, in order.  Every lane of a producer warp runs the
@@ -2023,7 +2025,8 @@ __device__ __forceinline__ bool seg_walk_next(SegWalk& w, Seg& s, const DecodeAr
     // A verify lane reads its leader's whole context, each row up to its own token.
     const int ctx = w.vt > 0 ? context_of(a, ci.leader, false) : INT_MAX;
     const int causal = w.vt > 0 ? w.vt - 1 - (ci.moff - ci.leader * w.vt) : 0;
-    s = Seg{0, kvh, ci.leader, ci.moff, ci.mcount, -1, s0, s1, ctx, slot, mark_end, causal};
+    const int final = w.vt > 0 && s0 == 0 && s1 == len;
+    s = Seg{0, kvh, ci.leader, ci.moff, ci.mcount, -1, s0, s1, ctx, slot, mark_end, causal, final};
     return true;
   }
   while (true) {
@@ -2032,7 +2035,7 @@ __device__ __forceinline__ bool seg_walk_next(SegWalk& w, Seg& s, const DecodeAr
       w.tmask &= w.tmask - 1;
       const int T = __shfl_sync(kFull, w.tT, l), b = w.tm0 + l;
       const int fp = __shfl_sync(kFull, w.tfp, l), ctx = __shfl_sync(kFull, w.tctx, l);
-      s = Seg{1, w.tkvh, b, 0, 1, b, 8 * fp, 8 * fp + T, ctx, fp, (ctx + kPartition - 1) / kPartition, 0};
+      s = Seg{1, w.tkvh, b, 0, 1, b, 8 * fp, 8 * fp + T, ctx, fp, (ctx + kPartition - 1) / kPartition, 0, 0};
       return true;
     }
     if (w.tdone) return false;
@@ -2061,7 +2064,8 @@ __device__ __forceinline__ bool seg_walk_next(SegWalk& w, Seg& s, const DecodeAr
   }
 }
 
-template <typename T, int D, int STAGES>
+// ROWS_OUT: verify launches, whose segments may write their rows' outputs (see Seg).
+template <typename T, int D, int STAGES, bool ROWS_OUT>
 __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
     decode_shared_seg_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
                              const __grid_constant__ CUtensorMap tmap_v, int tma_k,
@@ -2227,6 +2231,7 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
           desc[qb * 16 + 7] = s.mark_end;
           desc[qb * 16 + 8] = s.leader;
           desc[qb * 16 + 13] = s.causal;
+          desc[qb * 16 + 14] = s.final;
           desc[qb * 16 + 0] = 1;
         }
       }
@@ -2529,6 +2534,8 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
       if (busy) {
         const int32_t rbase = prow_s[qb * S::kRows + tid];  // workspace row base of this thread's query row
         const int32_t prow = rbase < 0 ? -1 : rbase + slot;
+        const bool final = ROWS_OUT && desc[qb * 16 + 14] != 0;  // the outputs themselves (see Seg)
+        const int32_t orow = rbase < 0 ? -1 : rbase / a.max_partitions;
         const float inv = l > 0.f ? 1.f / l : 0.f;
         const uint32_t ocol = S::kOCol + 128u * (uint32_t)qb;
         constexpr int kTileStride = 20;  // floats
@@ -2549,15 +2556,25 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
           int32_t pr[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            pr[i] = __shfl_sync(kFull, prow, 8 * i + rsub);
+            pr[i] = __shfl_sync(kFull, final ? orow : prow, 8 * i + rsub);
             v[i] = *reinterpret_cast<const float4*>(tile + (8 * i + rsub) * kTileStride + 4 * csub);
           }
           __syncwarp();
+          if (ROWS_OUT && final) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            if (pr[i] >= 0) *reinterpret_cast<float4*>(a.o_part + (int64_t)pr[i] * D + 16 * cb + 4 * csub) = v[i];
+            for (int i = 0; i < 4; ++i)
+              if (pr[i] >= 0)
+                *reinterpret_cast<uint2*>(reinterpret_cast<T*>(a.out) + (int64_t)pr[i] * D + 16 * cb + 4 * csub) =
+                    make_uint2(pack2<T>(v[i].x, v[i].y), pack2<T>(v[i].z, v[i].w));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              if (pr[i] >= 0) *reinterpret_cast<float4*>(a.o_part + (int64_t)pr[i] * D + 16 * cb + 4 * csub) = v[i];
+          }
         }
-        if (prow >= 0) {
+        if (ROWS_OUT && final) {
+          if (prow >= 0) a.l_part[prow] = -1.f;  // slot 0: this row is done
+        } else if (prow >= 0) {
           a.m_part[prow] = m_use == -INFINITY ? -INFINITY : m_use * kLn2;
           a.l_part[prow] = l;
           for (int p = slot + 1; p < mark_end; ++p) {  // the lane's slots no segment takes: empty
@@ -3042,7 +3059,7 @@ __global__ void __launch_bounds__(Tc05dShape<D, STAGES>::kThreads, 2)
 // an unwritten row is never read.  Launched as a programmatic dependent of the kernel that writes the
 // partials, it waits for that grid before reading them.
 // ---------------------------------------------------------------------------
-template <typename T, int D, int WPI, bool SPARSE>
+template <typename T, int D, int WPI, int SPARSE>
 __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel(const DecodeArgs a, int num_seqs) {
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
   constexpr int VPL = D / 32;
@@ -3063,7 +3080,7 @@ __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel
     np = (context_of(a, b, false) + kPartition - 1) / kPartition;
     base = item * a.max_partitions;
   }
-  const bool merge = live && np > 1;
+  bool merge = live && np > 1;
 
   // This warp's partitions are p = sub + WPI * (lane + 32 c), c = 0, 1, ...
   // Lane `lane` holds m and l of its first one; the first UNROLL partial rows
@@ -3098,6 +3115,11 @@ __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel
   if (merge && pf < np) {
     m_first = a.m_part[base + pf];
     l_first = a.l_part[base + pf];
+  }
+  if constexpr (SPARSE == 2) {
+    // Slot 0 marked done (l = -1): the balanced kernel wrote this row's output
+    // (read in the same round trip as the weights).
+    if (merge && a.l_part[base] < 0.f) merge = false;
   }
   float x[UNROLL][VPL];
   if constexpr (!SPARSE) load_rows(x, sub, 0, merge ? min(32, (np - sub + WPI - 1) / WPI) : 0);
@@ -3353,6 +3375,8 @@ struct VerifyShape {
 template <typename T, int D, int NW, int STAGES, int NT>
 __global__ void __launch_bounds__(NW * 32) decode_verify_tc_kernel(const DecodeArgs a, const VerifyArgs v) {
   const AfterPrerequisiteGrid after{threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0};
+  // The merge, launched after this kernel as a programmatic dependent, may start now (it waits for this grid).
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   using S = VerifyShape<D, NW, STAGES, NT>;
   constexpr int KSTEPS = D / 16;
   constexpr int MTILES = D / 16;
@@ -3957,9 +3981,10 @@ cudaError_t launch_shared_seg(const DecodeArgs& a, pa_dtype dtype, int num_chunk
                               bool dependent, cudaStream_t stream, bool fold_tails = true, int verify_tokens = 0) {
   constexpr int kStages = D == 128 ? 5 : 8;
   using S = SegShape<D, kStages>;
-  static std::atomic<uint64_t> done{0};
-  auto kernel = decode_shared_seg_kernel<T, D, kStages>;
-  cudaError_t err = ensure_smem(kernel, S::kSmemBytes, done);
+  static std::atomic<uint64_t> done[2] = {{0}, {0}};
+  auto kernel = verify_tokens > 0 ? decode_shared_seg_kernel<T, D, kStages, true>
+                                  : decode_shared_seg_kernel<T, D, kStages, false>;
+  cudaError_t err = ensure_smem(kernel, S::kSmemBytes, done[verify_tokens > 0 ? 1 : 0]);
   if (err != cudaSuccess) return err;
   // K and V go through the tensor-memory-access unit when the caches fit tensor
   // maps (cp.async otherwise, and for V groups the context ends inside).
@@ -4052,7 +4077,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-template <typename T, int D, bool SPARSE>
+template <typename T, int D, int SPARSE>
 cudaError_t launch_reduce_dim(const DecodeArgs& a, int num_seqs, cudaStream_t stream, bool dependent) {
   const int64_t items = (int64_t)num_seqs * a.num_q_heads;
   auto grid = [&](int ipc) { return dim3((unsigned)((items + ipc - 1) / ipc)); };
@@ -4067,15 +4092,19 @@ cudaError_t launch_reduce_dim(const DecodeArgs& a, int num_seqs, cudaStream_t st
 
 template <typename T>
 cudaError_t launch_reduce(const DecodeArgs& a, int head_dim, int num_seqs, cudaStream_t stream,
-                          bool dependent = false, bool sparse = false) {
+                          bool dependent = false, int sparse = 0) {
   if ((int64_t)num_seqs * a.num_q_heads > 0x7fffffffLL) return cudaErrorInvalidValue;
+  // sparse: 0 every slot written; 1 empty slots marked l = 0; 2 also rows marked done
+  auto pick = [&](auto d) -> cudaError_t {
+    constexpr int Dv = decltype(d)::value;
+    if (sparse == 2) return launch_reduce_dim<T, Dv, 2>(a, num_seqs, stream, dependent);
+    if (sparse == 1) return launch_reduce_dim<T, Dv, 1>(a, num_seqs, stream, dependent);
+    return launch_reduce_dim<T, Dv, 0>(a, num_seqs, stream, dependent);
+  };
   switch (head_dim) {
-    case 64: return sparse ? launch_reduce_dim<T, 64, true>(a, num_seqs, stream, dependent)
-                           : launch_reduce_dim<T, 64, false>(a, num_seqs, stream, dependent);
-    case 128: return sparse ? launch_reduce_dim<T, 128, true>(a, num_seqs, stream, dependent)
-                            : launch_reduce_dim<T, 128, false>(a, num_seqs, stream, dependent);
-    case 256: return sparse ? launch_reduce_dim<T, 256, true>(a, num_seqs, stream, dependent)
-                            : launch_reduce_dim<T, 256, false>(a, num_seqs, stream, dependent);
+    case 64: return pick(std::integral_constant<int, 64>{});
+    case 128: return pick(std::integral_constant<int, 128>{});
+    case 256: return pick(std::integral_constant<int, 256>{});
   }
   return cudaErrorInvalidValue;
 }
@@ -4318,7 +4347,7 @@ pa_status launch_partitions(const DecodeArgs& a, pa_dtype dtype, int head_dim, i
 }
 
 pa_status launch_reduce_any(const DecodeArgs& a, pa_dtype dtype, int head_dim, int num_seqs, cudaStream_t s,
-                            bool dependent = false, bool sparse = false) {
+                            bool dependent = false, int sparse = 0) {
   const cudaError_t err =
       dtype == PA_F32    ? launch_reduce<float>(a, head_dim, num_seqs, s, dependent, sparse)
       : dtype == PA_BF16 ? launch_reduce<__nv_bfloat16>(a, head_dim, num_seqs, s, dependent, sparse)
@@ -4543,7 +4572,7 @@ extern "C" pa_status pa_decode_verify(const void* q, const void* key_cache, cons
                              : launch_verify_cc<__half>(a, v, head_dim, num_seqs, partitions, s);
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode_verify partition kernel: %s", cudaGetErrorString(err));
   if (partitions <= 1) return PA_OK;
-  return launch_reduce_any(a, dtype, head_dim, num_seqs, s, /*dependent=*/false, /*sparse=*/balanced);
+  return launch_reduce_any(a, dtype, head_dim, num_seqs, s, /*dependent=*/true, /*sparse=*/balanced ? 2 : 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -4723,7 +4752,32 @@ extern "C" pa_status pa_decode_shared_prefix(const void* q, const void* key_cach
                              : launch_shared_seg<__half, 128>(a, dtype, num_chunks, chunks, members, num_members,
                                                               first_partition, num_seqs, others, s);
     if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode shared-prefix kernel: %s", cudaGetErrorString(err));
-    return launch_reduce_any(a, dtype, head_dim, num_seqs, s, /*dependent=*/true, /*sparse=*/true);
+    return launch_reduce_any(a, dtype, head_dim, num_seqs, s, /*dependent=*/true, /*sparse=*/1);
+  }
+  if (joint && unit_bound < kSegMaxUnits && choice == PA_SHARED_PREFIX_AUTO) {
+    // Tail-heavy plans: the balanced kernel on the shared lanes only, then the
+    // per-sequence kernel on every partition from each sequence's first_partition
+    // (a programmatic dependent: its CTAs take the SMs the joint grid's CTAs
+    // leave), then the sparse merge.
+    if (!aligned16(chunks)) return fail(PA_ERR_INVALID, "decode_shared_prefix: chunks must be 16-byte aligned");
+    cudaError_t err;
+    if (head_dim == 64)
+      err = dtype == PA_BF16 ? launch_shared_seg<__nv_bfloat16, 64>(a, dtype, num_chunks, chunks, members, num_members,
+                                                                     first_partition, num_seqs, false, s, false)
+                             : launch_shared_seg<__half, 64>(a, dtype, num_chunks, chunks, members, num_members,
+                                                             first_partition, num_seqs, false, s, false);
+    else
+      err = dtype == PA_BF16 ? launch_shared_seg<__nv_bfloat16, 128>(a, dtype, num_chunks, chunks, members, num_members,
+                                                                      first_partition, num_seqs, false, s, false)
+                             : launch_shared_seg<__half, 128>(a, dtype, num_chunks, chunks, members, num_members,
+                                                              first_partition, num_seqs, false, s, false);
+    if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode shared-prefix kernel: %s", cudaGetErrorString(err));
+    DecodeArgs ap = a;
+    ap.first_partition = first_partition;
+    ap.partition_base = min_shared_partitions < partitions - 1 ? min_shared_partitions : partitions - 1;
+    st = launch_partitions(ap, dtype, head_dim, num_seqs, partitions, s, /*dependent=*/true);
+    if (st != PA_OK) return st;
+    return launch_reduce_any(a, dtype, head_dim, num_seqs, s, /*dependent=*/true, /*sparse=*/1);
   }
   if (joint) {
     if (!aligned16(chunks)) return fail(PA_ERR_INVALID, "decode_shared_prefix: chunks must be 16-byte aligned");

@@ -11,7 +11,10 @@ from tests.parity import assert_decode_close, bits_of, host_bits
 
 pytestmark = pytest.mark.gpu
 
-JOINT = {"tcgen05": pa.PA_SHARED_PREFIX_TCGEN05, "tcgen05_items": pa.PA_SHARED_PREFIX_TCGEN05_ITEMS,
+# auto: the balanced kernel with the members' tails folded in (few, short tails), or on the shared
+# lanes only with the per-sequence kernel on the tails (many or long tails)
+JOINT = {"auto": pa.PA_SHARED_PREFIX_AUTO,
+         "tcgen05": pa.PA_SHARED_PREFIX_TCGEN05, "tcgen05_items": pa.PA_SHARED_PREFIX_TCGEN05_ITEMS,
          "tcgen05_2cta": pa.PA_SHARED_PREFIX_TCGEN05_2CTA, "tcgen05_serial": pa.PA_SHARED_PREFIX_TCGEN05_SERIAL,
          "mma_sync": pa.PA_SHARED_PREFIX_MMA_SYNC}
 
