@@ -79,7 +79,7 @@ def parse_args(argv=None):
     ap.add_argument("--verify-rows", type=int, default=0, choices=[0, 8, 16, 32],
                     help="with --verify-tokens: rows per CTA of the per-sequence verify kernel (0: default)")
     ap.add_argument("--verify-path", choices=["auto", "per_sequence", "joint"], default="auto",
-                    help="with --verify-tokens: joint kernel for the partitions all tokens see (auto: when T*G > 16)")
+                    help="with --verify-tokens: joint kernel for the partitions all tokens see (auto: when T*G > 8)")
     return ap.parse_args(argv)
 
 
@@ -536,7 +536,7 @@ class StepBench:
             self.ws = torch.empty(need, dtype=torch.uint8, device="cuda") if need > 0 else None
             self.part_bytes = verify_call_bytes(w, ctx_np, self.unique, T)
             self.verify_joint = (args.verify_path == "joint" or
-                                 (args.verify_path == "auto" and T * w.group_size > 16 and args.kernel != "cc" and
+                                 (args.verify_path == "auto" and T * w.group_size > 8 and args.kernel != "cc" and
                                   w.dtype in ("bf16", "f16") and w.head_dim in (64, 128) and
                                   w.block_size % 16 == 0 and max_ctx > 512))
 

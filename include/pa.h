@@ -241,7 +241,7 @@ PA_API pa_status pa_decode_reduce(const int32_t* context_lens, int32_t num_seqs,
  * and the error returns, is as for pa_decode; in addition
  * num_query_tokens >= 1 and num_query_tokens * num_q_heads <= 2^24.
  * bf16 / f16 caches with block_size a multiple of 16 run on tensor cores:
- * when T * G > 16 (head_dim 64 or 128) the joint path runs (the T tokens of
+ * when T * G > 8 (head_dim 64 or 128) the joint path runs (the T tokens of
  * a sequence are members of one group: each page is read once for all T * G
  * rows; the plan is built on the device from context_lens, inside the
  * workspace).  With the default shared-prefix kernel, the balanced tcgen05
@@ -255,7 +255,7 @@ PA_API pa_status pa_decode_reduce(const int32_t* context_lens, int32_t num_seqs,
  * apply.
  * ---------------------------------------------------------------------- */
 typedef enum {
-  PA_VERIFY_AUTO = 0,          /* joint path when T * G > 16 */
+  PA_VERIFY_AUTO = 0,          /* joint path when T * G > 8 */
   PA_VERIFY_PER_SEQUENCE = 1,  /* per-sequence partition kernels only */
   PA_VERIFY_JOINT = 2          /* joint kernel whenever the call allows it; PA_ERR_UNSUPPORTED otherwise */
 } pa_verify_path;

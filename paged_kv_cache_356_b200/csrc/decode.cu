@@ -4431,9 +4431,9 @@ extern "C" pa_status pa_decode_reduce(const int32_t* context_lens, int32_t num_s
 namespace {
 std::atomic<int> g_verify_path{PA_VERIFY_AUTO};
 
-// Above this many rows (T * G) per kv head the joint kernel takes the visible partitions (at 16
-// rows the per-sequence kernel alone is still faster).
-constexpr int kVerifyJointRows = 16;
+// Above this many rows (T * G) per kv head AUTO takes the joint path (at 8 rows, one token of a
+// group of 8, the per-sequence kernel alone is faster).
+constexpr int kVerifyJointRows = 8;
 
 // The partials (the pa_decode layout with T * H_q heads), then the joint kernel's plan:
 // chunks int32 [num_seqs * T][4] at most, members int32 [num_seqs * T].
