@@ -111,17 +111,16 @@ def partition_kernel_bytes(w, ctx, unique_kv):
     return unique_kv + q + tables + lens + partials + rows
 
 
-def verify_call_bytes(w, ctx, unique_kv, num_tokens):
-    """Algorithmic bytes of one pa_decode_verify call (partition kernel + merge): KV + q + tables +
-    lengths, the partials written and read back, and every output row written once."""
+def call_bytes(w, ctx, unique_kv, num_tokens=1):
+    """Algorithmic bytes of one whole attention call (pa_decode_verify, pa_decode_shared_prefix):
+    the unique KV, q, the tables' used entries and the lengths read once, and every output row
+    written once.  Partials are the kernels' own traffic, not the call's."""
     eb = w.elem_bytes
-    nparts = [-(-int(c) // 512) for c in ctx]
     rows = w.num_seqs * num_tokens * w.num_q_heads
     q = rows * w.head_dim * eb
     tables = 4 * sum(-(-int(c) // w.block_size) for c in ctx)
     lens = 4 * w.num_seqs
-    partials = sum(n for n in nparts if n > 1) * num_tokens * w.num_q_heads * (w.head_dim + 2) * 4
-    return unique_kv + q + tables + lens + 2 * partials + rows * w.head_dim * eb
+    return unique_kv + q + tables + lens + rows * w.head_dim * eb
 
 
 def describe(w):
@@ -516,7 +515,8 @@ class StepBench:
         tables_np = run.block_tables.cpu().numpy()
         self.ctx_np = ctx_np = run.context_lens.cpu().numpy()
         self.unique, self.logical = kv_bytes(w, tables_np, ctx_np)
-        self.part_bytes = partition_kernel_bytes(w, ctx_np, self.unique)
+        self.part_bytes = (partition_kernel_bytes(w, ctx_np, self.unique) if run.plan is None else
+                           call_bytes(w, ctx_np, self.unique))
         self.max_ctx = max_ctx = w.max_blocks_per_seq * w.block_size
         self.kd, self.vd, self.sd = run.step_write
         self.q, self.out, self.ws = run.q, run.out, run.workspace
@@ -534,7 +534,7 @@ class StepBench:
             self.out = torch.empty_like(self.q)
             need = pa.pa_decode_verify_workspace_size(w.num_seqs, T, w.num_q_heads, w.head_dim, max_ctx)
             self.ws = torch.empty(need, dtype=torch.uint8, device="cuda") if need > 0 else None
-            self.part_bytes = verify_call_bytes(w, ctx_np, self.unique, T)
+            self.part_bytes = call_bytes(w, ctx_np, self.unique, T)
             self.verify_joint = (args.verify_path == "joint" or
                                  (args.verify_path == "auto" and T * w.group_size > 8 and args.kernel != "cc" and
                                   w.dtype in ("bf16", "f16") and w.head_dim in (64, 128) and
@@ -830,14 +830,15 @@ def run_ours(args):
                                    {"chunks": run.plan["num_chunks"], "members": run.plan["num_members"],
                                     "shared_partitions": run.plan["max_shared_partitions"]}),
             "roofline": {"bound": "hbm",
-                         "kernel": (("pa_decode_verify call: plan kernel + joint tcgen05 kernel (partitions all "
-                                     "tokens see) + decode_verify_tc_kernel (the rest) + merge, timed together"
+                         "kernel": (("pa_decode_verify call: plan kernel + balanced tcgen05 kernel over whole "
+                                     "contexts (per-row causal limits) + per-sequence kernel (one-partition "
+                                     "sequences) + merge, timed together"
                                      if sb.verify_joint else
                                      "pa_decode_verify call: decode_verify_tc_kernel + merge (timed together)")
                                     if T > 0 else
                                     "decode_tc_kernel (pa_decode_partitions)" if run.plan is None else
-                                    "pa_decode_shared_prefix call: joint tcgen05 kernel + per-sequence "
-                                    "decode_tc_kernel + merge (timed together)"),
+                                    "pa_decode_shared_prefix call: balanced tcgen05 kernel (+ per-sequence "
+                                    "kernel) + sparse merge, timed together"),
                          "achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} (copy bandwidth)",
                          "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic,
