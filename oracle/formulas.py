@@ -12,7 +12,7 @@ def blocks_needed(num_tokens: int, block_size: int) -> int:
 
     Glossary, "Step-by-Step Implementation Framework" (42 tokens take 3 pages
     of 16); Internals, "Implementation: Custom Block Manager Simulation in
-    Python" (allocate_sequence rounds the token count up to whole blocks).
+    Python" (a sequence is given its token count rounded up to whole blocks).
     """
     if num_tokens < 0 or block_size <= 0:
         raise ValueError("num_tokens must be >= 0 and block_size > 0")

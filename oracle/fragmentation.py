@@ -9,7 +9,7 @@ most that any holder has stored in it.  "Architectural Recommendations for
 Infrastructure Engineers", item 3: raise an alert when the free pages fall
 below 10 percent of the pool.
 
-``pool_stats`` reads an allocator state as ``PagedBlockManager.state()``
+``pool_stats`` reads an allocator state as ``PagePool.state()``
 returns it and states every quantity by its definition.
 """
 from __future__ import annotations

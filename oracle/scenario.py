@@ -10,7 +10,7 @@ from __future__ import annotations
 import numpy as np
 
 from . import attention, cache_ops
-from .allocator import PagedBlockManager
+from .allocator import PagePool
 
 
 def run(workload, with_data: bool = True, decode_seqs=None) -> dict:
@@ -22,7 +22,7 @@ def run(workload, with_data: bool = True, decode_seqs=None) -> dict:
     ``decode_seqs`` restricts the fp64 attention to those sequences.
     """
     w = workload
-    mgr = PagedBlockManager(w.num_blocks, w.block_size, w.initial_free_order())
+    mgr = PagePool(w.num_blocks, w.block_size, w.initial_free_order())
     store = np.uint16 if w.dtype in ("bf16", "f16") else np.float32
     kc = vc = None
     if with_data:
@@ -33,12 +33,12 @@ def run(workload, with_data: bool = True, decode_seqs=None) -> dict:
     for op in w.trace:
         kind = op[0]
         if kind == "allocate":
-            mgr.allocate_sequence(op[1], op[2])
+            mgr.admit(op[1], op[2])
         elif kind == "fork":
-            mgr.fork(op[1], op[2])
+            mgr.share(op[1], op[2])
         elif kind == "append":
             for _ in range(op[2]):
-                slot, pair = mgr.append_token(op[1])
+                slot, pair = mgr.extend(op[1])
                 append_slots.append(slot)
                 if pair is not None:
                     pending.append(pair)
@@ -57,9 +57,9 @@ def run(workload, with_data: bool = True, decode_seqs=None) -> dict:
         elif kind == "decode":
             tables = np.full((w.num_seqs, w.max_blocks_per_seq), -1, dtype=np.int32)
             for b in range(w.num_seqs):
-                t = mgr.block_tables[b]
+                t = mgr.tables[b]
                 tables[b, :len(t)] = t
-            ctx = np.array([mgr.num_tokens[b] for b in range(w.num_seqs)], dtype=np.int32)
+            ctx = np.array([mgr.lengths[b] for b in range(w.num_seqs)], dtype=np.int32)
             result["block_tables"] = tables
             result["context_lens"] = ctx
             if with_data:

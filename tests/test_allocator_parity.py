@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 
 from oracle import scenario
-from oracle.allocator import PagedBlockManager
+from oracle.allocator import PagePool
 from paged_kv_cache_356_b200 import binding as pa
 from paged_kv_cache_356_b200 import workloads
 
@@ -81,7 +81,7 @@ def test_random_streams_match_oracle(seed):
     bs = rnd.choice([1, 2, 3, 4, 16, 32])
     total = rnd.choice([8, 33, 64])
     order = rnd.sample(range(total), total)
-    ref = PagedBlockManager(total, bs, order)
+    ref = PagePool(total, bs, order)
     dut = pa.BlockAllocator(total, bs, order)
     live, next_id = [], 0
     for _ in range(500):
@@ -90,7 +90,7 @@ def test_random_streams_match_oracle(seed):
         if op < 0.2 or not live:
             n = rnd.randint(0, 3 * bs + 1)
             try:
-                ref.allocate_sequence(next_id, n)
+                ref.admit(next_id, n)
             except MemoryError as e:
                 ref_exc = e
             try:
@@ -102,14 +102,14 @@ def test_random_streams_match_oracle(seed):
             next_id += 1
         elif op < 0.35:
             parent = rnd.choice(live)
-            ref.fork(parent, next_id)
+            ref.share(parent, next_id)
             dut.fork(parent, next_id)
             live.append(next_id)
             next_id += 1
         elif op < 0.85:
             s = rnd.choice(live)
             try:
-                r = ref.append_token(s)
+                r = ref.extend(s)
             except MemoryError as e:
                 ref_exc = e
             try:
@@ -122,7 +122,7 @@ def test_random_streams_match_oracle(seed):
                 assert (d[1], d[2]) == (pair if pair is not None else (-1, -1))
         else:
             s = rnd.choice(live)
-            ref.free_sequence(s)
+            ref.drop(s)
             dut.free_sequence(s)
             live.remove(s)
         assert (ref_exc is None) == (dut_exc is None)
@@ -164,7 +164,7 @@ def _random_ops(seed, total=300):
     bs = rng.choice([1, 3, 16, 32])
     order = list(range(total))
     rng.shuffle(order)
-    ref = PagedBlockManager(total, bs, order)
+    ref = PagePool(total, bs, order)
     dut = pa.BlockAllocator(total, bs, np.array(order, dtype=np.int32))
     live, next_id = [], 0
     for _ in range(250):
@@ -172,24 +172,24 @@ def _random_ops(seed, total=300):
         try:
             if op == 0 or not live:
                 n = rng.randrange(0, 70)
-                ref.allocate_sequence(next_id, n)
+                ref.admit(next_id, n)
                 dut.allocate_sequence(next_id, n)
                 live.append(next_id)
                 next_id += 1
             elif op == 1:
                 parent = rng.choice(live)
-                ref.fork(parent, next_id)
+                ref.share(parent, next_id)
                 dut.fork(parent, next_id)
                 live.append(next_id)
                 next_id += 1
             elif op == 2:
                 s = rng.choice(live)
                 for _ in range(rng.randrange(1, 9)):
-                    ref.append_token(s)
+                    ref.extend(s)
                     dut.append_token(s)
             else:
                 s = rng.choice(live)
-                ref.free_sequence(s)
+                ref.drop(s)
                 dut.free_sequence(s)
                 live.remove(s)
         except MemoryError:
@@ -202,7 +202,7 @@ def test_pool_stats_match_the_oracle_after_every_op(seed):
     from oracle import fragmentation
     for ref, dut in _random_ops(seed):
         for alarm in (0.10, 0.5):
-            want = fragmentation.pool_stats(ref.state(), ref.total_pages, ref.block_size, alarm)
+            want = fragmentation.pool_stats(ref.state(), ref.num_pages, ref.block_size, alarm)
             assert dut.stats(alarm) == want
 
 
@@ -238,22 +238,22 @@ def test_batched_appends_equal_sequential_ones_in_the_oracle(seed):
     total = 500
     order = list(range(total))
     rng.shuffle(order)
-    ref = PagedBlockManager(total, bs, order)
+    ref = PagePool(total, bs, order)
     dut = pa.BlockAllocator(total, bs, np.array(order, dtype=np.int32))
     live = []
     for s in range(6):
         n = rng.randrange(0, 40)
-        ref.allocate_sequence(s, n)
+        ref.admit(s, n)
         dut.allocate_sequence(s, n)
         live.append(s)
     for child in range(6, 12):
         parent = rng.choice(live)
-        ref.fork(parent, child)
+        ref.share(parent, child)
         dut.fork(parent, child)
         live.append(child)
     for _ in range(30):
         batch = [rng.choice(live) for _ in range(rng.randrange(1, 12))]
-        want = [ref.append_token(s) for s in batch]
+        want = [ref.extend(s) for s in batch]
         slots, pairs = dut.append_tokens(batch)
         assert [int(x) for x in slots] == [w[0] for w in want]
         assert [tuple(int(v) for v in p) for p in pairs] == [w[1] if w[1] else (-1, -1) for w in want]
