@@ -31,12 +31,16 @@
 // then merges partitions: M = max m_p, w_p = l_p e^(m_p - M),
 // out = sum w_p o_p / sum w_p.
 //
-// pa_decode_shared_prefix computes the same partials, but a whole partition
-// that a group of sequences shares (the same physical pages: forked beams, a
-// common prompt) is read once for the whole group by a joint kernel serving up
-// to PA_PREFIX_QUERIES_PER_CTA queries -- a dense contraction, run on the
-// fifth-generation tensor cores (decode_shared_tc05p_kernel) -- while the
-// per-sequence kernel covers the remaining partitions and the merge follows.
+// pa_decode_shared_prefix computes the same result, but a whole partition that
+// a group of sequences shares (the same physical pages: forked beams, a common
+// prompt) is read once for the whole group by a joint kernel serving up to
+// PA_PREFIX_QUERIES_PER_CTA queries -- a dense contraction on the
+// fifth-generation tensor cores.  The default joint kernel is the balanced one
+// (decode_shared_seg_kernel): equal ranges of 64-token steps per SM over the
+// shared partitions, with the members' own tokens folded in or left to the
+// per-sequence kernel; a merge follows.  pa_decode_verify treats a sequence's T
+// draft tokens as such a group over its own context, each row masked at its
+// own causal limit.
 #include <math.h>
 
 #include <algorithm>
@@ -4110,7 +4114,8 @@ cudaError_t launch_reduce(const DecodeArgs& a, int head_dim, int num_seqs, cudaS
 }
 
 // `v.skip_visible`: launched as a programmatic dependent of the joint kernel,
-// which covers the partitions every token sees in full.
+// which covers the partitions every token sees in full (1) or every partition
+// of the sequences longer than one (2).
 template <typename T, int D, int NW, int STAGES, int NT>
 cudaError_t launch_verify_tc(const DecodeArgs& a, VerifyArgs v, int num_seqs, int partitions, cudaStream_t stream) {
   using S = VerifyShape<D, NW, STAGES, NT>;
@@ -4120,7 +4125,7 @@ cudaError_t launch_verify_tc(const DecodeArgs& a, VerifyArgs v, int num_seqs, in
   if (err != cudaSuccess) return err;
   v.row_groups = (v.num_tokens * a.group + S::kRows - 1) / S::kRows;
   if ((int64_t)a.num_kv_heads * v.row_groups > 65535) return cudaErrorInvalidValue;
-  // After the visible partitions a sequence has at most 1 + ceil((T - 1) / 512) left.
+  // After the partitions every token sees a sequence has at most 1 + ceil((T - 1) / 512) left.
   const int tail = 1 + (v.num_tokens - 1 + kPartition - 1) / kPartition;
   const dim3 grid(num_seqs, a.num_kv_heads * v.row_groups,
                   v.skip_visible == 2 ? 1 : v.skip_visible ? std::min(partitions, tail) : partitions);
