@@ -2076,7 +2076,7 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
                              const int32_t* __restrict__ chunks, int num_chunks,
                              const int32_t* __restrict__ members, int num_members,
                              const int32_t* __restrict__ first_partition, int num_seqs, int fold_tails,
-                             int verify_tokens, int wait_at_start, int fault) {
+                             int verify_tokens, int wait_at_start, int fault, int32_t* __restrict__ merge_list) {
   using S = SegShape<D, STAGES>;
   constexpr int E = S::kEpilogueSteps;
   extern __shared__ uint8_t smem_raw[];
@@ -2541,6 +2541,17 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
         const bool final = ROWS_OUT && desc[qb * 16 + 14] != 0;  // the outputs themselves (see Seg)
         const int32_t orow = rbase < 0 ? -1 : rbase / a.max_partitions;
         const float inv = l > 0.f ? 1.f / l : 0.f;
+        if constexpr (ROWS_OUT) {
+          // The first run of a lane that other runs continue lists its rows for the
+          // merge (which then covers those rows only).
+          if (!final && slot == 0 && merge_list != nullptr) {
+            const unsigned want = __ballot_sync(kFull, prow >= 0);
+            int first = 0;
+            if (lane == 0 && want) first = atomicAdd(merge_list, __popc(want));
+            first = __shfl_sync(kFull, first, 0);
+            if (prow >= 0) merge_list[1 + first + __popc(want & ((1u << lane) - 1u))] = orow;
+          }
+        }
         const uint32_t ocol = S::kOCol + 128u * (uint32_t)qb;
         constexpr int kTileStride = 20;  // floats
         float* tile = reinterpret_cast<float*>(base_ptr + S::kQOff + qb * S::kQBytes) + warp * 32 * kTileStride;
@@ -3064,7 +3075,8 @@ __global__ void __launch_bounds__(Tc05dShape<D, STAGES>::kThreads, 2)
 // partials, it waits for that grid before reading them.
 // ---------------------------------------------------------------------------
 template <typename T, int D, int WPI, int SPARSE>
-__global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel(const DecodeArgs a, int num_seqs) {
+__global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel(const DecodeArgs a, int num_seqs,
+                                                                                 const int32_t* list) {
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
   constexpr int VPL = D / 32;
   constexpr int NW = WPI > 4 ? WPI : 4;
@@ -3075,8 +3087,16 @@ __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int sub = warp % WPI;  // warp within its item
-  const int64_t item = (int64_t)blockIdx.x * IPC + warp / WPI;
-  const bool live = item < (int64_t)num_seqs * a.num_q_heads;
+  // `list` (optional): [0] = count, then the items to merge (the rows whose lane
+  // the balanced kernel split); otherwise every (sequence, query head) item.
+  const int64_t slot_i = (int64_t)blockIdx.x * IPC + warp / WPI;
+  int64_t item = slot_i;
+  bool live = item < (int64_t)num_seqs * a.num_q_heads;
+  if (list != nullptr) {
+    live = slot_i < (int64_t)list[0];
+    item = live ? (int64_t)list[1 + slot_i] : 0;
+    live = live && item >= 0 && item < (int64_t)num_seqs * a.num_q_heads;
+  }
   int np = 0;
   int64_t base = 0;
   if (live) {
@@ -3279,8 +3299,10 @@ __device__ __forceinline__ int verify_visible_partitions(int ctx, int num_tokens
 // sequence longer than one partition (`whole` = 1: the balanced kernel, which
 // applies each row's causal limit).
 __global__ void verify_plan_kernel(const DecodeArgs a, int num_seqs, int num_tokens, int per_chunk, int cps,
-                                   int whole, int32_t* __restrict__ chunks, int32_t* __restrict__ members) {
+                                   int whole, int32_t* __restrict__ chunks, int32_t* __restrict__ members,
+                                   int32_t* __restrict__ merge_list) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b == 0 && merge_list != nullptr) merge_list[0] = 0;  // the merge's item count
   if (b >= num_seqs) return;
   const int ctx = context_of(a, b, false);
   const int sp = whole ? (ctx > kPartition ? (ctx + 63) / 64 : 0) : verify_visible_partitions(ctx, num_tokens);
@@ -3982,7 +4004,8 @@ cudaError_t launch_shared_tc05d(const DecodeArgs& a, const CUtensorMap& mk, cons
 template <typename T, int D>
 cudaError_t launch_shared_seg(const DecodeArgs& a, pa_dtype dtype, int num_chunks, const int32_t* chunks,
                               const int32_t* members, int num_members, const int32_t* first_partition, int num_seqs,
-                              bool dependent, cudaStream_t stream, bool fold_tails = true, int verify_tokens = 0) {
+                              bool dependent, cudaStream_t stream, bool fold_tails = true, int verify_tokens = 0,
+                              int32_t* merge_list = nullptr) {
   constexpr int kStages = D == 128 ? 5 : 8;
   using S = SegShape<D, kStages>;
   static std::atomic<uint64_t> done[2] = {{0}, {0}};
@@ -4005,7 +4028,7 @@ cudaError_t launch_shared_seg(const DecodeArgs& a, pa_dtype dtype, int num_chunk
   // any other kernel it waits before its first read.
   return launch_pdl(kernel, dim3(sm_count()), dim3(S::kThreads), S::kSmemBytes, stream, true, a, mk, mv, tma_k,
                     chunks, num_chunks, members, num_members, first_partition, num_seqs, fold_tails ? 1 : 0,
-                    verify_tokens, dependent ? 0 : 1, (int)g_fault.load());
+                    verify_tokens, dependent ? 0 : 1, (int)g_fault.load(), merge_list);
 }
 
 std::atomic<int> g_shared_kernel{PA_SHARED_PREFIX_AUTO};
@@ -4082,28 +4105,34 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 template <typename T, int D, int SPARSE>
-cudaError_t launch_reduce_dim(const DecodeArgs& a, int num_seqs, cudaStream_t stream, bool dependent) {
-  const int64_t items = (int64_t)num_seqs * a.num_q_heads;
+cudaError_t launch_reduce_dim(const DecodeArgs& a, int num_seqs, cudaStream_t stream, bool dependent,
+                              const int32_t* list, int64_t list_cap) {
+  const int64_t items = list ? std::min<int64_t>(list_cap, (int64_t)num_seqs * a.num_q_heads)
+                             : (int64_t)num_seqs * a.num_q_heads;
   auto grid = [&](int ipc) { return dim3((unsigned)((items + ipc - 1) / ipc)); };
   // Warps per (sequence, query head), by partition count (an 8-warp form,
   // tried for more than 32 partitions, measured no faster).
   if (a.max_partitions <= 16)
-    return launch_pdl(decode_reduce_kernel<T, D, 1, SPARSE>, grid(4), dim3(128), 0, stream, dependent, a, num_seqs);
+    return launch_pdl(decode_reduce_kernel<T, D, 1, SPARSE>, grid(4), dim3(128), 0, stream, dependent, a, num_seqs,
+                      list);
   if (a.max_partitions <= 48)
-    return launch_pdl(decode_reduce_kernel<T, D, 2, SPARSE>, grid(2), dim3(128), 0, stream, dependent, a, num_seqs);
-  return launch_pdl(decode_reduce_kernel<T, D, 4, SPARSE>, grid(1), dim3(128), 0, stream, dependent, a, num_seqs);
+    return launch_pdl(decode_reduce_kernel<T, D, 2, SPARSE>, grid(2), dim3(128), 0, stream, dependent, a, num_seqs,
+                      list);
+  return launch_pdl(decode_reduce_kernel<T, D, 4, SPARSE>, grid(1), dim3(128), 0, stream, dependent, a, num_seqs,
+                    list);
 }
 
 template <typename T>
 cudaError_t launch_reduce(const DecodeArgs& a, int head_dim, int num_seqs, cudaStream_t stream,
-                          bool dependent = false, int sparse = 0) {
+                          bool dependent = false, int sparse = 0, const int32_t* list = nullptr,
+                          int64_t list_cap = 0) {
   if ((int64_t)num_seqs * a.num_q_heads > 0x7fffffffLL) return cudaErrorInvalidValue;
   // sparse: 0 every slot written; 1 empty slots marked l = 0; 2 also rows marked done
   auto pick = [&](auto d) -> cudaError_t {
     constexpr int Dv = decltype(d)::value;
-    if (sparse == 2) return launch_reduce_dim<T, Dv, 2>(a, num_seqs, stream, dependent);
-    if (sparse == 1) return launch_reduce_dim<T, Dv, 1>(a, num_seqs, stream, dependent);
-    return launch_reduce_dim<T, Dv, 0>(a, num_seqs, stream, dependent);
+    if (sparse == 2) return launch_reduce_dim<T, Dv, 2>(a, num_seqs, stream, dependent, list, list_cap);
+    if (sparse == 1) return launch_reduce_dim<T, Dv, 1>(a, num_seqs, stream, dependent, list, list_cap);
+    return launch_reduce_dim<T, Dv, 0>(a, num_seqs, stream, dependent, list, list_cap);
   };
   switch (head_dim) {
     case 64: return pick(std::integral_constant<int, 64>{});
@@ -4352,11 +4381,12 @@ pa_status launch_partitions(const DecodeArgs& a, pa_dtype dtype, int head_dim, i
 }
 
 pa_status launch_reduce_any(const DecodeArgs& a, pa_dtype dtype, int head_dim, int num_seqs, cudaStream_t s,
-                            bool dependent = false, int sparse = 0) {
+                            bool dependent = false, int sparse = 0, const int32_t* list = nullptr,
+                            int64_t list_cap = 0) {
   const cudaError_t err =
-      dtype == PA_F32    ? launch_reduce<float>(a, head_dim, num_seqs, s, dependent, sparse)
-      : dtype == PA_BF16 ? launch_reduce<__nv_bfloat16>(a, head_dim, num_seqs, s, dependent, sparse)
-                         : launch_reduce<__half>(a, head_dim, num_seqs, s, dependent, sparse);
+      dtype == PA_F32    ? launch_reduce<float>(a, head_dim, num_seqs, s, dependent, sparse, list, list_cap)
+      : dtype == PA_BF16 ? launch_reduce<__nv_bfloat16>(a, head_dim, num_seqs, s, dependent, sparse, list, list_cap)
+                         : launch_reduce<__half>(a, head_dim, num_seqs, s, dependent, sparse, list, list_cap);
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode reduce kernel: %s", cudaGetErrorString(err));
   return PA_OK;
 }
@@ -4444,7 +4474,7 @@ constexpr int kVerifyJointRows = 8;
 // chunks int32 [num_seqs * T][4] at most, members int32 [num_seqs * T].
 struct VerifyLayout {
   WorkspaceLayout parts;
-  size_t chunks_off, members_off, total;
+  size_t chunks_off, members_off, list_off, total;
 };
 
 VerifyLayout verify_layout(int64_t num_seqs, int64_t num_tokens, int64_t num_q_heads, int64_t head_dim,
@@ -4453,7 +4483,9 @@ VerifyLayout verify_layout(int64_t num_seqs, int64_t num_tokens, int64_t num_q_h
   v.parts = workspace_layout(num_seqs, num_tokens * num_q_heads, head_dim, partitions);
   v.chunks_off = v.parts.total;
   v.members_off = v.chunks_off + align256((size_t)num_seqs * num_tokens * 16);
-  v.total = v.members_off + align256((size_t)num_seqs * num_tokens * 4);
+  // the merge's item list: a count, then up to one entry per row
+  v.list_off = v.members_off + align256((size_t)num_seqs * num_tokens * 4);
+  v.total = v.list_off + align256((1 + (size_t)num_seqs * num_tokens * num_q_heads) * 4);
   return v;
 }
 }  // namespace
@@ -4517,6 +4549,7 @@ extern "C" pa_status pa_decode_verify(const void* q, const void* key_cache, cons
   const bool joint = joint_ok && (path == PA_VERIFY_JOINT ||
                                   (path == PA_VERIFY_AUTO && (int64_t)num_query_tokens * G > kVerifyJointRows));
   bool balanced = false;  // the balanced joint kernel ran (its merge skips the slots it leaves empty)
+  const int32_t* verify_merge_list = nullptr;  // with it: the rows its split lanes left to the merge
   if (joint) {
     const VerifyLayout lay = verify_layout(num_seqs, num_query_tokens, num_q_heads, head_dim, partitions);
     if (workspace_bytes < lay.total)
@@ -4524,6 +4557,8 @@ extern "C" pa_status pa_decode_verify(const void* q, const void* key_cache, cons
                   workspace_bytes);
     int32_t* chunks = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.chunks_off);
     int32_t* members = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.members_off);
+    int32_t* list = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.list_off);
+    verify_merge_list = list;
     const int cps = (num_query_tokens + per_chunk - 1) / per_chunk;
     const int num_members = num_seqs * num_query_tokens;
     // The balanced kernel takes every partition of the sequences longer than one
@@ -4537,7 +4572,8 @@ extern "C" pa_status pa_decode_verify(const void* q, const void* key_cache, cons
     balanced = (shared_choice == PA_SHARED_PREFIX_AUTO || shared_choice == PA_SHARED_PREFIX_TCGEN05) &&
                units < kSegMaxUnits;
     verify_plan_kernel<<<(num_seqs + 127) / 128, 128, 0, s>>>(a, num_seqs, num_query_tokens, per_chunk, cps,
-                                                                balanced ? 1 : 0, chunks, members);
+                                                                balanced ? 1 : 0, chunks, members,
+                                                                balanced ? list : nullptr);
     err = cudaGetLastError();
     if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode_verify plan kernel: %s", cudaGetErrorString(err));
     // The joint kernel indexes q, the partials and its members with H_q heads per member.
@@ -4550,14 +4586,14 @@ extern "C" pa_status pa_decode_verify(const void* q, const void* key_cache, cons
       const int T = num_query_tokens;
       err = head_dim == 64
                 ? (dtype == PA_BF16 ? launch_shared_seg<__nv_bfloat16, 64>(aj, dtype, nc, chunks, members, num_members,
-                                                                           nullptr, num_members, false, s, false, T)
+                                                                           nullptr, num_members, false, s, false, T, list)
                                     : launch_shared_seg<__half, 64>(aj, dtype, nc, chunks, members, num_members,
-                                                                    nullptr, num_members, false, s, false, T))
+                                                                    nullptr, num_members, false, s, false, T, list))
                 : (dtype == PA_BF16 ? launch_shared_seg<__nv_bfloat16, 128>(aj, dtype, nc, chunks, members,
                                                                             num_members, nullptr, num_members, false,
-                                                                            s, false, T)
+                                                                            s, false, T, list)
                                     : launch_shared_seg<__half, 128>(aj, dtype, nc, chunks, members, num_members,
-                                                                     nullptr, num_members, false, s, false, T));
+                                                                     nullptr, num_members, false, s, false, T, list));
     } else {
       const dim3 grid(num_seqs * cps, num_kv_heads, max_visible);
       err = dtype == PA_BF16 ? launch_shared_dim<__nv_bfloat16>(aj, head_dim, grid, chunks, members, num_members,
@@ -4577,7 +4613,14 @@ extern "C" pa_status pa_decode_verify(const void* q, const void* key_cache, cons
                              : launch_verify_cc<__half>(a, v, head_dim, num_seqs, partitions, s);
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode_verify partition kernel: %s", cudaGetErrorString(err));
   if (partitions <= 1) return PA_OK;
-  return launch_reduce_any(a, dtype, head_dim, num_seqs, s, /*dependent=*/true, /*sparse=*/balanced ? 2 : 0);
+  if (balanced) {
+    // Only the rows of the lanes the balanced kernel split need merging: at most
+    // one lane of at most PA_PREFIX_QUERIES_PER_CTA rows per CTA boundary.
+    const int64_t cap = (int64_t)(sm_count() + 1) * PA_PREFIX_QUERIES_PER_CTA;
+    return launch_reduce_any(a, dtype, head_dim, num_seqs, s, /*dependent=*/true, /*sparse=*/2,
+                             verify_merge_list, cap);
+  }
+  return launch_reduce_any(a, dtype, head_dim, num_seqs, s, /*dependent=*/true);
 }
 
 // ---------------------------------------------------------------------------
