@@ -79,6 +79,8 @@ struct DecodeArgs {
   const int32_t* first_partition;  // optional: partitions [0, first) of b come from the shared-prefix kernel
   int skip_members;                // with first_partition: sequences with first > 0 are left out entirely
   int partition_base;              // grid z of the partition kernels starts at this partition
+  int wait_first;                  // tensor-core kernel launched as a programmatic dependent: wait for the
+                                   // grid before it ahead of the first read
   int max_blocks_per_seq;
   int num_q_heads;
   int num_kv_heads;
@@ -291,6 +293,8 @@ __global__ void __launch_bounds__(NW * 32) decode_tc_kernel(const DecodeArgs a) 
   const AfterPrerequisiteGrid after{threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0};
   // A joint kernel launched after this one as a programmatic dependent may start now.
   if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  // Launched early after the step's cache write: nothing is read before that grid is done.
+  if (a.wait_first) asm volatile("griddepcontrol.wait;\n" ::: "memory");
   using S = TcShape<D, NW, STAGES>;
   constexpr int KSTEPS = D / 16;
   constexpr int MTILES = D / 16;
@@ -4406,7 +4410,10 @@ extern "C" pa_status pa_decode(const void* q, const void* key_cache, const void*
                                 workspace, workspace_bytes, dev_status, a, partitions);
   if (st != PA_OK || num_seqs == 0) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = launch_partitions(a, dtype, head_dim, num_seqs, partitions, s);
+  // The partition kernel, too, launches as a programmatic dependent of the kernel
+  // before it and waits for that grid before its first read.
+  a.wait_first = 1;
+  st = launch_partitions(a, dtype, head_dim, num_seqs, partitions, s, /*dependent=*/true);
   if (st != PA_OK || partitions <= 1) return st;
   // A programmatic dependent: its CTAs take the SMs the partition kernel's last
   // wave leaves idle and wait there for that grid to finish.
@@ -4426,7 +4433,9 @@ extern "C" pa_status pa_decode_partitions(const void* q, const void* key_cache, 
                                 num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, out, dtype,
                                 workspace, workspace_bytes, dev_status, a, partitions);
   if (st != PA_OK || num_seqs == 0) return st;
-  return launch_partitions(a, dtype, head_dim, num_seqs, partitions, static_cast<cudaStream_t>(stream));
+  a.wait_first = 1;  // a programmatic dependent of the kernel before it (see pa_decode)
+  return launch_partitions(a, dtype, head_dim, num_seqs, partitions, static_cast<cudaStream_t>(stream),
+                           /*dependent=*/true);
 }
 
 extern "C" pa_status pa_decode_reduce(const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
