@@ -235,8 +235,9 @@ PA_API pa_status pa_decode_reduce(const int32_t* context_lens, int32_t num_seqs,
  *                 with num_query_tokens * num_q_heads query heads per
  *                 sequence (m_part may sit up to 8 ln 2 below the
  *                 partition's maximum score), then room for the joint
- *                 kernel's work plan (20 bytes per query token, each array
- *                 256-byte aligned).
+ *                 kernel's work plan (20 bytes per query token) and the
+ *                 merge's item list (4 bytes per query row plus a count),
+ *                 each array 256-byte aligned.
  * Everything else, including the supported sizes, the device status bits
  * and the error returns, is as for pa_decode; in addition
  * num_query_tokens >= 1 and num_query_tokens * num_q_heads <= 2^24.

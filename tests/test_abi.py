@@ -75,15 +75,17 @@ def test_device_calls_reject_cpu_tensors():
 
 
 def test_verify_workspace_size_matches_documented_layout():
-    """The pa_decode partials with T * H_q heads per sequence, then the joint kernel's plan arrays."""
+    """The pa_decode partials with T * H_q heads per sequence, then the joint kernel's plan arrays and
+    the merge's item list (a count, then one int32 per query row)."""
     align = lambda x: (x + 255) // 256 * 256  # noqa: E731
     assert binding.pa_decode_verify_workspace_size(4, 3, 8, 128, 512) == 0          # one partition
     assert binding.pa_decode_verify_workspace_size(4, 0, 8, 128, 4096) == 0         # no query token
     b, t, hq, d, ctx = 256, 4, 64, 128, 8192
     parts = binding.pa_decode_workspace_size(b, t * hq, d, ctx)
-    assert binding.pa_decode_verify_workspace_size(b, t, hq, d, ctx) == parts + align(16 * b * t) + align(4 * b * t)
+    assert binding.pa_decode_verify_workspace_size(b, t, hq, d, ctx) == (
+        parts + align(16 * b * t) + align(4 * b * t) + align(4 * (1 + b * t * hq)))
     assert binding.pa_decode_verify_workspace_size(3, 7, 5, 64, 1025) == (
-        binding.pa_decode_workspace_size(3, 35, 64, 1025) + align(16 * 21) + align(4 * 21))
+        binding.pa_decode_workspace_size(3, 35, 64, 1025) + align(16 * 21) + align(4 * 21) + align(4 * (1 + 21 * 5)))
 
 
 def test_verify_and_pool_setters_validate_on_the_host():
