@@ -199,7 +199,10 @@ PA_API pa_status pa_decode(const void* q, const void* key_cache, const void* val
  * pa_decode_partitions writes the output rows of one-partition sequences and
  * the workspace partials of the others; pa_decode_reduce merges those
  * partials into their output rows (max_context_len = max_blocks_per_seq *
- * block_size of the partition call) and leaves the other rows untouched. */
+ * block_size of the partition call) and leaves the other rows untouched.
+ * Both kernels launch as programmatic dependents of the kernel before them on
+ * the stream (so that their CTAs are resident when it ends) and wait for that
+ * grid to finish before their first read: stream order is kept. */
 PA_API pa_status pa_decode_partitions(const void* q, const void* key_cache, const void* value_cache,
                                       const int32_t* block_tables, int32_t max_blocks_per_seq,
                                       const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
