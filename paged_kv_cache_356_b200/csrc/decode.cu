@@ -2152,7 +2152,16 @@ __global__ void __launch_bounds__(SegShape<D, STAGES>::kThreads, 1)
     // Launched as a programmatic dependent of an arbitrary kernel: nothing is read
     // before that grid has finished (its launch and the set-up below overlap it).
     // Every global write of this grid follows a producer's load, hence this wait.
-    if (wait_at_start) asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    if (wait_at_start) {
+      // The plan and the lengths into L2 meanwhile (a prefetch returns nothing to
+      // the thread, and L2 holds any later write of the grid before, so this is
+      // safe whatever that grid writes): the walk's first loads then hit L2.
+      const int32_t* arr = pw == 0 ? chunks : pw == 1 ? members : pw == 2 ? first_partition : a.context_lens;
+      const int64_t words = pw == 0 ? 4 * (int64_t)num_chunks : pw == 1 ? num_members : num_seqs;
+      if (arr != nullptr && 32 * (int64_t)lane < words)
+        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(arr + 32 * (int64_t)lane));
+      asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    }
     seg_walk_init<E>(walk, a, chunks, num_chunks, members, num_members, first_partition, num_seqs, fold_tails != 0,
                      verify_tokens, pw == 0 && lane == 0 && blockIdx.x == 0);
     have = next_seg(seg);
