@@ -60,3 +60,19 @@ def test_fragmentation_rows_match_the_oracle_and_the_pages_bound():
     assert all(r["paged_waste_fraction"] < 0.04 < r["contiguous_waste_fraction"] for r in ind)
     beam = [r for r in rows if r["workload"] == "beam32k"]
     assert all(r["shared_pages"] > 0 and r["contiguous_over_paged_slots"] > 5 for r in beam)
+
+
+def test_call_bytes_count_inputs_and_outputs_once():
+    """A whole call's algorithmic bytes: unique KV + q + the tables' used entries + lengths + every
+    output row once, with T query tokens per sequence; the partition kernel's own figure adds the
+    partials it writes (and writes the rows of one-partition sequences directly)."""
+    w = workloads.tiny()                      # 2 sequences of 36 and 42 tokens, 4 q / 1 kv heads, D 64, fp32
+    ctx = np.array(w.context_lens)
+    unique = 1234
+    eb, rows_per_seq = w.elem_bytes, w.num_q_heads
+    tables = 4 * sum(-(-int(c) // w.block_size) for c in ctx)
+    for T in (1, 3):
+        want = unique + 2 * (2 * T * rows_per_seq * w.head_dim * eb) + tables + 4 * w.num_seqs
+        assert bench.call_bytes(w, ctx, unique, T) == want
+    # both sequences fit one partition: the partition kernel writes their rows, no partials
+    assert bench.partition_kernel_bytes(w, ctx, unique) == bench.call_bytes(w, ctx, unique, 1)
