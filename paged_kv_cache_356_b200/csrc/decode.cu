@@ -3223,21 +3223,16 @@ __global__ void __launch_bounds__(WPI > 4 ? 32 * WPI : 128) decode_reduce_kernel
       }
       const int cnt = min(32, (np - p0 + WPI - 1) / WPI);
       if (c > 0) load_rows(x, p0, 0, cnt);
+      // One batch of UNROLL rows at a time, the next requested once this one is
+      // added (no second buffer: fewer registers, more warps per SM, which is
+      // what this latency-bound kernel needs).
       for (int k = 0; k < cnt; k += UNROLL) {
-        float xn[UNROLL][VPL];
-        const bool more = k + UNROLL < cnt;
-        if (more) load_rows(xn, p0, k + UNROLL, cnt);
+        if (k > 0) load_rows(x, p0, k, cnt);
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
           const float wk = __shfl_sync(kFull, wt, min(k + u, 31));
 #pragma unroll
           for (int i = 0; i < VPL; ++i) acc[i] = fmaf(k + u < cnt ? wk : 0.f, x[u][i], acc[i]);
-        }
-        if (more) {
-#pragma unroll
-          for (int u = 0; u < UNROLL; ++u)
-#pragma unroll
-            for (int i = 0; i < VPL; ++i) x[u][i] = xn[u][i];
         }
       }
     }
